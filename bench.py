@@ -1,0 +1,408 @@
+"""Benchmark of the MoE-layer forward pass on B200: tokens/s and active
+TFLOP/s, with the dominant kernel's roofline fraction, the end-to-end number
+through the host API and the fp64 oracle timed on the host cores.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   (the fp64 CPU oracle, timed alone)
+
+N > 1 runs under torchrun: every rank processes its own batch of tokens with
+the same (replicated) weights and no collective on the data path (weak
+scaling); the timed region is bracketed by barriers and the max over ranks is
+reported. Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from sparse_mixture_experts_renorm_b200.workloads import WORKLOADS, make_inputs, make_tokens  # noqa: E402
+
+METRIC = "MoE-layer tokens/s and TFLOP/s (active) at 1 B200; % of bf16 TC / HBM roofline"
+KERNELS = ["router_topk", "route_scan", "permute", "grouped_gemm_gateup_swiglu", "grouped_gemm_down", "combine"]
+KERNEL_SOURCES = {
+    "router_topk": "router.cu", "route_scan": "router.cu", "permute": "permute.cu", "combine": "permute.cu",
+    "grouped_gemm_gateup_swiglu": "gemm_tc.cu", "grouped_gemm_down": "gemm_tc.cu",
+}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(kernel):
+    src = os.path.join(ROOT, "sparse_mixture_experts_renorm_b200", "csrc", KERNEL_SOURCES[kernel])
+    with open(src, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def load_traffic(workload, kernel):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current source of that kernel."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        table = json.load(f)
+    ent = table.get(workload, {}).get(kernel)
+    if not ent or ent.get("source_sha") != source_hash(kernel):
+        return None
+    return ent.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------ algorithmic work
+
+def algorithmic(wl, counts):
+    """Algorithmic FLOPs and DRAM bytes per launch of each kernel (the minimum
+    traffic: every input read once, every output written once)."""
+    T, d, E, k, I = wl.T, wl.d, wl.E, wl.k, wl.I
+    R = T * k
+    el = 2 if wl.dtype == "bf16" else 4
+    used = int((np.asarray(counts) > 0).sum())
+    nb = (T + 31) // 32
+    return {
+        "router_topk": dict(flops=2.0 * T * d * E, bytes=T * d * el + E * d * el + T * k * 12 + nb * E * 8),
+        "route_scan": dict(flops=0.0, bytes=nb * E * 12 + (E + 1) * 8 + E * 4),
+        "permute": dict(flops=0.0, bytes=T * d * el + R * d * el + R * 12),
+        "grouped_gemm_gateup_swiglu": dict(flops=4.0 * R * d * I,
+                                           bytes=2 * used * I * d * el + R * d * el + R * I * el),
+        "grouped_gemm_down": dict(flops=2.0 * R * d * I, bytes=used * d * I * el + R * I * el + R * d * 4),
+        "combine": dict(flops=2.0 * R * d, bytes=R * d * 4 + T * d * 4 + R * 8),
+    }
+
+
+# --------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.path = None
+        try:
+            props = torch.cuda.get_device_properties(device)
+            bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+        except Exception:
+            bus = None
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader", "-lms", "200"]
+        if bus:
+            cmd += ["-i", bus]
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                except Exception:
+                    ts = None
+                rows.append((ts, parts))
+        sel = [p for ts, p in rows if ts is not None and t0 - 1.0 <= ts <= t1 + 1.0] or [p for _, p in rows]
+        for parts in sel:
+            try:
+                sm.append(float(parts[2].split()[0]))
+                smax.append(float(parts[3].split()[0]))
+                power.append(float(parts[4].split()[0]))
+            except Exception:
+                pass
+            for nm, v in zip(names, parts[6:10]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sel),
+                "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def cpu_oracle_rate(inp_cpu, wl, budget_s, max_tokens=None):
+    """Whole-layer fp64 oracle on the first n tokens: (tokens/s, n, seconds,
+    threads). n is calibrated on one token to take about budget_s."""
+    import oracle
+
+    threads = len(os.sched_getaffinity(0))
+    oracle.set_num_threads(threads)
+
+    def run(n):
+        x = inp_cpu.x[:n]
+        t0 = time.perf_counter()
+        oracle.forward(x, inp_cpu.w_router, inp_cpu.b_router, inp_cpu.w_gate, inp_cpu.w_up, inp_cpu.w_down, wl.k,
+                       wl.renorm)
+        return time.perf_counter() - t0
+
+    t1 = run(1)
+    n = int(max(1, min(wl.T if max_tokens is None else max_tokens, budget_s / max(t1, 1e-6))))
+    dt = run(n)
+    return n / dt, n, dt, threads
+
+
+def inputs_to_cpu(inp):
+    from sparse_mixture_experts_renorm_b200.workloads import Inputs
+
+    c = lambda t: None if t is None else t.detach().to("cpu")  # noqa: E731
+    return Inputs(inp.wl, c(inp.x), c(inp.w_router), c(inp.b_router), c(inp.w_gate), c(inp.w_up), c(inp.w_down))
+
+
+# ------------------------------------------------------------------- reference
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = inputs_to_cpu(make_inputs(wl, dev, seed=0))
+    threads = len(os.sched_getaffinity(0))
+    # each step: the whole layer on a bounded contiguous sample of the batch
+    per_step_budget = float(os.environ.get("MOE_REF_STEP_S", "3.0"))
+    _, n, _, _ = cpu_oracle_rate(inp, wl, per_step_budget)
+    import oracle
+
+    oracle.set_num_threads(threads)
+
+    def step(i):
+        lo = (i * n) % max(1, wl.T - n + 1)
+        x = inp.x[lo:lo + n]
+        oracle.forward(x, inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k, wl.renorm)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    tok_s = n * args.steps / dt
+    sample = f"{n} of {wl.T} tokens per step (router, top-k, statistics, dispatch, experts, combine in fp64)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "tflops_active": wl.active_flops / wl.T * tok_s / 1e12,
+        "config": config_of(wl, args.gpus),
+        "cpu_baseline": {"value": tok_s, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": tok_s, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(wl, n_gpus):
+    return {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "I": wl.I, "renorm": wl.renorm,
+            "router_bias": "zipf" if wl.zipf_bias else None, "global_batch_tokens": wl.T * n_gpus,
+            "parallelism": f"dp{n_gpus} (replicated weights, independent token batches, no collective)",
+            "l2": "inputs larger than L2: every step streams all expert weights "
+                  f"({3 * wl.E * wl.d * wl.I * (2 if wl.dtype == 'bf16' else 4) / 1e9:.2f} GB) through HBM"}
+
+
+# ------------------------------------------------------------------------ ours
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mixtral_prefill", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    wl = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        return run_reference(args, wl)
+
+    import torch.distributed as dist
+
+    from sparse_mixture_experts_renorm_b200 import MoELayer
+    from sparse_mixture_experts_renorm_b200 import _binding as B
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    inp = make_inputs(wl, dev, seed=0)  # same weights on every rank
+    x = make_tokens(wl, wl.T, dev, seed=1000 + rank) if world > 1 else inp.x
+    layer = MoELayer(inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k, wl.renorm, wl.T)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        layer(x)
+    torch.cuda.synchronize()
+    status = int(layer.status.item())
+    if status:
+        raise RuntimeError(f"device status word {status:#x} after warm-up")
+
+    nk = B.MOE_NUM_KERNELS
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
+    for row in evs:  # create the events outside the timed region
+        for ev in row:
+            ev.record(stream)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev)
+    time.sleep(0.3)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        layer(x, events=evs[i])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    clocks = sampler.stop(t_wall0, t_wall1)
+    ms = start.elapsed_time(stop)
+    per_kernel = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(nk)] for i in range(args.steps)])
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    status = int(layer.status.item())
+    if status:
+        raise RuntimeError(f"device status word {status:#x} after the timed region")
+
+    # ---- end to end through the host API: pinned x in, out + aux back
+    e2e_steps = max(1, min(args.steps, 50))
+    x_host = x.detach().to("cpu").pin_memory()
+    out_host = torch.empty((wl.T, wl.d), dtype=torch.float32).pin_memory()
+    aux_host = torch.empty((1,), dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(x)
+    for _ in range(2):
+        layer.forward_host(x_host, out_host, aux_host, x_dev)
+    torch.cuda.synchronize()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    s2.record(stream)
+    for _ in range(e2e_steps):
+        layer.forward_host(x_host, out_host, aux_host, x_dev)
+    e2.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = s2.elapsed_time(e2)
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+
+    counts = layer.counts.cpu().numpy()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    tokens = wl.T * world * args.steps
+    tok_s = tokens / (ms / 1e3)
+    tflops = wl.active_flops * world * args.steps / (ms / 1e3) / 1e12
+    peaks, peak_src = load_peaks()
+    region_s = ms / 1e3
+    sustained = region_s >= 1.0
+    tc_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    hbm_peak = peaks["hbm_gbs"]
+    work = algorithmic(wl, counts)
+    avg = per_kernel.mean(axis=0)
+    kern = []
+    for j, name in enumerate(KERNELS):
+        w = work[name]
+        t_s = avg[j] / 1e3
+        ent = {"name": name, "avg_us": float(avg[j] * 1e3), "share": float(avg[j] / avg.sum()),
+               "tflops": w["flops"] / t_s / 1e12 if t_s > 0 else None,
+               "gbs": w["bytes"] / t_s / 1e9 if t_s > 0 else None}
+        kern.append(ent)
+    dom = int(np.argmax(avg))
+    dname = KERNELS[dom]
+    w = work[dname]
+    t_dom = avg[dom] / 1e3
+    # which roof binds this kernel at its algorithmic work
+    tensor_bound = (w["flops"] / (tc_peak * 1e12)) >= (w["bytes"] / (hbm_peak * 1e9)) and wl.dtype == "bf16"
+    if tensor_bound:
+        achieved = w["flops"] / t_dom / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": achieved / tc_peak}
+    else:
+        achieved = w["bytes"] / t_dom / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak}
+    roof["kernel"] = dname
+    roof["traffic"] = load_traffic(wl.name, dname)
+    roof["peak_source"] = (f"{peak_src} ({'sustained' if sustained and tensor_bound else 'burst'}"
+                           f"{' bf16' if tensor_bound else ' HBM copy'})")
+    roof["algorithmic_per_launch"] = w["flops"] if tensor_bound else w["bytes"]
+
+    line = {
+        "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded, random-init weights)",
+        "tflops_active": tflops,
+        "config": config_of(wl, world),
+        "roofline": roof,
+        "kernels": kern,
+        "e2e": {"value": wl.T * world * e2e_steps / (ms_e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x.numel() * x.element_size()),
+                "d2h_bytes_per_step": int(wl.T * wl.d * 4 + 4)},
+        "gpu_launches": nk * args.steps,
+        "clocks": clocks,
+        "counts": counts.tolist() if wl.E <= 16 else {"max": int(counts.max()), "min": int(counts.min()),
+                                                      "mean": float(counts.mean())},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        inp_cpu = inputs_to_cpu(inp)
+        rate, n, dt, threads = cpu_oracle_rate(inp_cpu, wl, args.cpu_budget_s)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": f"first {n} of {wl.T} tokens, whole layer in fp64, {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,166 @@
+/*
+ * moe.h — C ABI of the B200 (sm_100a) sparse top-k Mixture-of-Experts
+ * forward pass.
+ *
+ * The layer (axonml-nn layers/moe.rs: MoERouter::route, Expert::forward,
+ * MoELayer::forward, load_balancing_loss, expert_utilization; Mixtral MoE
+ * Block, exported PyTorch _moe_forward; Model Architecture Patterns,
+ * "Top-K Router" and "SwiGLU FFN"):
+ *
+ *   p[t,:]      = softmax_e( x[t,:] . W_r[e,:] + b[e] )
+ *   idx[t,:]    = the k largest p[t,e], ordered by p descending and, among
+ *                 equal p, by expert index ascending
+ *   gate[t,j]   = p[t,idx[t,j]] / sum_j' p[t,idx[t,j']]   (renorm = 1)
+ *               = p[t,idx[t,j]]                            (renorm = 0)
+ *   y_e(x)      = W_down[e] ( SiLU(W_gate[e] x) * (W_up[e] x) ),
+ *                 SiLU(z) = z / (1 + exp(-z))
+ *   out[t,:]    = sum_j gate[t,j] * y_{idx[t,j]}(x[t,:])
+ *   counts[e]   = #{(t,j) : idx[t,j] = e}
+ *   aux         = E * sum_e (counts[e] / (T*k)) * (sum_t p[t,e] / T)
+ *
+ * Conventions for every entry point:
+ *   - All tensors are row-major and contiguous. Weights use the nn.Linear
+ *     [out, in] layout, stacked per expert ("packed experts", KempnerForge
+ *     ModelConfig.moe_packed_experts): W_router [E, d], W_gate [E, I, d],
+ *     W_up [E, I, d], W_down [E, d, I].
+ *   - Pointers documented as "device" must be CUDA device (or managed)
+ *     memory on the current device; the caller owns every buffer. The
+ *     library allocates no device memory: all scratch lives in the caller's
+ *     workspace.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Calls are
+ *     asynchronous on it and never synchronise the host.
+ *   - Argument errors are returned synchronously before anything is
+ *     launched; moe_last_error_detail() then gives a one-line reason.
+ *     Errors detected on the device (a bounded wait that gave up, a
+ *     non-finite router logit) are OR-ed into the caller's device status word
+ *     as MOE_DEV_* bits, to be read after the stream is synchronised.
+ *   - Nothing aborts the process.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* NULL required pointer, T < 0, k < 1, k > E, d/I/E <= 0 */
+  MOE_ERR_UNSUPPORTED = 2, /* valid layer, but outside what the kernels take (see below) */
+  MOE_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed */
+  MOE_ERR_WORKSPACE = 6    /* workspace NULL or smaller than moe_workspace_size() */
+} moe_status;
+
+/* Bits of the device status word. */
+#define MOE_DEV_TIMEOUT 0x1   /* a bounded wait inside a kernel gave up; outputs are invalid */
+#define MOE_DEV_NONFINITE 0x2 /* a router logit was NaN or infinite; that token's outputs are undefined */
+#define MOE_DEV_INTERNAL 0x4  /* an internal consistency check failed (a dispatched row out of range);
+                                 the offending access was skipped and the outputs are invalid */
+
+typedef enum {
+  MOE_F32 = 0, /* x and all weights fp32; every product accumulated in fp32 (SIMT FFMA) */
+  MOE_BF16 = 1 /* x and all weights bf16; fp32 accumulation; SwiGLU hidden stored as bf16 */
+} moe_dtype;
+
+/*
+ * Limits (MOE_ERR_UNSUPPORTED beyond them):
+ *   E <= 256, k <= 8, T*k < 2^31, d*I < 2^31 per expert;
+ *   MOE_BF16: d % 64 == 0 and I % 64 == 0 (128-byte TMA rows);
+ *   MOE_F32 : d % 4 == 0 (16-byte rows).
+ */
+
+/*
+ * moe_workspace_size — bytes of device scratch moe_forward needs for this
+ * shape. Returns 0 if the shape is invalid or unsupported (see
+ * moe_last_error_detail). The workspace holds the per-block routing
+ * partials, the dispatch order, the expert-contiguous copy of x, the SwiGLU
+ * hidden activations [T*k, I] and the fp32 expert outputs [T*k, d].
+ */
+size_t moe_workspace_size(int T, int d, int E, int k, int I, moe_dtype dtype);
+
+/*
+ * moe_forward — the whole layer on one GPU.
+ *
+ *   x          device, [T, d], dtype
+ *   w_router   device, [E, d], dtype (router Linear, no bias)
+ *   b_router   device, [E] fp32, or NULL: per-expert logit bias added before
+ *              the softmax (the skewed-load workload's bias)
+ *   w_gate     device, [E, I, d], dtype
+ *   w_up       device, [E, I, d], dtype
+ *   w_down     device, [E, d, I], dtype
+ *   renorm     1: gates renormalised over the k selected experts (1/k each
+ *              if their sum is not positive); 0: raw top-k probabilities
+ *   out        device, [T, d] fp32 — written, never read
+ *   topk_idx   device, [T, k] int32 — selected experts, best first
+ *   topk_gate  device, [T, k] fp32 — their gates
+ *   counts     device, [E] int32, or NULL — assignments per expert
+ *   aux        device, [1] fp32, or NULL — load-balancing statistic
+ *   workspace  device, at least moe_workspace_size() bytes, 256-byte aligned
+ *   status_dev device, [1] int32, or NULL — MOE_DEV_* bits are OR-ed in; the
+ *              caller clears it. NULL: the library keeps its own word in the
+ *              workspace (cleared each call).
+ *
+ * T = 0 is valid: counts are zeroed and aux is set to 0 (axonml-nn moe.rs,
+ * load_balancing_loss returns zero when there are no tokens).
+ * Results are deterministic: the same inputs give bit-identical outputs.
+ */
+moe_status moe_forward(const void* x, const void* w_router, const float* b_router,
+                       const void* w_gate, const void* w_up, const void* w_down,
+                       int T, int d, int E, int k, int I, int renorm, moe_dtype dtype,
+                       float* out, int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                       float* aux, void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                       void* stream);
+
+/*
+ * Kernels of one moe_forward, in launch order (both dtypes):
+ *   0 router_topk, 1 route_scan, 2 permute, 3 grouped_gemm_gateup_swiglu,
+ *   4 grouped_gemm_down, 5 combine.
+ * moe_kernel_name(i) returns the name (a static string; NULL out of range).
+ */
+#define MOE_NUM_KERNELS 6
+const char* moe_kernel_name(int i);
+
+/*
+ * moe_forward_events — moe_forward, plus per-kernel timing marks: events[i]
+ * (a cudaEvent_t created by the caller) is recorded on `stream` just before
+ * kernel i is launched and events[MOE_NUM_KERNELS] after the last one, so
+ * cudaEventElapsedTime(events[i], events[i+1]) is kernel i's device time.
+ * n_events must be at least MOE_NUM_KERNELS + 1. With T = 0 no kernel runs
+ * and no event is recorded. Same results as moe_forward.
+ */
+moe_status moe_forward_events(const void* x, const void* w_router, const float* b_router,
+                              const void* w_gate, const void* w_up, const void* w_down,
+                              int T, int d, int E, int k, int I, int renorm, moe_dtype dtype,
+                              float* out, int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                              float* aux, void* workspace, size_t workspace_bytes,
+                              int32_t* status_dev, void* stream, void* const* events, int n_events);
+
+/*
+ * moe_get_permutation — copy out the dispatch order that the last
+ * moe_forward on this workspace (same shape arguments) produced
+ * (axonml-nn moe.rs, MoELayer::forward: rows grouped by expert in ascending
+ * expert order, tokens ascending within an expert):
+ *   offsets  device, [E+1] int32 — first dispatched row of each expert
+ *   perm_tok device, [T*k] int32 — token of each dispatched row
+ *   inv      device, [T, k] int32 — dispatched row of each (token, slot)
+ * Any of the three may be NULL. Enqueued on `stream`.
+ */
+moe_status moe_get_permutation(const void* workspace, size_t workspace_bytes, int T, int d, int E,
+                               int k, int I, moe_dtype dtype, int32_t* offsets, int32_t* perm_tok,
+                               int32_t* inv, void* stream);
+
+/*
+ * moe_last_error_detail — the reason for the calling thread's last non-OK
+ * status, NUL-terminated into buf (truncated to n bytes). Returns the full
+ * length of the message.
+ */
+size_t moe_last_error_detail(char* buf, size_t n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

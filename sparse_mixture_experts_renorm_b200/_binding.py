@@ -1,0 +1,87 @@
+"""ctypes binding of ``libmoe_b200.so`` (the C ABI in ``include/moe.h``).
+
+Argument marshalling only: every step of the forward pass runs in the
+library's CUDA kernels. torch is used for device memory and the current
+stream. There is no fallback: if the library or a GPU is missing, the calls
+raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe_b200.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_WORKSPACE = 0, 1, 2, 3, 6
+MOE_DEV_TIMEOUT, MOE_DEV_NONFINITE, MOE_DEV_INTERNAL = 0x1, 0x2, 0x4
+MOE_F32, MOE_BF16 = 0, 1
+
+STATUS_NAMES = {
+    MOE_OK: "MOE_OK",
+    MOE_ERR_INVALID_ARG: "MOE_ERR_INVALID_ARG",
+    MOE_ERR_UNSUPPORTED: "MOE_ERR_UNSUPPORTED",
+    MOE_ERR_CUDA: "MOE_ERR_CUDA",
+    MOE_ERR_WORKSPACE: "MOE_ERR_WORKSPACE",
+}
+
+EXPORTED = ("moe_workspace_size", "moe_forward", "moe_forward_events", "moe_kernel_name", "moe_get_permutation",
+            "moe_last_error_detail")
+MOE_NUM_KERNELS = 6
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {detail}")
+        self.status = status
+        self.detail = detail
+
+
+_lib = None
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load the CUDA library (once). Raises if it has not been built."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(
+            f"{p} is missing: build it with `python -m sparse_mixture_experts_renorm_b200.build` "
+            "(there is no non-CUDA fallback)"
+        )
+    lib = ctypes.CDLL(p)
+    P, I32, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.moe_workspace_size.argtypes = [I32, I32, I32, I32, I32, I32]
+    lib.moe_workspace_size.restype = SZ
+    lib.moe_forward.argtypes = [P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, P, P, P, P, P, P, SZ, P, P]
+    lib.moe_forward.restype = I32
+    lib.moe_forward_events.argtypes = lib.moe_forward.argtypes + [ctypes.POINTER(ctypes.c_void_p), I32]
+    lib.moe_forward_events.restype = I32
+    lib.moe_kernel_name.argtypes = [I32]
+    lib.moe_kernel_name.restype = ctypes.c_char_p
+    lib.moe_get_permutation.argtypes = [P, SZ, I32, I32, I32, I32, I32, I32, P, P, P, P]
+    lib.moe_get_permutation.restype = I32
+    lib.moe_last_error_detail.argtypes = [ctypes.c_char_p, SZ]
+    lib.moe_last_error_detail.restype = SZ
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def last_error_detail(lib=None) -> str:
+    lib = lib or load_library()
+    buf = ctypes.create_string_buffer(1024)
+    lib.moe_last_error_detail(buf, len(buf))
+    return buf.value.decode()
+
+
+def kernel_names(lib=None) -> list[str]:
+    lib = lib or load_library()
+    return [lib.moe_kernel_name(i).decode() for i in range(MOE_NUM_KERNELS)]
+
+
+def check(status: int, lib=None) -> None:
+    if status != MOE_OK:
+        raise MoEError(status, last_error_detail(lib))

@@ -1,0 +1,122 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point declared in include/moe.h, sizes its workspace, and
+rejects bad arguments with the documented status before launching anything
+(the validation rules of KempnerForge's ModelConfig.__post_init__ and of
+axonml-nn's MoERouter::new: top_k > 0, top_k <= num_experts, positive dims)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_mixture_experts_renorm_b200 import _binding as B
+from sparse_mixture_experts_renorm_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.load_library()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "moe.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:size_t|moe_status|const char\s*\*)\s*(moe_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    assert set(B.EXPORTED) <= set(header_functions())
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_kernel_names(lib):
+    names = B.kernel_names(lib)
+    assert names[0] == "router_topk" and names[-1] == "combine" and len(names) == B.MOE_NUM_KERNELS
+    assert lib.moe_kernel_name(B.MOE_NUM_KERNELS) is None
+
+
+def test_forward_events_needs_events(lib):
+    fake = ctypes.c_void_p(4096)
+    arr = (ctypes.c_void_p * 3)()
+    st = lib.moe_forward_events(fake, fake, None, fake, fake, fake, 8, 128, 4, 2, 256, 1, B.MOE_F32, fake, fake, fake,
+                                None, None, fake, 1 << 40, None, None, arr, 3)
+    assert st == B.MOE_ERR_INVALID_ARG
+
+
+def test_workspace_size(lib):
+    n = lib.moe_workspace_size(4096, 4096, 8, 2, 14336, B.MOE_BF16)
+    R = 4096 * 2
+    # at least the expert-contiguous x, the hidden activations and the fp32 expert outputs
+    assert n >= R * 4096 * 2 + R * 14336 * 2 + R * 4096 * 4
+    assert n < R * 4096 * 2 + R * 14336 * 2 + R * 4096 * 4 + 64 * 1024 * 1024
+    assert lib.moe_workspace_size(0, 128, 4, 2, 256, B.MOE_F32) > 0
+
+
+@pytest.mark.parametrize("T,d,E,k,I,dt,expect", [
+    (-1, 128, 4, 2, 256, B.MOE_F32, B.MOE_ERR_INVALID_ARG),
+    (8, 0, 4, 2, 256, B.MOE_F32, B.MOE_ERR_INVALID_ARG),
+    (8, 128, 0, 1, 256, B.MOE_F32, B.MOE_ERR_INVALID_ARG),
+    (8, 128, 4, 0, 256, B.MOE_F32, B.MOE_ERR_INVALID_ARG),
+    (8, 128, 4, 5, 256, B.MOE_F32, B.MOE_ERR_INVALID_ARG),
+    (8, 128, 4, 2, 0, B.MOE_F32, B.MOE_ERR_INVALID_ARG),
+    (8, 128, 4, 2, 256, 7, B.MOE_ERR_INVALID_ARG),
+    (8, 128, 300, 2, 256, B.MOE_F32, B.MOE_ERR_UNSUPPORTED),
+    (8, 128, 16, 9, 256, B.MOE_F32, B.MOE_ERR_UNSUPPORTED),
+    (8, 96, 4, 2, 256, B.MOE_BF16, B.MOE_ERR_UNSUPPORTED),
+    (8, 128, 4, 2, 200, B.MOE_BF16, B.MOE_ERR_UNSUPPORTED),
+    (8, 130, 4, 2, 256, B.MOE_F32, B.MOE_ERR_UNSUPPORTED),
+])
+def test_shape_validation(lib, T, d, E, k, I, dt, expect):
+    assert lib.moe_workspace_size(T, d, E, k, I, dt) == 0
+    fake = ctypes.c_void_p(4096)  # never dereferenced: validation fails first
+    st = lib.moe_forward(fake, fake, None, fake, fake, fake, T, d, E, k, I, 1, dt, fake, fake, fake, None, None,
+                         fake, 1 << 40, None, None)
+    assert st == expect
+    assert len(B.last_error_detail(lib)) > 0
+
+
+def test_null_pointers_and_workspace(lib):
+    fake = ctypes.c_void_p(4096)
+    args = dict(T=8, d=128, E=4, k=2, I=256)
+    st = lib.moe_forward(None, fake, None, fake, fake, fake, 8, 128, 4, 2, 256, 1, B.MOE_F32, fake, fake, fake, None,
+                         None, fake, 1 << 40, None, None)
+    assert st == B.MOE_ERR_INVALID_ARG
+    assert "NULL" in B.last_error_detail(lib)
+    need = lib.moe_workspace_size(*args.values(), B.MOE_F32)
+    st = lib.moe_forward(fake, fake, None, fake, fake, fake, 8, 128, 4, 2, 256, 1, B.MOE_F32, fake, fake, fake, None,
+                         None, fake, need - 1, None, None)
+    assert st == B.MOE_ERR_WORKSPACE
+    st = lib.moe_forward(fake, fake, None, fake, fake, fake, 8, 128, 4, 2, 256, 1, B.MOE_F32, fake, fake, fake, None,
+                         None, None, need, None, None)
+    assert st == B.MOE_ERR_WORKSPACE
+    st = lib.moe_forward(fake, fake, None, fake, fake, fake, 8, 128, 4, 2, 256, 2, B.MOE_F32, fake, fake, fake, None,
+                         None, fake, need, None, None)
+    assert st == B.MOE_ERR_INVALID_ARG
+    misaligned = ctypes.c_void_p(4096 + 8)
+    st = lib.moe_forward(misaligned, fake, None, fake, fake, fake, 8, 128, 4, 2, 256, 1, B.MOE_F32, fake, fake, fake,
+                         None, None, fake, need, None, None)
+    assert st == B.MOE_ERR_INVALID_ARG
+    st = lib.moe_forward(fake, fake, None, fake, fake, fake, 8, 128, 4, 2, 256, 1, B.MOE_F32, fake, fake, fake, None,
+                         None, ctypes.c_void_p(4096 + 16), need, None, None)
+    assert st == B.MOE_ERR_INVALID_ARG
+    assert "256-byte" in B.last_error_detail(lib)
+
+
+def test_get_permutation_validation(lib):
+    fake = ctypes.c_void_p(4096)
+    st = lib.moe_get_permutation(fake, 16, 8, 128, 4, 2, 256, B.MOE_F32, None, None, None, None)
+    assert st == B.MOE_ERR_WORKSPACE
+    st = lib.moe_get_permutation(fake, 1 << 30, 8, 128, 4, 5, 256, B.MOE_F32, None, None, None, None)
+    assert st == B.MOE_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="missing"):
+        B.load_library(str(tmp_path / "nope.so"))

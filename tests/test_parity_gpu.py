@@ -1,0 +1,166 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs, at every workload size and on the edge cases."""
+import numpy as np
+import pytest
+import torch
+
+import parity
+from sparse_mixture_experts_renorm_b200 import _binding as B
+from sparse_mixture_experts_renorm_b200 import get_permutation, moe_forward
+from sparse_mixture_experts_renorm_b200.workloads import WORKLOADS, Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def run(wl, inp=None, seed=0):
+    if inp is None:
+        inp = make_inputs(wl, "cuda", seed)
+    res = moe_forward(inp.x, inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k, wl.renorm)
+    torch.cuda.synchronize()
+    perm = get_permutation(res, wl.T, wl.d, wl.E, wl.k, wl.I, inp.x.dtype)
+    torch.cuda.synchronize()
+    return inp, res, perm
+
+
+def check(wl, inp, res, perm, tokens=None):
+    rep = parity.check(inp, res, perm, wl.k, wl.renorm, wl.dtype, tokens=tokens)
+    print(f"\n[{wl.name}] {rep}")
+    return rep
+
+
+# --------------------------------------------------------------- edge cases --
+
+EDGE = [
+    Workload("f32_ragged", T=300, d=64, E=6, k=3, I=96, renorm=True, dtype="f32", router_std=0.5),
+    Workload("f32_norenorm", T=77, d=36, E=5, k=2, I=20, renorm=False, dtype="f32", router_std=0.5),
+    Workload("f32_dense_E1", T=33, d=32, E=1, k=1, I=48, renorm=True, dtype="f32"),
+    Workload("f32_T1", T=1, d=128, E=4, k=2, I=256, renorm=True, dtype="f32", router_std=0.5),
+    Workload("bf16_T1", T=1, d=128, E=4, k=2, I=128, renorm=True, dtype="bf16", router_std=0.3),
+    Workload("bf16_T7", T=7, d=128, E=4, k=2, I=128, renorm=True, dtype="bf16", router_std=0.3),
+    Workload("bf16_ragged_tails", T=129, d=192, E=5, k=3, I=320, renorm=True, dtype="bf16", router_std=0.3),
+    Workload("bf16_norenorm_bias", T=300, d=256, E=8, k=2, I=512, renorm=False, dtype="bf16", zipf_bias=True),
+    Workload("bf16_dense_E1", T=200, d=128, E=1, k=1, I=256, renorm=True, dtype="bf16"),
+    Workload("bf16_k_eq_E", T=150, d=128, E=4, k=4, I=192, renorm=True, dtype="bf16"),
+    Workload("bf16_max_E256_k8", T=96, d=64, E=256, k=8, I=64, renorm=True, dtype="bf16", router_std=0.5),
+    Workload("bf16_many_tiles", T=1000, d=256, E=3, k=2, I=384, renorm=True, dtype="bf16", router_std=0.1),
+]
+
+
+@pytest.mark.parametrize("wl", EDGE, ids=[w.name for w in EDGE])
+def test_edge_case(wl):
+    inp, res, perm = run(wl, seed=3)
+    check(wl, inp, res, perm)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_zero_router_ties_to_lower_index(dtype):
+    wl = Workload("zero_router", T=70, d=128, E=6, k=3, I=128, renorm=True, dtype=dtype)
+    inp = make_inputs(wl, "cuda", 5)
+    inp.w_router.zero_()
+    inp, res, perm = run(wl, inp)
+    idx = res.topk_idx.cpu().numpy()
+    assert (idx == np.arange(3)).all()
+    np.testing.assert_allclose(res.topk_gate.cpu().numpy(), 1.0 / 3, rtol=1e-6)
+    np.testing.assert_array_equal(res.counts.cpu().numpy(), [70, 70, 70, 0, 0, 0])
+    assert abs(float(res.aux.cpu()[0]) - 1.0) < 1e-6
+    check(wl, inp, res, perm)
+
+
+def test_duplicate_router_rows_tie():
+    wl = Workload("dup_rows", T=64, d=128, E=5, k=2, I=128, renorm=True, dtype="bf16")
+    inp = make_inputs(wl, "cuda", 6)
+    big = torch.sign(inp.x.float().mean(0)) * 0.5
+    inp.w_router[3] = big.to(inp.w_router.dtype)
+    inp.w_router[1] = inp.w_router[3]
+    inp, res, perm = run(wl, inp)
+    idx = res.topk_idx.cpu().numpy()
+    probs_equal_top = [t for t in range(wl.T) if set(idx[t]) == {1, 3}]
+    assert probs_equal_top, "the shared row should win for some tokens"
+    for t in probs_equal_top:
+        assert list(idx[t]) == [1, 3]
+    check(wl, inp, res, perm)
+
+
+def test_unused_experts():
+    wl = Workload("unused", T=257, d=128, E=6, k=2, I=192, renorm=True, dtype="bf16")
+    inp = make_inputs(wl, "cuda", 7)
+    inp.b_router = torch.tensor([0, -40.0, 0, -40.0, 0, 0], device="cuda")
+    inp, res, perm = run(wl, inp)
+    counts = res.counts.cpu().numpy()
+    assert counts[1] == 0 and counts[3] == 0
+    check(wl, inp, res, perm)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_zero_tokens(dtype):
+    wl = Workload("empty", T=0, d=128, E=4, k=2, I=128, renorm=True, dtype=dtype)
+    inp = make_inputs(wl, "cuda", 0)
+    res = moe_forward(inp.x, inp.w_router, None, inp.w_gate, inp.w_up, inp.w_down, 2, True)
+    torch.cuda.synchronize()
+    assert res.out.shape == (0, 128)
+    np.testing.assert_array_equal(res.counts.cpu().numpy(), 0)
+    assert float(res.aux.cpu()[0]) == 0.0
+    assert int(res.status.cpu()[0]) == 0
+
+
+def test_bit_deterministic():
+    wl = Workload("determinism", T=777, d=256, E=8, k=2, I=384, renorm=True, dtype="bf16")
+    inp = make_inputs(wl, "cuda", 8)
+    a = moe_forward(inp.x, inp.w_router, None, inp.w_gate, inp.w_up, inp.w_down, 2, True)
+    b = moe_forward(inp.x, inp.w_router, None, inp.w_gate, inp.w_up, inp.w_down, 2, True)
+    torch.cuda.synchronize()
+    assert torch.equal(a.out, b.out)
+    assert torch.equal(a.topk_idx, b.topk_idx) and torch.equal(a.topk_gate, b.topk_gate)
+    assert torch.equal(a.aux, b.aux)
+
+
+def test_nonfinite_logit_sets_status_and_stays_in_bounds():
+    wl = Workload("nonfinite", T=64, d=128, E=4, k=2, I=128, renorm=True, dtype="bf16")
+    inp = make_inputs(wl, "cuda", 9)
+    inp.x[5, 3] = float("inf")
+    inp.x[9, 0] = float("nan")
+    res = moe_forward(inp.x, inp.w_router, None, inp.w_gate, inp.w_up, inp.w_down, 2, True)
+    torch.cuda.synchronize()
+    st = int(res.status.cpu()[0])
+    assert st & B.MOE_DEV_NONFINITE
+    assert not st & (B.MOE_DEV_TIMEOUT | B.MOE_DEV_INTERNAL)
+    idx = res.topk_idx.cpu().numpy()
+    assert ((idx >= 0) & (idx < 4)).all()
+    assert int(res.counts.cpu().sum()) == 128
+    # tokens without a non-finite value are unaffected
+    good = [t for t in range(64) if t not in (5, 9)]
+    assert torch.isfinite(res.out[good]).all()
+
+
+# ---------------------------------------------------------------- workloads --
+
+def test_tiny_f32_all_tokens():
+    wl = WORKLOADS["tiny_f32"]
+    inp, res, perm = run(wl)
+    check(wl, inp, res, perm)
+
+
+def test_small_bf16_sampled():
+    wl = WORKLOADS["small_bf16"]
+    inp, res, perm = run(wl)
+    check(wl, inp, res, perm, parity.sample_tokens(perm, wl.T, wl.k, n_random=256, cap=600))
+
+
+def test_mixtral_prefill_full_size_sampled():
+    wl = WORKLOADS["mixtral_prefill"]
+    inp, res, perm = run(wl)
+    check(wl, inp, res, perm, parity.sample_tokens(perm, wl.T, wl.k, n_random=24, edge=2, cap=64))
+
+
+def test_fine_grained_full_size_sampled():
+    wl = WORKLOADS["fine_grained"]
+    inp, res, perm = run(wl)
+    counts = res.counts.cpu().numpy()
+    assert counts[0] > 2 * counts.mean(), "the Zipf-like bias should skew the load towards expert 0"
+    check(wl, inp, res, perm, parity.sample_tokens(perm, wl.T, wl.k, n_random=24, edge=1, cap=96))
+
+
+def test_mixtral_decode_all_tokens():
+    wl = WORKLOADS["mixtral_decode"]
+    inp, res, perm = run(wl)
+    check(wl, inp, res, perm)
