@@ -53,17 +53,25 @@ def source_hash(kernel):
 
 
 def load_traffic(workload, kernel):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current source of that kernel."""
-    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
-    if not os.path.exists(p):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    from a committed ncu summary under profiles/, if it was taken on the
+    current source of that kernel; else None."""
+    d = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(d):
         return None
-    with open(p) as f:
-        table = json.load(f)
-    ent = table.get(workload, {}).get(kernel)
-    if not ent or ent.get("source_sha") != source_hash(kernel):
-        return None
-    return ent.get("bytes_per_launch")
+    want = source_hash(kernel)
+    for fn in sorted(os.listdir(d)):
+        if not fn.endswith((".md", ".txt")):
+            continue
+        with open(os.path.join(d, fn)) as f:
+            for line in f:
+                if not line.startswith("traffic:"):
+                    continue
+                parts = line.split()
+                kv = dict(p.split("=", 1) for p in parts[3:] if "=" in p)
+                if parts[1] == workload and parts[2] == kernel and kv.get("source_sha") == want:
+                    return int(kv["bytes_per_launch"])
+    return None
 
 
 # ------------------------------------------------------------ algorithmic work
@@ -75,7 +83,7 @@ def algorithmic(wl, counts):
     R = T * k
     el = 2 if wl.dtype == "bf16" else 4
     used = int((np.asarray(counts) > 0).sum())
-    nb = (T + 31) // 32
+    nb = (T + 127) // 128 if wl.dtype == "bf16" else (T + 31) // 32
     return {
         "router_topk": dict(flops=2.0 * T * d * E, bytes=T * d * el + E * d * el + T * k * 12 + nb * E * 8),
         "route_scan": dict(flops=0.0, bytes=nb * E * 12 + (E + 1) * 8 + E * 4),
@@ -104,7 +112,7 @@ class ClockSampler:
             bus = None
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader", "-lms", "200"]
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader", "-lms", "100"]
         if bus:
             cmd += ["-i", bus]
         try:
@@ -132,11 +140,15 @@ class ClockSampler:
                 if len(parts) < 10:
                     continue
                 try:
-                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    base, _, frac = parts[0].partition(".")
+                    ts = time.mktime(time.strptime(base, "%Y/%m/%d %H:%M:%S")) + float("0." + (frac or "0"))
                 except Exception:
                     ts = None
                 rows.append((ts, parts))
-        sel = [p for ts, p in rows if ts is not None and t0 - 1.0 <= ts <= t1 + 1.0] or [p for _, p in rows]
+        sel = [p for ts, p in rows if ts is not None and t0 <= ts <= t1]
+        if not sel:  # region shorter than the sampling period: nearest samples
+            near = sorted((abs(ts - 0.5 * (t0 + t1)), i) for i, (ts, _) in enumerate(rows) if ts is not None)
+            sel = [rows[i][1] for _, i in near[:2]]
         for parts in sel:
             try:
                 sm.append(float(parts[2].split()[0]))
@@ -170,8 +182,11 @@ def cpu_oracle_rate(inp_cpu, wl, budget_s, max_tokens=None):
                        wl.renorm)
         return time.perf_counter() - t0
 
-    t1 = run(1)
-    n = int(max(1, min(wl.T if max_tokens is None else max_tokens, budget_s / max(t1, 1e-6))))
+    cap = wl.T if max_tokens is None else max_tokens
+    run(1)  # load the library and touch the weights
+    n0 = min(cap, 4)
+    per_token = run(n0) / n0
+    n = int(max(1, min(cap, budget_s / max(per_token, 1e-9))))
     dt = run(n)
     return n / dt, n, dt, threads
 
@@ -312,22 +327,27 @@ def main():
     if status:
         raise RuntimeError(f"device status word {status:#x} after the timed region")
 
-    # ---- end to end through the host API: pinned x in, out + aux back
+    # ---- end to end through the host API: pinned x in, out + aux back, with
+    # the copies of neighbouring steps overlapped with the compute
+    from sparse_mixture_experts_renorm_b200 import HostPipeline
+
     e2e_steps = max(1, min(args.steps, 50))
     x_host = x.detach().to("cpu").pin_memory()
-    out_host = torch.empty((wl.T, wl.d), dtype=torch.float32).pin_memory()
-    aux_host = torch.empty((1,), dtype=torch.float32).pin_memory()
-    x_dev = torch.empty_like(x)
-    for _ in range(2):
-        layer.forward_host(x_host, out_host, aux_host, x_dev)
+    outs = [torch.empty((wl.T, wl.d), dtype=torch.float32).pin_memory() for _ in range(2)]
+    auxs = [torch.empty((1,), dtype=torch.float32).pin_memory() for _ in range(2)]
+    pipe = HostPipeline(layer)
+    for i in range(3):
+        pipe.submit(x_host, outs[i & 1], auxs[i & 1])
+    pipe.synchronize()
     torch.cuda.synchronize()
     s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
-    s2.record(stream)
-    for _ in range(e2e_steps):
-        layer.forward_host(x_host, out_host, aux_host, x_dev)
-    e2.record(stream)
+    s2.record(pipe.h2d)
+    for i in range(e2e_steps):
+        pipe.submit(x_host, outs[i & 1], auxs[i & 1])
+    e2.record(pipe.d2h)
+    pipe.synchronize()
     torch.cuda.synchronize()
     barrier()
     ms_e2e = s2.elapsed_time(e2)

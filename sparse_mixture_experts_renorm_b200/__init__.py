@@ -17,7 +17,8 @@ import torch
 from . import _binding as B
 from ._binding import MoEError, load_library
 
-__all__ = ["MoEError", "MoEOutputs", "MoELayer", "moe_forward", "workspace_size", "get_permutation", "load_library"]
+__all__ = ["MoEError", "MoEOutputs", "MoELayer", "HostPipeline", "moe_forward", "workspace_size", "get_permutation",
+           "load_library"]
 
 
 def _dtype_code(t: torch.dtype) -> int:
@@ -163,3 +164,53 @@ class MoELayer:
         self(x_dev)
         out_host.copy_(self.out, non_blocking=True)
         aux_host.copy_(self.aux, non_blocking=True)
+
+
+class HostPipeline:
+    """Runs batches that live in pinned host memory through a ``MoELayer``
+    with the copies overlapped: batch i+1 is copied in and batch i-1 copied
+    out while batch i computes (two device buffers each for x and out, one
+    stream per direction). ``submit`` returns without synchronising; the
+    host output buffer may be read after ``synchronize``."""
+
+    def __init__(self, layer: "MoELayer"):
+        self.layer = layer
+        dev = layer.w_gate.device
+        T, d = layer.T, layer.d
+        self.x_dev = [torch.empty((T, d), dtype=layer.dtype, device=dev) for _ in range(2)]
+        self.out_dev = [torch.empty((T, d), dtype=torch.float32, device=dev) for _ in range(2)]
+        self.aux_dev = [torch.empty((1,), dtype=torch.float32, device=dev) for _ in range(2)]
+        self.compute = torch.cuda.current_stream(dev)
+        self.h2d = torch.cuda.Stream(dev)
+        self.d2h = torch.cuda.Stream(dev)
+        self.in_ready = [torch.cuda.Event() for _ in range(2)]
+        self.computed = [torch.cuda.Event() for _ in range(2)]
+        self.out_free = [torch.cuda.Event() for _ in range(2)]
+        self.i = 0
+
+    def submit(self, x_host, out_host, aux_host) -> None:
+        b = self.i & 1
+        L = self.layer
+        if self.i >= 2:
+            self.h2d.wait_event(self.computed[b])  # x buffer b no longer read
+        with torch.cuda.stream(self.h2d):
+            self.x_dev[b].copy_(x_host, non_blocking=True)
+            self.in_ready[b].record(self.h2d)
+        self.compute.wait_event(self.in_ready[b])
+        if self.i >= 2:
+            self.compute.wait_event(self.out_free[b])  # out buffer b copied out
+        moe_forward(self.x_dev[b], L.w_router, L.b_router, L.w_gate, L.w_up, L.w_down, L.k, L.renorm,
+                    out=self.out_dev[b], topk_idx=L.topk_idx, topk_gate=L.topk_gate, counts=L.counts,
+                    aux=self.aux_dev[b], workspace=L.workspace, status=L.status,
+                    stream=self.compute.cuda_stream)
+        self.computed[b].record(self.compute)
+        self.d2h.wait_event(self.computed[b])
+        with torch.cuda.stream(self.d2h):
+            out_host.copy_(self.out_dev[b], non_blocking=True)
+            aux_host.copy_(self.aux_dev[b], non_blocking=True)
+            self.out_free[b].record(self.d2h)
+        self.i += 1
+
+    def synchronize(self) -> None:
+        self.d2h.synchronize()
+        self.compute.synchronize()

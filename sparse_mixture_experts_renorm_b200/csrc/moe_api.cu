@@ -89,7 +89,7 @@ int device_sm_count() {
 
 Workspace workspace_layout(int T, int d, int E, int k, int I, moe_dtype dtype) {
   const size_t R = (size_t)T * k;
-  const size_t nb = (size_t)router_blocks(T);
+  const size_t nb = (size_t)router_blocks(T, MOE_F32);  // the finer blocking of the two routers
   const size_t el = dtype == MOE_BF16 ? 2 : 4;
   Workspace w;
   size_t o = 0;
@@ -214,10 +214,10 @@ moe_status forward_impl(const void* x, const void* w_router, const float* b_rout
                       status, stream);
   if (err != cudaSuccess) return fail_cuda(err, "router kernel");
   marks.mark(stream);
-  err = launch_route_scan(T, E, k, blk_cnt, blk_psum, cnt, offsets, mtile, aux_p, stream);
+  err = launch_route_scan(router_blocks(T, dtype), T, E, k, blk_cnt, blk_psum, cnt, offsets, mtile, aux_p, stream);
   if (err != cudaSuccess) return fail_cuda(err, "routing scan kernel");
   marks.mark(stream);
-  err = launch_permute(dtype, x, T, d, E, k, topk_idx, lrank, blk_cnt, perm_tok, inv, xp, status, stream);
+  err = launch_permute(dtype, x, T, d, E, k, router_block_tokens(dtype), topk_idx, lrank, blk_cnt, perm_tok, inv, xp, status, stream);
   if (err != cudaSuccess) return fail_cuda(err, "permute kernel");
 
   if (dtype == MOE_BF16) {

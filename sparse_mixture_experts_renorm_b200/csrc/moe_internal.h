@@ -11,9 +11,11 @@
 
 namespace moe {
 
-// Router: tokens per CTA (one CTA's routing partials form one block of the
-// two-level scan that gives every dispatched row its position).
-constexpr int kRouterTokens = 32;
+// Router: tokens per CTA. One CTA's routing partials form one block of the
+// two-level scan that gives every dispatched row its position: 128 tokens
+// (the UMMA M) for the bf16 tensor-core router, 32 for the fp32 SIMT router.
+constexpr int kRouterTokensTc = 128;
+constexpr int kRouterTokensSimt = 32;
 constexpr int kRouterThreads = 128;
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 8;
@@ -56,7 +58,11 @@ struct Workspace {
 
 Workspace workspace_layout(int T, int d, int E, int k, int I, moe_dtype dtype);
 
-inline int router_blocks(int T) { return (T + kRouterTokens - 1) / kRouterTokens; }
+inline int router_block_tokens(moe_dtype dtype) { return dtype == MOE_BF16 ? kRouterTokensTc : kRouterTokensSimt; }
+inline int router_blocks(int T, moe_dtype dtype) {
+  const int rb = router_block_tokens(dtype);
+  return (T + rb - 1) / rb;
+}
 
 // Encode a 2-D bf16 tensor map (rows x cols, row-major) with a box of
 // box_rows x 64 columns and the 128-byte swizzle. Returns false on failure.
@@ -68,10 +74,14 @@ cudaError_t launch_router(moe_dtype dtype, const void* x, const void* w_router, 
                           int d, int E, int k, int renorm, int32_t* topk_idx, float* topk_gate, int32_t* lrank,
                           int32_t* blk_cnt, float* blk_psum, int32_t* status, cudaStream_t stream);
 
-cudaError_t launch_route_scan(int T, int E, int k, int32_t* blk_cnt, const float* blk_psum, int32_t* counts,
+cudaError_t launch_router_tc(const void* x, const void* w_router, const float* b_router, int T, int d, int E, int k,
+                             int renorm, int32_t* topk_idx, float* topk_gate, int32_t* lrank, int32_t* blk_cnt,
+                             float* blk_psum, int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_route_scan(int nb, int T, int E, int k, int32_t* blk_cnt, const float* blk_psum, int32_t* counts,
                               int32_t* offsets, int32_t* mtile128, float* aux, cudaStream_t stream);
 
-cudaError_t launch_permute(moe_dtype dtype, const void* x, int T, int d, int E, int k, const int32_t* topk_idx,
+cudaError_t launch_permute(moe_dtype dtype, const void* x, int T, int d, int E, int k, int rb, const int32_t* topk_idx,
                            const int32_t* lrank, const int32_t* blk_base, int32_t* perm_tok, int32_t* inv,
                            void* xp, int32_t* status, cudaStream_t stream);
 

@@ -9,103 +9,104 @@
 namespace moe {
 namespace {
 
-// One warp per token. Lanes j < k compute the row of slot j from the
-// per-block base row of its expert plus its rank inside the router block;
-// then the warp copies the token's row of x (16-byte vectors, read once) to
-// each of its k rows.
-__global__ void __launch_bounds__(256) permute_kernel(const uint4* __restrict__ x, int T, int nvec, int E, int k,
-                                                      int R, const int32_t* __restrict__ topk_idx,
-                                                      const int32_t* __restrict__ lrank,
-                                                      const int32_t* __restrict__ blk_base,
-                                                      int32_t* __restrict__ perm_tok, int32_t* __restrict__ inv,
-                                                      uint4* __restrict__ xp, int32_t* status) {
-  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (t >= T) return;
-  int row = -1;
-  if (lane < k) {
-    const int e = topk_idx[(size_t)t * k + lane];
-    if (e >= 0 && e < E) row = blk_base[(size_t)(t / kRouterTokens) * E + e] + lrank[(size_t)t * k + lane];
+constexpr int kCopyThreads = 256;  // 16-byte vectors per block (4 KB of a row)
+
+// Block (token t, chunk c): threads j < k compute the row of slot j from the
+// per-block base row of its expert plus its rank inside the router block
+// (chunk 0 also records perm_tok / inv); then every thread copies one 16-byte
+// vector of x[t] to each of the token's k rows.
+__global__ void __launch_bounds__(kCopyThreads) permute_kernel(const uint4* __restrict__ x, int nvec, int E, int k,
+                                                              int rb, int R, const int32_t* __restrict__ topk_idx,
+                                                              const int32_t* __restrict__ lrank,
+                                                              const int32_t* __restrict__ blk_base,
+                                                              int32_t* __restrict__ perm_tok, int32_t* __restrict__ inv,
+                                                              uint4* __restrict__ xp, int32_t* status) {
+  const int t = blockIdx.x;
+  __shared__ int s_rows[kMaxTopK];
+  if (threadIdx.x < k) {
+    const int j = threadIdx.x;
+    const int e = topk_idx[(size_t)t * k + j];
+    int row = -1;
+    if (e >= 0 && e < E) row = blk_base[(size_t)(t / rb) * E + e] + lrank[(size_t)t * k + j];
     if (row < 0 || row >= R) {
       atomicOr(status, MOE_DEV_INTERNAL);
       row = -1;
-    } else {
+    } else if (blockIdx.y == 0) {
       perm_tok[row] = t;
-      inv[(size_t)t * k + lane] = row;
+      inv[(size_t)t * k + j] = row;
     }
+    s_rows[j] = row;
   }
-  int rows[kMaxTopK];
+  __syncthreads();
+  const int i = blockIdx.y * kCopyThreads + threadIdx.x;
+  if (i >= nvec) return;
+  const uint4 v = __ldg(x + (size_t)t * nvec + i);
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) rows[j] = __shfl_sync(0xffffffffu, row, j);
-  const uint4* src = x + (size_t)t * nvec;
-  for (int i = lane; i < nvec; i += 32) {
-    const uint4 v = __ldg(src + i);
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j)
-      if (j < k && rows[j] >= 0) xp[(size_t)rows[j] * nvec + i] = v;
-  }
+  for (int j = 0; j < kMaxTopK; ++j)
+    if (j < k && s_rows[j] >= 0) xp[(size_t)s_rows[j] * nvec + i] = v;
 }
 
-// One warp per token; fp32 accumulation over the k slots in slot order.
-__global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ y, int T, int nvec4, int k, int R,
-                                                      const int32_t* __restrict__ inv,
-                                                      const float* __restrict__ gate, float4* __restrict__ out,
-                                                      int32_t* status) {
-  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (t >= T) return;
-  int row = 0;
-  float g = 0.f;
-  if (lane < k) {
-    row = inv[(size_t)t * k + lane];
-    g = gate[(size_t)t * k + lane];
+// Block (token t, chunk c): every thread sums one float4 of its token's k
+// expert rows, weighted by the gates, in slot order (fp32).
+__global__ void __launch_bounds__(kCopyThreads) combine_kernel(const float4* __restrict__ y, int nvec4, int k, int R,
+                                                              const int32_t* __restrict__ inv,
+                                                              const float* __restrict__ gate,
+                                                              float4* __restrict__ out, int32_t* status) {
+  const int t = blockIdx.x;
+  __shared__ int s_rows[kMaxTopK];
+  __shared__ float s_g[kMaxTopK];
+  if (threadIdx.x < k) {
+    const int j = threadIdx.x;
+    int row = inv[(size_t)t * k + j];
+    float g = gate[(size_t)t * k + j];
     if (row < 0 || row >= R) {
       atomicOr(status, MOE_DEV_INTERNAL);
       row = 0;
       g = 0.f;
     }
+    s_rows[j] = row;
+    s_g[j] = g;
   }
-  int rows[kMaxTopK];
-  float gs[kMaxTopK];
+  __syncthreads();
+  const int i = blockIdx.y * kCopyThreads + threadIdx.x;
+  if (i >= nvec4) return;
+  float4 v[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j)
+    if (j < k) v[j] = __ldg(y + (size_t)s_rows[j] * nvec4 + i);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j) {
-    rows[j] = __shfl_sync(0xffffffffu, row, j);
-    gs[j] = __shfl_sync(0xffffffffu, g, j);
-  }
-  for (int i = lane; i < nvec4; i += 32) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      if (j < k) {
-        const float4 v = __ldg(y + (size_t)rows[j] * nvec4 + i);
-        acc.x = fmaf(gs[j], v.x, acc.x);
-        acc.y = fmaf(gs[j], v.y, acc.y);
-        acc.z = fmaf(gs[j], v.z, acc.z);
-        acc.w = fmaf(gs[j], v.w, acc.w);
-      }
+    if (j < k) {
+      const float g = s_g[j];
+      acc.x = fmaf(g, v[j].x, acc.x);
+      acc.y = fmaf(g, v[j].y, acc.y);
+      acc.z = fmaf(g, v[j].z, acc.z);
+      acc.w = fmaf(g, v[j].w, acc.w);
     }
-    out[(size_t)t * nvec4 + i] = acc;
   }
+  out[(size_t)t * nvec4 + i] = acc;
 }
 
 }  // namespace
 
-cudaError_t launch_permute(moe_dtype dtype, const void* x, int T, int d, int E, int k, const int32_t* topk_idx,
+cudaError_t launch_permute(moe_dtype dtype, const void* x, int T, int d, int E, int k, int rb, const int32_t* topk_idx,
                            const int32_t* lrank, const int32_t* blk_base, int32_t* perm_tok, int32_t* inv, void* xp,
                            int32_t* status, cudaStream_t stream) {
   const int elem = dtype == MOE_BF16 ? 2 : 4;
   const int nvec = d * elem / 16;
-  const int blocks = (T + 7) / 8;
-  permute_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4*>(x), T, nvec, E, k, T * k, topk_idx, lrank,
-                                             blk_base, perm_tok, inv, static_cast<uint4*>(xp), status);
+  const dim3 grid(T, (nvec + kCopyThreads - 1) / kCopyThreads);
+  permute_kernel<<<grid, kCopyThreads, 0, stream>>>(static_cast<const uint4*>(x), nvec, E, k, rb, T * k, topk_idx, lrank,
+                                                    blk_base, perm_tok, inv, static_cast<uint4*>(xp), status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_combine(int T, int d, int k, const float* y, const int32_t* inv, const float* topk_gate, float* out,
                            int32_t* status, cudaStream_t stream) {
-  const int blocks = (T + 7) / 8;
-  combine_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(y), T, d / 4, k, T * k, inv, topk_gate,
-                                             reinterpret_cast<float4*>(out), status);
+  const int nvec4 = d / 4;
+  const dim3 grid(T, (nvec4 + kCopyThreads - 1) / kCopyThreads);
+  combine_kernel<<<grid, kCopyThreads, 0, stream>>>(reinterpret_cast<const float4*>(y), nvec4, k, T * k, inv,
+                                                    topk_gate, reinterpret_cast<float4*>(out), status);
   return cudaGetLastError();
 }
 

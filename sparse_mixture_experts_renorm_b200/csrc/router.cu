@@ -1,8 +1,9 @@
-// router.cu — kernel (a): router logits, softmax over E, top-k with ties to
-// the lower expert index, gates (optionally renormalised), per-block expert
-// histogram, per-block rank of every assignment and per-block sums of the
-// probabilities; then the single-CTA scan that turns the per-block counts into
-// expert offsets, per-block base rows, the tcgen05 tile schedule and the
+// router.cu — kernel (a) for fp32 (the bf16 router is router_tc.cu): router
+// logits, softmax over E, top-k with ties to the lower expert index, gates
+// (optionally renormalised), per-block expert histogram, per-block rank of
+// every assignment and per-block sums of the probabilities; then, for both
+// dtypes, the single-CTA scan that turns the per-block counts into expert
+// offsets, per-block base rows, the tcgen05 tile schedule and the
 // load-balancing statistic.
 //
 // Method: axonml-nn layers/moe.rs, MoERouter::route (Linear -> softmax ->
@@ -17,114 +18,12 @@
 namespace moe {
 namespace {
 
-__device__ __forceinline__ uint32_t u4_get(const uint4& v, int i) {
-  return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
-}
-
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                               uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Logits of the CTA's 32 tokens against every expert, bf16 inputs, fp32
-// accumulation on the tensor cores (m16n8k16). The 4 warps split d into
-// interleaved 64-column chunks; their partial sums are added in warp order.
-// Inside a chunk the k-slots of the MMA fragments are assigned to physical
-// columns so that every thread reads 16 contiguous bytes of x and of W_r;
-// A and B use the same assignment, so each product pairs x[t,c] with W_r[e,c].
-__device__ void router_logits_bf16(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ wr,
-                                   int T, int d, int E, int tok0, float* s_logit, int ld, float* s_part) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, tq = lane & 3;
-  for (int e0 = 0; e0 < E; e0 += 64) {
-    const int EC = min(64, E - e0);
-    const int NT = (EC + 7) >> 3;
-    float acc[2][8][4];
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[mt][nt][i] = 0.f;
-
-    for (int kc = warp * 64; kc < d; kc += 4 * 64) {
-      uint4 a[2][2][2];  // [m-tile][row g / row g+8][32-column half]
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-          const int t = tok0 + mt * 16 + hr * 8 + g;
-          if (t < T) {
-            const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d + kc + tq * 8);
-            a[mt][hr][0] = __ldg(src);
-            a[mt][hr][1] = __ldg(src + 4);
-          } else {
-            a[mt][hr][0] = make_uint4(0, 0, 0, 0);
-            a[mt][hr][1] = make_uint4(0, 0, 0, 0);
-          }
-        }
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        if (nt < NT) {
-          const int e = e0 + nt * 8 + g;
-          uint4 b[2];
-          if (e < E) {
-            const uint4* src = reinterpret_cast<const uint4*>(wr + (size_t)e * d + kc + tq * 8);
-            b[0] = __ldg(src);
-            b[1] = __ldg(src + 4);
-          } else {
-            b[0] = make_uint4(0, 0, 0, 0);
-            b[1] = make_uint4(0, 0, 0, 0);
-          }
-#pragma unroll
-          for (int half = 0; half < 2; ++half)
-#pragma unroll
-            for (int s = 0; s < 2; ++s) {
-              const uint32_t b0 = u4_get(b[half], 2 * s), b1 = u4_get(b[half], 2 * s + 1);
-#pragma unroll
-              for (int mt = 0; mt < 2; ++mt)
-                mma_bf16_16816(acc[mt][nt], u4_get(a[mt][0][half], 2 * s), u4_get(a[mt][1][half], 2 * s),
-                               u4_get(a[mt][0][half], 2 * s + 1), u4_get(a[mt][1][half], 2 * s + 1), b0, b1);
-            }
-        }
-      }
-    }
-    // accumulator (row g, cols 2tq..2tq+1) and (row g+8, same cols)
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const int row = mt * 16 + g, col = nt * 8 + 2 * tq;
-        float* p0 = s_part + (warp * 32 + row) * 64 + col;
-        float* p1 = s_part + (warp * 32 + row + 8) * 64 + col;
-        p0[0] = acc[mt][nt][0];
-        p0[1] = acc[mt][nt][1];
-        p1[0] = acc[mt][nt][2];
-        p1[1] = acc[mt][nt][3];
-      }
-    __syncthreads();
-    for (int i = threadIdx.x; i < kRouterTokens * EC; i += blockDim.x) {
-      const int row = i / EC, col = i - row * EC;
-      float s = s_part[(0 * 32 + row) * 64 + col];
-      s += s_part[(1 * 32 + row) * 64 + col];
-      s += s_part[(2 * 32 + row) * 64 + col];
-      s += s_part[(3 * 32 + row) * 64 + col];
-      s_logit[row * ld + e0 + col] = s;
-    }
-    __syncthreads();
-  }
-}
-
 // fp32 logits with plain FFMA (the fp32 workload is small; TF32 tensor cores
 // would not meet its 1e-4 tolerance).
 __device__ void router_logits_f32(const float* __restrict__ x, const float* __restrict__ wr, int T, int d, int E,
                                   int tok0, float* s_logit, int ld) {
-  for (int i = threadIdx.x; i < kRouterTokens * E; i += blockDim.x) {
-    const int e = i / kRouterTokens, row = i - e * kRouterTokens;
+  for (int i = threadIdx.x; i < kRouterTokensSimt * E; i += blockDim.x) {
+    const int e = i / kRouterTokensSimt, row = i - e * kRouterTokensSimt;
     const int t = tok0 + row;
     float s = 0.f;
     if (t < T) {
@@ -137,29 +36,24 @@ __device__ void router_logits_f32(const float* __restrict__ x, const float* __re
   __syncthreads();
 }
 
-template <typename Tin>
 __global__ void __launch_bounds__(kRouterThreads) router_kernel(
-    const Tin* __restrict__ x, const Tin* __restrict__ wr, const float* __restrict__ br, int T, int d, int E, int k,
+    const float* __restrict__ x, const float* __restrict__ wr, const float* __restrict__ br, int T, int d, int E, int k,
     int renorm, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate, int32_t* __restrict__ lrank,
     int32_t* __restrict__ blk_cnt, float* __restrict__ blk_psum, int32_t* status) {
   extern __shared__ float smem[];
   const int ld = E + 1;
-  float* s_p = smem;                         // [32][E+1] logits, then probabilities
-  float* s_part = smem + kRouterTokens * ld; // [4][32][64] per-warp partial logits (bf16 path)
-  __shared__ int32_t s_idx[kRouterTokens][kMaxTopK];
+  float* s_p = smem;  // [32][E+1] logits, then probabilities
+  __shared__ int32_t s_idx[kRouterTokensSimt][kMaxTopK];
 
-  const int tok0 = blockIdx.x * kRouterTokens;
-  const int ntok = min(kRouterTokens, T - tok0);
+  const int tok0 = blockIdx.x * kRouterTokensSimt;
+  const int ntok = min(kRouterTokensSimt, T - tok0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  if constexpr (sizeof(Tin) == 2)
-    router_logits_bf16(x, wr, T, d, E, tok0, s_p, ld, s_part);
-  else
-    router_logits_f32(x, wr, T, d, E, tok0, s_p, ld);
+  router_logits_f32(x, wr, T, d, E, tok0, s_p, ld);
 
   // ---- softmax, top-k and gates: one warp per token --------------------
   const int NE = (E + 31) >> 5;  // values per lane (<= 8)
-  for (int row = warp; row < kRouterTokens; row += kRouterThreads / 32) {
+  for (int row = warp; row < kRouterTokensSimt; row += kRouterThreads / 32) {
     if (row >= ntok) {
       if (lane < kMaxTopK) s_idx[row][lane] = -1;
       for (int e = lane; e < E; e += 32) s_p[row * ld + e] = 0.f;
@@ -303,6 +197,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int nb, int T, int E, 
   if (active) {
     int c = 0;
     double ps = 0.0;
+#pragma unroll 8
     for (int b = b0; b < b1; ++b) {
       c += blk_cnt[(size_t)b * E + e];
       ps += (double)blk_psum[(size_t)b * E + e];
@@ -354,39 +249,25 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int nb, int T, int E, 
 
 }  // namespace
 
-size_t router_smem_bytes(moe_dtype dtype, int E) {
-  size_t b = (size_t)kRouterTokens * (E + 1) * sizeof(float);
-  if (dtype == MOE_BF16) b += (size_t)4 * 32 * 64 * sizeof(float);
-  return b;
-}
-
 cudaError_t launch_router(moe_dtype dtype, const void* x, const void* w_router, const float* b_router, int T, int d,
                           int E, int k, int renorm, int32_t* topk_idx, float* topk_gate, int32_t* lrank,
                           int32_t* blk_cnt, float* blk_psum, int32_t* status, cudaStream_t stream) {
-  const int nb = router_blocks(T);
-  const size_t smem = router_smem_bytes(dtype, E);
-  if (dtype == MOE_BF16) {
-    auto kern = router_kernel<__nv_bfloat16>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    kern<<<nb, kRouterThreads, smem, stream>>>(static_cast<const __nv_bfloat16*>(x),
-                                               static_cast<const __nv_bfloat16*>(w_router), b_router, T, d, E, k,
-                                               renorm, topk_idx, topk_gate, lrank, blk_cnt, blk_psum, status);
-  } else {
-    auto kern = router_kernel<float>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    kern<<<nb, kRouterThreads, smem, stream>>>(static_cast<const float*>(x), static_cast<const float*>(w_router),
-                                               b_router, T, d, E, k, renorm, topk_idx, topk_gate, lrank, blk_cnt,
-                                               blk_psum, status);
-  }
+  if (dtype == MOE_BF16)
+    return launch_router_tc(x, w_router, b_router, T, d, E, k, renorm, topk_idx, topk_gate, lrank, blk_cnt, blk_psum,
+                            status, stream);
+  const int nb = router_blocks(T, MOE_F32);
+  const size_t smem = (size_t)kRouterTokensSimt * (E + 1) * sizeof(float);
+  cudaError_t err = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  router_kernel<<<nb, kRouterThreads, smem, stream>>>(static_cast<const float*>(x), static_cast<const float*>(w_router),
+                                                      b_router, T, d, E, k, renorm, topk_idx, topk_gate, lrank, blk_cnt,
+                                                      blk_psum, status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_route_scan(int T, int E, int k, int32_t* blk_cnt, const float* blk_psum, int32_t* counts,
+cudaError_t launch_route_scan(int nb, int T, int E, int k, int32_t* blk_cnt, const float* blk_psum, int32_t* counts,
                               int32_t* offsets, int32_t* mtile128, float* aux, cudaStream_t stream) {
-  route_scan_kernel<<<1, 1024, 0, stream>>>(router_blocks(T), T, E, k, blk_cnt, blk_psum, counts, offsets, mtile128,
-                                            aux);
+  route_scan_kernel<<<1, 1024, 0, stream>>>(nb, T, E, k, blk_cnt, blk_psum, counts, offsets, mtile128, aux);
   return cudaGetLastError();
 }
 

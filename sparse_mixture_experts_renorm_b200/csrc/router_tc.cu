@@ -1,0 +1,321 @@
+// router_tc.cu — kernel (a) for bf16: the router as a 128 x E tile on the
+// tcgen05 tensor cores, then softmax, top-k, gates, the per-block histogram,
+// the in-block rank of every assignment and the per-block probability sums,
+// with one thread per token.
+//
+// Method: axonml-nn layers/moe.rs, MoERouter::route (Linear -> softmax ->
+// stable descending sort -> first k -> renormalise, 1/k if the sum is not
+// positive), MoELayer::forward ("Track expert utilization"),
+// load_balancing_loss (E * sum_i f_i * P_i); Model Architecture Patterns,
+// "Top-K Router" (raw top-k softmax gates when not renormalised).
+//
+// Each CTA owns 128 tokens (the UMMA M); N is E rounded up to a multiple of 16
+// (TMA zero-fills the missing router rows). Warp 0 streams x and W_r through a
+// shared-memory ring by TMA, warp 1 issues 128 x N x 16 UMMAs into TMEM, and
+// warps 2-5 read each token's logits row from its own TMEM lane, so softmax and
+// top-k need no cross-thread reduction. After the MMAs the ring is reused for
+// the [128][E+1] probability tile that the per-block statistics read.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kRB = kRouterTokensTc;  // 128 tokens per CTA
+
+struct RouterCfg {
+  int npad;        // UMMA N
+  int stages;      // ring depth
+  int stage_bytes; // x tile + W_r tile
+  int tmem_cols;   // power of two >= max(32, npad)
+  int smem_bytes;  // dynamic shared memory
+};
+
+RouterCfg router_cfg(int E) {
+  RouterCfg c;
+  c.npad = ((E + 15) / 16) * 16;
+  c.stage_bytes = kRB * kBK * 2 + c.npad * kBK * 2;
+  c.stages = (192 * 1024) / c.stage_bytes;
+  if (c.stages > 8) c.stages = 8;
+  c.tmem_cols = 32;
+  while (c.tmem_cols < c.npad) c.tmem_cols <<= 1;
+  c.smem_bytes = c.stages * c.stage_bytes + 1024 + 12288;
+  return c;
+}
+
+// (v, e) ranks ahead of (bv, be): larger probability, or equal and lower index.
+__device__ __forceinline__ bool ahead(float v, int e, float bv, int be) { return v > bv || (v == bv && e < be); }
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                     const float* __restrict__ br, int T, int d, int E, int k, int renorm, int npad, int stages,
+                     int stage_bytes, int tmem_cols, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate,
+                     int32_t* __restrict__ lrank, int32_t* __restrict__ blk_cnt, float* __restrict__ blk_psum,
+                     int32_t* status, uint64_t limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes);
+  uint64_t* full = bars;           // [stages]
+  uint64_t* empty = bars + 8;      // [stages]
+  uint64_t* tfull = bars + 16;
+  uint64_t* done = bars + 17;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 18);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  int* s_idx = reinterpret_cast<int*>(s_tmem + 4);  // [128][kMaxTopK]
+  int* s_wcnt = s_idx + kRB * kMaxTopK;              // [4][E] per-warp counts, then exclusive prefix
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tok0 = blockIdx.x * kRB;
+  const int KB = d / kBK;
+  const int a_bytes = kRB * kBK * 2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(done, 1);
+    *s_abort = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, s_abort, status, limit_ns)) break;
+        mbar_arrive_expect_tx(&full[stage], stage_bytes);
+        uint8_t* st = ring + stage * stage_bytes;
+        tma_load_2d(st, &tmX, &full[stage], kb * kBK, tok0);
+        tma_load_2d(st + a_bytes, &tmW, &full[stage], kb * kBK, 0);
+        ++issued;
+        if (++stage == stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      const int n = issued < stages ? issued : stages;
+      for (int i = 0; i < n; ++i) {
+        if (stage == 0) {
+          stage = stages;
+          phase ^= 1u;
+        }
+        --stage;
+        mbar_wait(&full[stage], phase, nullptr, status, limit_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kRB, npad);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&full[stage], phase, s_abort, status, limit_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint8_t* st = ring + stage * stage_bytes;
+        const uint64_t adesc = sw128_kmajor_desc(smem_u32(st));
+        const uint64_t bdesc = sw128_kmajor_desc(smem_u32(st + a_bytes));
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk)
+          tc_mma_bf16(tmem_base, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2), idesc,
+                      (kb | kk) != 0 ? 1u : 0u);
+        tc_commit(&empty[stage]);
+        if (++stage == stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok) tc_commit(tfull);
+      tc_commit(done);
+      mbar_wait(done, 0, nullptr, status, limit_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ one thread per token --
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const int t = tok0 + r;
+    const bool valid = t < T;
+    const int ld = E + 1;
+    float* s_p = reinterpret_cast<float*>(ring);  // [128][E+1], reuses the ring after the MMAs
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull, 0, s_abort, status, limit_ns));
+    tc_fence_after();
+    const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    const int nchunks = (E + 31) >> 5;
+
+    // pass 1: logits (+ bias) into the probability tile, row maximum
+    float m = -INFINITY;
+    bool finite = true;
+    for (int c = 0; c < nchunks; ++c) {
+      uint32_t v[32];
+      __syncwarp();
+      if (ok) {
+        tmem_ld_x32(trow + c * 32, v);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0u;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int e = c * 32 + i;
+        if (e < E) {
+          float l = __uint_as_float(v[i]);
+          if (br) l += br[e];
+          finite = finite && isfinite(l);
+          m = fmaxf(m, l);
+          s_p[r * ld + e] = l;
+        }
+      }
+    }
+    // pass 2: exponentials and their sum (expert order)
+    float s = 0.f;
+    for (int e = 0; e < E; ++e) {
+      const float ex = expf(s_p[r * ld + e] - m);
+      s_p[r * ld + e] = ex;
+      s += ex;
+    }
+    // pass 3: probabilities and the k best under (p descending, index ascending)
+    float bv[kMaxTopK];
+    int be[kMaxTopK];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      bv[j] = -INFINITY;
+      be[j] = 0x7fffffff;
+    }
+    for (int e = 0; e < E; ++e) {
+      const float p = s_p[r * ld + e] / s;
+      s_p[r * ld + e] = valid ? p : 0.f;
+      const float pv = (p != p) ? -INFINITY : p;
+      if (ahead(pv, e, bv[kMaxTopK - 1], be[kMaxTopK - 1])) {
+        bv[kMaxTopK - 1] = pv;
+        be[kMaxTopK - 1] = e;
+#pragma unroll
+        for (int j = kMaxTopK - 1; j > 0; --j) {
+          if (ahead(bv[j], be[j], bv[j - 1], be[j - 1])) {
+            const float tv = bv[j];
+            bv[j] = bv[j - 1];
+            bv[j - 1] = tv;
+            const int te = be[j];
+            be[j] = be[j - 1];
+            be[j - 1] = te;
+          }
+        }
+      }
+    }
+    if (valid && !finite) atomicOr(status, MOE_DEV_NONFINITE);
+    float psel = 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j)
+      if (j < k) psel += bv[j];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j < k) {
+        float g;
+        if (!renorm)
+          g = bv[j];
+        else if (psel > 0.f)
+          g = bv[j] / psel;
+        else
+          g = 1.0f / (float)k;
+        if (valid) {
+          topk_idx[(size_t)t * k + j] = be[j];
+          topk_gate[(size_t)t * k + j] = g;
+        }
+        s_idx[r * kMaxTopK + j] = valid ? be[j] : -1;
+      }
+    }
+    __syncwarp();
+
+    // per-warp histogram and in-warp rank of each assignment
+    uint32_t myrank[kMaxTopK];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) myrank[j] = 0;
+    for (int e = 0; e < E; ++e) {
+      int jhit = -1;
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j)
+        if (j < k && s_idx[r * kMaxTopK + j] == e) jhit = j;
+      const uint32_t mask = __ballot_sync(0xffffffffu, jhit >= 0);
+      const uint32_t rk = __popc(mask & ((1u << lane) - 1u));
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j)
+        if (j == jhit) myrank[j] = rk;
+      if (lane == 0) s_wcnt[q * E + e] = __popc(mask);
+    }
+    epi_bar();
+    // block totals and the exclusive prefix over the 4 row quarters
+    for (int e = r; e < E; e += kRB) {
+      int run = 0;
+      for (int qq = 0; qq < 4; ++qq) {
+        const int c = s_wcnt[qq * E + e];
+        s_wcnt[qq * E + e] = run;
+        run += c;
+      }
+      blk_cnt[(size_t)blockIdx.x * E + e] = run;
+      float ps = 0.f;
+      for (int rr = 0; rr < kRB; ++rr) ps += s_p[rr * ld + e];
+      blk_psum[(size_t)blockIdx.x * E + e] = ps;
+    }
+    epi_bar();
+    if (valid) {
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j)
+        if (j < k) lrank[(size_t)t * k + j] = (int)myrank[j] + s_wcnt[q * E + be[j]];
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_router_tc(const void* x, const void* w_router, const float* b_router, int T, int d, int E, int k,
+                             int renorm, int32_t* topk_idx, float* topk_gate, int32_t* lrank, int32_t* blk_cnt,
+                             float* blk_psum, int32_t* status, cudaStream_t stream) {
+  const RouterCfg c = router_cfg(E);
+  CUtensorMap tmX, tmW;
+  if (!make_tmap_bf16_2d(&tmX, x, (uint64_t)T, (uint64_t)d, kRB) ||
+      !make_tmap_bf16_2d(&tmW, w_router, (uint64_t)E, (uint64_t)d, (uint32_t)c.npad))
+    return cudaErrorInvalidValue;
+  cudaError_t err = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, c.smem_bytes);
+  if (err != cudaSuccess) return err;
+  const int nb = (T + kRB - 1) / kRB;
+  router_tc_kernel<<<nb, kGemmThreads, c.smem_bytes, stream>>>(tmX, tmW, b_router, T, d, E, k, renorm, c.npad,
+                                                               c.stages, c.stage_bytes, c.tmem_cols, topk_idx,
+                                                               topk_gate, lrank, blk_cnt, blk_psum, status,
+                                                               kWaitLimitNs);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -9,8 +9,11 @@ Rules:
     checked against the oracle evaluated at the GPU's choice.
   * Counts and the dispatch order are checked exactly against the oracle's
     own dispatch of the GPU's indices (integer work is bit-exact).
-  * Gates within 2e-6 absolute (fp32 softmax and division), the statistic
-    within 1e-4 absolute.
+  * Gates within 2e-6 absolute for fp32 and 2e-5 for bf16, the statistic
+    within 1e-4 absolute. A gate is a softmax ratio of two or more logits,
+    |dg| <= max|dl| / 2, and the bf16 router accumulates its d products on the
+    tensor cores in fp32 (not round-to-nearest at every add), which leaves a
+    logit error of a few 1e-5 at d = 4096 (a relative 1e-6 of sum |x_c w_c|).
   * Outputs: max-abs <= 2e-2 and relative Frobenius <= 1e-2 for bf16;
     both <= 1e-4 for fp32.
 """
@@ -23,6 +26,7 @@ import oracle
 
 GAP_THRESHOLD = 1e-4
 TOL = {"bf16": dict(max_abs=2e-2, rel_fro=1e-2), "f32": dict(max_abs=1e-4, rel_fro=1e-4)}
+GATE_TOL = {"bf16": 2e-5, "f32": 2e-6}
 
 
 def _np(t):
@@ -67,7 +71,7 @@ def check(inp, res, perm, k, renorm, dtype, tokens=None, h_round=False, report=N
     gate_ref = oracle.gates_for(probs, idx_g, renorm)
     gerr = float(np.abs(gate_g - gate_ref).max()) if T else 0.0
     rep["gate_max_abs"] = gerr
-    assert gerr <= 2e-6, f"gate error {gerr}"
+    assert gerr <= GATE_TOL[dtype], f"gate error {gerr}"
 
     # --- counts, statistic, dispatch order (exact) -------------------------
     counts_ref, _, aux_ref = oracle.stats(probs, idx_g)
