@@ -32,8 +32,8 @@ from sparse_mixture_experts_renorm_b200.workloads import WORKLOADS, make_inputs,
 METRIC = "MoE-layer tokens/s and TFLOP/s (active) at 1 B200; % of bf16 TC / HBM roofline"
 KERNELS = ["router_topk", "route_scan", "permute", "grouped_gemm_gateup_swiglu", "grouped_gemm_down", "combine"]
 KERNEL_SOURCES = {
-    "router_topk": "router.cu", "route_scan": "router.cu", "permute": "permute.cu", "combine": "permute.cu",
-    "grouped_gemm_gateup_swiglu": "gemm_tc.cu", "grouped_gemm_down": "gemm_tc.cu",
+    "router_topk": "router_tc.cu", "route_scan": "router.cu", "permute": "permute.cu", "combine": "permute.cu",
+    "grouped_gemm_gateup_swiglu": "gemm_tc2.cu", "grouped_gemm_down": "gemm_tc2.cu",
 }
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -48,6 +48,8 @@ def load_peaks():
 
 def source_hash(kernel):
     src = os.path.join(ROOT, "sparse_mixture_experts_renorm_b200", "csrc", KERNEL_SOURCES[kernel])
+    if not os.path.exists(src):
+        return None
     with open(src, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 

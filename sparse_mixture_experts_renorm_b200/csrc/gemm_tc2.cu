@@ -1,0 +1,412 @@
+// gemm_tc2.cu — kernel (c): the two grouped expert GEMMs on tcgen05 with a
+// pair of CTAs (cta_group::2) per 256 x 256 output tile.
+//
+//   mode 0 (gate/up):  H[r, :] = SiLU(Xp[r] . W_gate[e]^T) * (Xp[r] . W_up[e]^T)
+//   mode 1 (down):     Y[r, :] = H[r] . W_down[e]^T
+//
+// for every dispatched row r of expert e (axonml-nn layers/moe.rs,
+// Expert::forward: down(SiLU(gate(x)) * up(x)); Model Architecture Patterns,
+// "SwiGLU FFN"). Rows are expert-contiguous, so expert e's rows form the M
+// dimension of its own GEMM; 256-row tiles that run past the expert's last row
+// compute on neighbouring rows (or TMA zero fill) and are masked at the store.
+//
+// A cluster of two CTAs on two SMs owns one tile at a time. Each CTA stages
+// its own 128 rows of A and one half of the 256 B rows (mode 0: CTA 0 the 128
+// gate rows, CTA 1 the 128 up rows of the same hidden units; mode 1: 128
+// W_down rows each) through a 6-stage TMA ring, both signalling the leading
+// CTA's barrier. One thread of the leading CTA issues 256x256x16 UMMAs that
+// read A and B from both CTAs' shared memory and write each CTA's 128 rows of
+// the fp32 accumulator into that CTA's TMEM (double-buffered, 2 x 256
+// columns); commits are multicast to both CTAs. Each CTA's 4 epilogue warps
+// drain their own TMEM lanes (SwiGLU + bf16 in mode 0, fp32 in mode 1) and
+// release the accumulator to the leader. Per UMMA FLOP this moves a third
+// fewer bytes from L2 to shared memory than one CTA per 128 x 256 tile.
+//
+// Persistent: clusters walk a device-side tile list built from the routing
+// counts (experts in order; n-tile outer, m-tile inner inside an expert, so
+// clusters running together share weight tiles in L2). Every wait is bounded.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kStages2 = 6;
+constexpr int kHalfBytes = 128 * kBK * 2;          // 16 KB: 128 rows x 64 bf16
+constexpr int kStage2Bytes = 2 * kHalfBytes;       // A half + B half per CTA
+constexpr int kGemm2SmemBytes = kStages2 * kStage2Bytes + 1024 + 4096;
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t num_clusters_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Shared::cluster address of the same shared variable in CTA `rank`.
+__device__ __forceinline__ uint32_t map_to_cta(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA tile load into this CTA's shared memory whose completion is counted on
+// the barrier at `bar_cluster` (the leading CTA's).
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
+                                                 int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* smem_result, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_result)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on the barrier at this offset in both CTAs of the pair once the
+// pair's UMMAs issued so far have completed.
+__device__ __forceinline__ void tc_commit_pair_both(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"((uint16_t)0x3)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair_local(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+struct TileCoord {
+  int e, m, n;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(int tile, int n_tiles, const int* s_mt, int E) {
+  const int q = tile / n_tiles;
+  int lo = 0, hi = E;  // s_mt[lo] <= q < s_mt[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s_mt[mid] <= q)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  TileCoord c;
+  c.e = lo;
+  const int mt_e = s_mt[lo + 1] - s_mt[lo];
+  const int local = tile - s_mt[lo] * n_tiles;
+  c.n = local / mt_e;
+  c.m = local - c.n * mt_e;
+  return c;
+}
+
+__device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + __expf(-z)); }
+
+template <int kMode>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                            const __grid_constant__ CUtensorMap tmB1, const int32_t* __restrict__ offsets,
+                            const int32_t* __restrict__ mtile256, int E, int N, int K, void* __restrict__ out,
+                            int32_t* status, uint64_t limit_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;                              // [stages][128 x 64]
+  uint8_t* sB = smem + kStages2 * kHalfBytes;      // [stages][128 x 64]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages2 * kStage2Bytes);
+  uint64_t* full = bars;                 // leader: A+B bytes of both CTAs
+  uint64_t* empty = bars + kStages2;     // both: stage consumed by the pair's UMMAs
+  uint64_t* tfull = bars + 2 * kStages2; // both: accumulator ready
+  uint64_t* tempty = tfull + 2;          // leader: 256 epilogue arrivals
+  uint64_t* done = tempty + 2;           // leader: every UMMA completed
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  int* s_off = reinterpret_cast<int*>(s_tmem + 4);  // [E+1]
+  int* s_mt = s_off + (E + 1);                       // [E+1]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cid = (int)cluster_id_x();
+  const int ncl = (int)num_clusters_x();
+  const int n_tiles = kMode == 0 ? (N + 127) / 128 : (N + 255) / 256;
+  const int KB = K / kBK;
+
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) {
+    s_off[i] = offsets[i];
+    s_mt[i] = mtile256[i];
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages2; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 256);
+    }
+    mbar_init(done, 1);
+    *s_abort = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    if (kMode == 0) tma_prefetch_desc(&tmB1);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(s_tmem, 2 * kBN);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer's barriers are initialised before any remote signal
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  const int total = s_mt[E] * n_tiles;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      const CUtensorMap* tmB = (kMode == 0 && !leader) ? &tmB1 : &tmB0;
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int tile = cid; ok && tile < total; tile += ncl) {
+        const TileCoord tc = decode_tile(tile, n_tiles, s_mt, E);
+        const int arow = s_off[tc.e] + tc.m * 256 + (int)rank * 128;
+        const int brow = kMode == 0 ? tc.e * N + tc.n * 128 : tc.e * N + tc.n * 256 + (int)rank * 128;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, s_abort, status, limit_ns)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fbar = map_to_cta(&full[stage], 0);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kStage2Bytes);
+          tma_load_2d_pair(sA + stage * kHalfBytes, &tmA, fbar, kb * kBK, arow);
+          tma_load_2d_pair(sB + stage * kHalfBytes, tmB, fbar, kb * kBK, brow);
+          ++issued;
+          if (++stage == kStages2) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Loads land on the leader's barriers: the leader waits for the last
+      // phase of each stage it armed (these cover both CTAs' bytes).
+      if (leader) {
+        const int n = issued < kStages2 ? issued : kStages2;
+        for (int i = 0; i < n; ++i) {
+          if (stage == 0) {
+            stage = kStages2;
+            phase ^= 1u;
+          }
+          --stage;
+          mbar_wait(&full[stage], phase, nullptr, status, limit_ns);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------ MMA issuer (leader only) --
+    if (leader && lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(256, kBN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = cid; ok && tile < total; tile += ncl) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, s_abort, status, limit_ns)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, s_abort, status, limit_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = sw128_kmajor_desc(smem_u32(sA + stage * kHalfBytes));
+          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sB + stage * kHalfBytes));
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            tc_mma_bf16_pair(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2),
+                             idesc, (kb | kk) != 0 ? 1u : 0u);
+          tc_commit_pair_both(&empty[stage]);
+          if (++stage == kStages2) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_both(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      tc_commit_pair_local(done);
+      mbar_wait(done, 0, nullptr, status, limit_ns);
+    }
+    __syncwarp();
+  } else {
+    // --------------------------------------------------------- epilogue --
+    const int q = warp & 3;
+    const int r = q * 32 + lane;  // this CTA's row within its 128-row half
+    const uint32_t tempty_leader0 = map_to_cta(&tempty[0], 0);
+    const uint32_t tempty_leader1 = map_to_cta(&tempty[1], 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = cid; tile < total; tile += ncl) {
+      const TileCoord tc = decode_tile(tile, n_tiles, s_mt, E);
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, s_abort, status, limit_ns))) break;
+      tc_fence_after();
+      const int cnt = s_off[tc.e + 1] - s_off[tc.e];
+      const int row_in_expert = tc.m * 256 + (int)rank * 128 + r;
+      const bool row_ok = row_in_expert < cnt;
+      const size_t grow = static_cast<size_t>(s_off[tc.e]) + static_cast<size_t>(row_in_expert);
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kBN);
+      if (kMode == 0) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t g[32], u[32];
+          __syncwarp();
+          tmem_ld_x32(tbase + c * 32, g);
+          tmem_ld_x32(tbase + 128 + c * 32, u);
+          tmem_ld_wait();
+          const int col0 = tc.n * 128 + c * 32;
+          if (row_ok && col0 < N) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float h0 = silu_f32(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
+              const float h1 = silu_f32(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+              pk[i] = pack_bf16x2(h0, h1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + grow * N + col0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld_x32(tbase + c * 32, v);
+          tmem_ld_wait();
+          const int col0 = tc.n * 256 + c * 32;
+          if (row_ok && col0 < N) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + grow * N + col0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          }
+        }
+      }
+      __syncwarp();
+      tc_fence_before();
+      mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no CTA leaves while its peer may still touch its shared memory or TMEM
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 2 * kBN);
+  }
+}
+
+int max_active_pairs(const void* kern, int smem) {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+template <int kMode>
+cudaError_t launch_tc2(const CUtensorMap& tmA, const CUtensorMap& tmB0, const CUtensorMap& tmB1,
+                       const int32_t* offsets, const int32_t* mtile256, int R, int E, int N, int K, void* out,
+                       int32_t* status, cudaStream_t stream) {
+  auto kern = grouped_gemm_tc2_kernel<kMode>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemm2SmemBytes);
+  if (err != cudaSuccess) return err;
+  const int pairs = max_active_pairs(reinterpret_cast<const void*>(kern), kGemm2SmemBytes);
+  if (pairs <= 0) return cudaErrorInvalidConfiguration;
+  const int n_tiles = kMode == 0 ? (N + 127) / 128 : (N + 255) / 256;
+  const long long max_tiles = (long long)(R / 256 + E) * n_tiles;
+  const int clusters = (int)(max_tiles < pairs ? max_tiles : pairs);
+  if (clusters <= 0) return cudaSuccess;
+  kern<<<2 * clusters, kGemmThreads, kGemm2SmemBytes, stream>>>(tmA, tmB0, tmB1, offsets, mtile256, E, N, K, out,
+                                                               status, kWaitLimitNs);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_gateup_tc2(const CUtensorMap& tm_xp, const CUtensorMap& tm_wg, const CUtensorMap& tm_wu,
+                                   const int32_t* offsets, const int32_t* mtile256, int R, int E, int I, int d, void* h,
+                                   int32_t* status, cudaStream_t stream) {
+  return launch_tc2<0>(tm_xp, tm_wg, tm_wu, offsets, mtile256, R, E, I, d, h, status, stream);
+}
+
+cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_h, const CUtensorMap& tm_wd, const int32_t* offsets,
+                                 const int32_t* mtile256, int R, int E, int I, int d, float* y, int32_t* status,
+                                 cudaStream_t stream) {
+  return launch_tc2<1>(tm_h, tm_wd, tm_wd, offsets, mtile256, R, E, d, I, y, status, stream);
+}
+
+}  // namespace moe

@@ -72,19 +72,6 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-int device_sm_count() {
-  static int cache[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (dev < 0 || dev >= 64) return 0;
-  if (cache[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    cache[dev] = n;
-  }
-  return cache[dev];
-}
-
 }  // namespace
 
 Workspace workspace_layout(int T, int d, int E, int k, int I, moe_dtype dtype) {
@@ -96,7 +83,7 @@ Workspace workspace_layout(int T, int d, int E, int k, int I, moe_dtype dtype) {
   w.status = o;   o = align256(o + 4);
   w.offsets = o;  o = align256(o + 4 * (size_t)(E + 1));
   w.counts = o;   o = align256(o + 4 * (size_t)E);
-  w.mtile128 = o; o = align256(o + 4 * (size_t)(E + 1));
+  w.mtile = o;    o = align256(o + 4 * (size_t)(E + 1));
   w.aux = o;      o = align256(o + 4);
   w.blk_cnt = o;  o = align256(o + 4 * nb * E);
   w.blk_psum = o; o = align256(o + 4 * nb * E);
@@ -197,7 +184,7 @@ moe_status forward_impl(const void* x, const void* w_router, const float* b_rout
   }
 
   int32_t* offsets = reinterpret_cast<int32_t*>(ws + w.offsets);
-  int32_t* mtile = reinterpret_cast<int32_t*>(ws + w.mtile128);
+  int32_t* mtile = reinterpret_cast<int32_t*>(ws + w.mtile);
   int32_t* blk_cnt = reinterpret_cast<int32_t*>(ws + w.blk_cnt);
   float* blk_psum = reinterpret_cast<float*>(ws + w.blk_psum);
   int32_t* lrank = reinterpret_cast<int32_t*>(ws + w.lrank);
@@ -221,20 +208,18 @@ moe_status forward_impl(const void* x, const void* w_router, const float* b_rout
   if (err != cudaSuccess) return fail_cuda(err, "permute kernel");
 
   if (dtype == MOE_BF16) {
-    const int sms = device_sm_count();
-    if (sms <= 0) return fail(MOE_ERR_CUDA, "could not query the SM count of the current device");
     CUtensorMap tm_xp, tm_wg, tm_wu, tm_h, tm_wd;
     if (!make_tmap_bf16_2d(&tm_xp, xp, (uint64_t)R, (uint64_t)d, kBM) ||
         !make_tmap_bf16_2d(&tm_wg, w_gate, (uint64_t)E * I, (uint64_t)d, 128) ||
         !make_tmap_bf16_2d(&tm_wu, w_up, (uint64_t)E * I, (uint64_t)d, 128) ||
         !make_tmap_bf16_2d(&tm_h, h, (uint64_t)R, (uint64_t)I, kBM) ||
-        !make_tmap_bf16_2d(&tm_wd, w_down, (uint64_t)E * d, (uint64_t)I, kBN))
+        !make_tmap_bf16_2d(&tm_wd, w_down, (uint64_t)E * d, (uint64_t)I, 128))
       return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point unavailable or bad pointer)");
     marks.mark(stream);
-    err = launch_gemm_gateup_tc(tm_xp, tm_wg, tm_wu, offsets, mtile, R, E, I, d, h, status, sms, stream);
+    err = launch_gemm_gateup_tc2(tm_xp, tm_wg, tm_wu, offsets, mtile, R, E, I, d, h, status, stream);
     if (err != cudaSuccess) return fail_cuda(err, "gate/up grouped GEMM");
     marks.mark(stream);
-    err = launch_gemm_down_tc(tm_h, tm_wd, offsets, mtile, R, E, I, d, y, status, sms, stream);
+    err = launch_gemm_down_tc2(tm_h, tm_wd, offsets, mtile, R, E, I, d, y, status, stream);
     if (err != cudaSuccess) return fail_cuda(err, "down grouped GEMM");
   } else {
     marks.mark(stream);

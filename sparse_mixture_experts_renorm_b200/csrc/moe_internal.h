@@ -21,7 +21,8 @@ constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 8;
 
 // tcgen05 grouped GEMM tiling.
-constexpr int kBM = 128;          // rows (dispatched tokens) per tile = UMMA M
+constexpr int kTileM = 256;       // rows (dispatched tokens) per tile of the CTA pair
+constexpr int kBM = 128;          // rows per CTA
 constexpr int kBN = 256;          // UMMA N: 128 gate + 128 up columns, or 256 down columns
 constexpr int kBK = 64;           // K per pipeline stage (one 128-byte swizzle row of bf16)
 constexpr int kStages = 4;        // shared-memory pipeline depth
@@ -43,7 +44,7 @@ struct Workspace {
   size_t status;      // int32 [1]     device status word used when the caller passes none
   size_t offsets;     // int32 [E+1]   first dispatched row of each expert
   size_t counts;      // int32 [E]     assignments per expert (when the caller passes none)
-  size_t mtile128;    // int32 [E+1]   prefix of ceil(count/128) (tcgen05 tile schedule)
+  size_t mtile;       // int32 [E+1]   prefix of ceil(count/kTileM) (tcgen05 tile schedule)
   size_t aux;         // fp32  [1]     statistic (when the caller passes none)
   size_t blk_cnt;     // int32 [nb*E]  per-router-block counts, then per-block base rows
   size_t blk_psum;    // fp32  [nb*E]  per-router-block sums of probabilities
@@ -79,7 +80,7 @@ cudaError_t launch_router_tc(const void* x, const void* w_router, const float* b
                              float* blk_psum, int32_t* status, cudaStream_t stream);
 
 cudaError_t launch_route_scan(int nb, int T, int E, int k, int32_t* blk_cnt, const float* blk_psum, int32_t* counts,
-                              int32_t* offsets, int32_t* mtile128, float* aux, cudaStream_t stream);
+                              int32_t* offsets, int32_t* mtile, float* aux, cudaStream_t stream);
 
 cudaError_t launch_permute(moe_dtype dtype, const void* x, int T, int d, int E, int k, int rb, const int32_t* topk_idx,
                            const int32_t* lrank, const int32_t* blk_base, int32_t* perm_tok, int32_t* inv,
@@ -88,14 +89,14 @@ cudaError_t launch_permute(moe_dtype dtype, const void* x, int T, int d, int E, 
 cudaError_t launch_combine(int T, int d, int k, const float* y, const int32_t* inv, const float* topk_gate,
                            float* out, int32_t* status, cudaStream_t stream);
 
-// tcgen05 grouped GEMMs (bf16). mode 0: H = SiLU(Xp Wg^T) * (Xp Wu^T) per
-// expert; mode 1: Y = H Wd^T per expert.
-cudaError_t launch_gemm_gateup_tc(const CUtensorMap& tm_xp, const CUtensorMap& tm_wg, const CUtensorMap& tm_wu,
-                                  const int32_t* offsets, const int32_t* mtile128, int R, int E, int I, int d,
-                                  void* h, int32_t* status, int num_sms, cudaStream_t stream);
-cudaError_t launch_gemm_down_tc(const CUtensorMap& tm_h, const CUtensorMap& tm_wd, const int32_t* offsets,
-                                const int32_t* mtile128, int R, int E, int I, int d, float* y, int32_t* status,
-                                int num_sms, cudaStream_t stream);
+// tcgen05 grouped GEMMs (bf16), one CTA pair per 256 x 256 tile. mode 0:
+// H = SiLU(Xp Wg^T) * (Xp Wu^T) per expert; mode 1: Y = H Wd^T per expert.
+cudaError_t launch_gemm_gateup_tc2(const CUtensorMap& tm_xp, const CUtensorMap& tm_wg, const CUtensorMap& tm_wu,
+                                   const int32_t* offsets, const int32_t* mtile, int R, int E, int I, int d, void* h,
+                                   int32_t* status, cudaStream_t stream);
+cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_h, const CUtensorMap& tm_wd, const int32_t* offsets,
+                                 const int32_t* mtile, int R, int E, int I, int d, float* y, int32_t* status,
+                                 cudaStream_t stream);
 
 // fp32 SIMT grouped GEMMs.
 cudaError_t launch_gemm_gateup_simt(const float* xp, const float* wg, const float* wu, const int32_t* offsets,

@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(
 __global__ void __launch_bounds__(1024) route_scan_kernel(int nb, int T, int E, int k, int32_t* __restrict__ blk_cnt,
                                                           const float* __restrict__ blk_psum,
                                                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                                                          int32_t* __restrict__ mtile128, float* __restrict__ aux) {
+                                                          int32_t* __restrict__ mtile, float* __restrict__ aux) {
   __shared__ int s_cnt[1024];
   __shared__ double s_ps[1024];
   __shared__ int s_tot[kMaxExperts];
@@ -225,14 +225,14 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int nb, int T, int E, 
     for (int ee = 0; ee < E; ++ee) {
       s_off[ee] = off;
       offsets[ee] = off;
-      mtile128[ee] = mt;
+      mtile[ee] = mt;
       if (counts) counts[ee] = s_tot[ee];
       a += ((double)s_tot[ee] / ((double)T * (double)k)) * (s_ptot[ee] / (double)T);
       off += s_tot[ee];
-      mt += (s_tot[ee] + kBM - 1) / kBM;
+      mt += (s_tot[ee] + kTileM - 1) / kTileM;
     }
     offsets[E] = off;
-    mtile128[E] = mt;
+    mtile[E] = mt;
     s_off[E] = off;
     if (aux) *aux = (float)((double)E * a);
   }
@@ -266,8 +266,8 @@ cudaError_t launch_router(moe_dtype dtype, const void* x, const void* w_router, 
 }
 
 cudaError_t launch_route_scan(int nb, int T, int E, int k, int32_t* blk_cnt, const float* blk_psum, int32_t* counts,
-                              int32_t* offsets, int32_t* mtile128, float* aux, cudaStream_t stream) {
-  route_scan_kernel<<<1, 1024, 0, stream>>>(nb, T, E, k, blk_cnt, blk_psum, counts, offsets, mtile128, aux);
+                              int32_t* offsets, int32_t* mtile, float* aux, cudaStream_t stream) {
+  route_scan_kernel<<<1, 1024, 0, stream>>>(nb, T, E, k, blk_cnt, blk_psum, counts, offsets, mtile, aux);
   return cudaGetLastError();
 }
 
