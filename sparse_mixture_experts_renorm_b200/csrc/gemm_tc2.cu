@@ -33,7 +33,11 @@ namespace {
 constexpr int kStages2 = 6;
 constexpr int kHalfBytes = 128 * kBK * 2;          // 16 KB: 128 rows x 64 bf16
 constexpr int kStage2Bytes = 2 * kHalfBytes;       // A half + B half per CTA
-constexpr int kGemm2SmemBytes = kStages2 * kStage2Bytes + 1024 + 4096;
+constexpr int kSmallRows = 16;                     // B box for tiles of <= 32 tokens
+constexpr int kEpiBytes = 2 * 64 * 33 * 4;  // gate and up halves of a 32-token chunk (mode 0)
+constexpr int kGemm2SmemBytes = kStages2 * kStage2Bytes + kEpiBytes + 1024 + 4096;
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -133,15 +137,17 @@ __device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + __expf(-
 
 template <int kMode>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
-    grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                            const __grid_constant__ CUtensorMap tmB1, const int32_t* __restrict__ offsets,
-                            const int32_t* __restrict__ mtile256, int E, int N, int K, void* __restrict__ out,
-                            int32_t* status, uint64_t limit_ns) {
+    grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                            const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBs,
+                            const int32_t* __restrict__ offsets, const int32_t* __restrict__ mtile256, int E,
+                            int N, int K, void* __restrict__ out, int32_t* status, uint64_t limit_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;                              // [stages][128 x 64]
-  uint8_t* sB = smem + kStages2 * kHalfBytes;      // [stages][128 x 64]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages2 * kStage2Bytes);
+  uint8_t* sA = smem;                           // [stages][128 weight rows x 64]
+  uint8_t* sB = smem + kStages2 * kHalfBytes;   // [stages][<=128 token rows x 64]
+  float* sG = reinterpret_cast<float*>(smem + kStages2 * kStage2Bytes);  // [64][33] gate chunk (mode 0)
+  float* sU = sG + 64 * 33;                                              // [64][33] up chunk (mode 0)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages2 * kStage2Bytes + kEpiBytes);
   uint64_t* full = bars;                 // leader: A+B bytes of both CTAs
   uint64_t* empty = bars + kStages2;     // both: stage consumed by the pair's UMMAs
   uint64_t* tfull = bars + 2 * kStages2; // both: accumulator ready
@@ -157,7 +163,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const bool leader = rank == 0;
   const int cid = (int)cluster_id_x();
   const int ncl = (int)num_clusters_x();
-  const int n_tiles = kMode == 0 ? (N + 127) / 128 : (N + 255) / 256;
+  // weight blocks per expert: 128 hidden units (gate + up rows) or 256 output features
+  const int n_wb = kMode == 0 ? (N + 127) / 128 : (N + 255) / 256;
   const int KB = K / kBK;
 
   for (int i = threadIdx.x; i <= E; i += blockDim.x) {
@@ -178,9 +185,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     fence_mbarrier_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB0);
-    if (kMode == 0) tma_prefetch_desc(&tmB1);
+    tma_prefetch_desc(&tmA0);
+    if (kMode == 0) tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmBs);
   }
   if (warp == 1) {
     tmem_alloc_pair(s_tmem, 2 * kBN);
@@ -191,29 +199,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   cluster_sync();  // the peer's barriers are initialised before any remote signal
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
-  const int total = s_mt[E] * n_tiles;
+  const int total = s_mt[E] * n_wb;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
     if (lane == 0) {
-      const CUtensorMap* tmB = (kMode == 0 && !leader) ? &tmB1 : &tmB0;
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
       for (int tile = cid; ok && tile < total; tile += ncl) {
-        const TileCoord tc = decode_tile(tile, n_tiles, s_mt, E);
-        const int arow = s_off[tc.e] + tc.m * 256 + (int)rank * 128;
-        const int brow = kMode == 0 ? tc.e * N + tc.n * 128 : tc.e * N + tc.n * 256 + (int)rank * 128;
+        const TileCoord tc = decode_tile(tile, n_wb, s_mt, E);
+        const int ntok = min(256, s_off[tc.e + 1] - s_off[tc.e] - tc.m * 256);
+        const int half = ((ntok + 15) & ~15) >> 1;  // token rows of B held by each CTA
+        const bool small = half <= kSmallRows;
+        const int brow = s_off[tc.e] + tc.m * 256 + (int)rank * half;
+        const int arow = kMode == 0 ? tc.e * N + tc.n * 128 + (int)rank * 64 : tc.e * N + tc.n * 256 + (int)rank * 128;
+        const uint32_t bytes = 2u * (uint32_t)(kHalfBytes + (small ? kSmallRows * 128 : kHalfBytes));
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, s_abort, status, limit_ns)) {
             ok = false;
             break;
           }
           const uint32_t fbar = map_to_cta(&full[stage], 0);
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * kStage2Bytes);
-          tma_load_2d_pair(sA + stage * kHalfBytes, &tmA, fbar, kb * kBK, arow);
-          tma_load_2d_pair(sB + stage * kHalfBytes, tmB, fbar, kb * kBK, brow);
+          if (leader) mbar_arrive_expect_tx(&full[stage], bytes);
+          if (kMode == 0) {
+            // rows 0-63: gate rows of this CTA's 64 hidden units, 64-127: up rows
+            tma_load_2d_pair(sA + stage * kHalfBytes, &tmA0, fbar, kb * kBK, arow);
+            tma_load_2d_pair(sA + stage * kHalfBytes + kHalfBytes / 2, &tmA1, fbar, kb * kBK, arow);
+          } else {
+            tma_load_2d_pair(sA + stage * kHalfBytes, &tmA0, fbar, kb * kBK, arow);
+          }
+          tma_load_2d_pair(sB + stage * kHalfBytes, small ? &tmBs : &tmB, fbar, kb * kBK, brow);
           ++issued;
           if (++stage == kStages2) {
             stage = 0;
@@ -239,13 +256,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------ MMA issuer (leader only) --
     if (leader && lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(256, kBN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = cid; ok && tile < total; tile += ncl) {
+        const TileCoord tc = decode_tile(tile, n_wb, s_mt, E);
+        const int ntok = min(256, s_off[tc.e + 1] - s_off[tc.e] - tc.m * 256);
+        const uint32_t idesc = idesc_bf16_f32(256, (ntok + 15) & ~15);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, s_abort, status, limit_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
@@ -280,57 +299,70 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // --------------------------------------------------------- epilogue --
+    // TMEM lane = weight row of this CTA, column = token of the tile.
     const int q = warp & 3;
-    const int r = q * 32 + lane;  // this CTA's row within its 128-row half
     const uint32_t tempty_leader0 = map_to_cta(&tempty[0], 0);
     const uint32_t tempty_leader1 = map_to_cta(&tempty[1], 0);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = cid; tile < total; tile += ncl) {
-      const TileCoord tc = decode_tile(tile, n_tiles, s_mt, E);
+      const TileCoord tc = decode_tile(tile, n_wb, s_mt, E);
+      const int ntok = min(256, s_off[tc.e + 1] - s_off[tc.e] - tc.m * 256);
+      const size_t row0 = static_cast<size_t>(s_off[tc.e]) + static_cast<size_t>(tc.m * 256);
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, s_abort, status, limit_ns))) break;
       tc_fence_after();
-      const int cnt = s_off[tc.e + 1] - s_off[tc.e];
-      const int row_in_expert = tc.m * 256 + (int)rank * 128 + r;
-      const bool row_ok = row_in_expert < cnt;
-      const size_t grow = static_cast<size_t>(s_off[tc.e]) + static_cast<size_t>(row_in_expert);
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kBN);
+      const int nchunks = (ntok + 31) >> 5;
       if (kMode == 0) {
+        // TMEM lanes 0-63 hold the gate rows, 64-127 the up rows of this
+        // CTA's 64 hidden units. Per 32-token chunk both halves go to shared
+        // memory; then every thread finishes 16 (token, unit) pairs and
+        // writes them as two 16-byte vectors of H.
+        const int j = (q & 1) * 32 + lane;
+        float* sdst = (q < 2 ? sG : sU) + j * 33;
+        const int et = threadIdx.x - 64;  // 0..127
+        const int tt = et >> 2;           // token of the chunk
+        const int ug = (et & 3) * 16;     // first of its 16 units
+        const int hid0 = tc.n * 128 + (int)rank * 64;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t g[32], u[32];
-          __syncwarp();
-          tmem_ld_x32(tbase + c * 32, g);
-          tmem_ld_x32(tbase + 128 + c * 32, u);
-          tmem_ld_wait();
-          const int col0 = tc.n * 128 + c * 32;
-          if (row_ok && col0 < N) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float h0 = silu_f32(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
-              const float h1 = silu_f32(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
-              pk[i] = pack_bf16x2(h0, h1);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + grow * N + col0);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-          }
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
+        for (int c = 0; c < nchunks; ++c) {
           uint32_t v[32];
           __syncwarp();
           tmem_ld_x32(tbase + c * 32, v);
           tmem_ld_wait();
-          const int col0 = tc.n * 256 + c * 32;
-          if (row_ok && col0 < N) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + grow * N + col0);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          for (int t = 0; t < 32; ++t) sdst[t] = __uint_as_float(v[t]);
+          epi_bar();
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int u0 = ug + 2 * i;
+            const float h0 = silu_f32(sG[u0 * 33 + tt]) * sU[u0 * 33 + tt];
+            const float h1 = silu_f32(sG[(u0 + 1) * 33 + tt]) * sU[(u0 + 1) * 33 + tt];
+            pk[i] = pack_bf16x2(h0, h1);
+          }
+          epi_bar();
+          const int tok = c * 32 + tt;
+          if (tok < ntok && hid0 < N) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + (row0 + tok) * N + hid0 + ug);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
+        }
+      } else {
+        // lane = output feature
+        const int o = tc.n * 256 + (int)rank * 128 + q * 32 + lane;
+        float* ybase = static_cast<float*>(out) + row0 * N + o;
+#pragma unroll 1
+        for (int c = 0; c < nchunks; ++c) {
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld_x32(tbase + c * 32, v);
+          tmem_ld_wait();
+          if (o < N) {
+#pragma unroll
+            for (int t = 0; t < 32; ++t)
+              if (c * 32 + t < ntok) ybase[(size_t)(c * 32 + t) * N] = __uint_as_float(v[t]);
           }
         }
       }
@@ -378,35 +410,35 @@ int max_active_pairs(const void* kern, int smem) {
 }
 
 template <int kMode>
-cudaError_t launch_tc2(const CUtensorMap& tmA, const CUtensorMap& tmB0, const CUtensorMap& tmB1,
-                       const int32_t* offsets, const int32_t* mtile256, int R, int E, int N, int K, void* out,
-                       int32_t* status, cudaStream_t stream) {
+cudaError_t launch_tc2(const CUtensorMap& tmA0, const CUtensorMap& tmA1, const CUtensorMap& tmB,
+                       const CUtensorMap& tmBs, const int32_t* offsets, const int32_t* mtile256, int R, int E, int N,
+                       int K, void* out, int32_t* status, cudaStream_t stream) {
   auto kern = grouped_gemm_tc2_kernel<kMode>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemm2SmemBytes);
   if (err != cudaSuccess) return err;
   const int pairs = max_active_pairs(reinterpret_cast<const void*>(kern), kGemm2SmemBytes);
   if (pairs <= 0) return cudaErrorInvalidConfiguration;
-  const int n_tiles = kMode == 0 ? (N + 127) / 128 : (N + 255) / 256;
-  const long long max_tiles = (long long)(R / 256 + E) * n_tiles;
+  const int n_wb = kMode == 0 ? (N + 127) / 128 : (N + 255) / 256;
+  const long long max_tiles = (long long)(R / 256 + E) * n_wb;
   const int clusters = (int)(max_tiles < pairs ? max_tiles : pairs);
   if (clusters <= 0) return cudaSuccess;
-  kern<<<2 * clusters, kGemmThreads, kGemm2SmemBytes, stream>>>(tmA, tmB0, tmB1, offsets, mtile256, E, N, K, out,
-                                                               status, kWaitLimitNs);
+  kern<<<2 * clusters, kGemmThreads, kGemm2SmemBytes, stream>>>(tmA0, tmA1, tmB, tmBs, offsets, mtile256, E, N, K,
+                                                               out, status, kWaitLimitNs);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_gemm_gateup_tc2(const CUtensorMap& tm_xp, const CUtensorMap& tm_wg, const CUtensorMap& tm_wu,
-                                   const int32_t* offsets, const int32_t* mtile256, int R, int E, int I, int d, void* h,
-                                   int32_t* status, cudaStream_t stream) {
-  return launch_tc2<0>(tm_xp, tm_wg, tm_wu, offsets, mtile256, R, E, I, d, h, status, stream);
+cudaError_t launch_gemm_gateup_tc2(const CUtensorMap& tm_wg, const CUtensorMap& tm_wu, const CUtensorMap& tm_xp,
+                                   const CUtensorMap& tm_xp_small, const int32_t* offsets, const int32_t* mtile256,
+                                   int R, int E, int I, int d, void* h, int32_t* status, cudaStream_t stream) {
+  return launch_tc2<0>(tm_wg, tm_wu, tm_xp, tm_xp_small, offsets, mtile256, R, E, I, d, h, status, stream);
 }
 
-cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_h, const CUtensorMap& tm_wd, const int32_t* offsets,
-                                 const int32_t* mtile256, int R, int E, int I, int d, float* y, int32_t* status,
-                                 cudaStream_t stream) {
-  return launch_tc2<1>(tm_h, tm_wd, tm_wd, offsets, mtile256, R, E, d, I, y, status, stream);
+cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_wd, const CUtensorMap& tm_h, const CUtensorMap& tm_h_small,
+                                 const int32_t* offsets, const int32_t* mtile256, int R, int E, int I, int d, float* y,
+                                 int32_t* status, cudaStream_t stream) {
+  return launch_tc2<1>(tm_wd, tm_wd, tm_h, tm_h_small, offsets, mtile256, R, E, d, I, y, status, stream);
 }
 
 }  // namespace moe

@@ -208,18 +208,23 @@ moe_status forward_impl(const void* x, const void* w_router, const float* b_rout
   if (err != cudaSuccess) return fail_cuda(err, "permute kernel");
 
   if (dtype == MOE_BF16) {
-    CUtensorMap tm_xp, tm_wg, tm_wu, tm_h, tm_wd;
-    if (!make_tmap_bf16_2d(&tm_xp, xp, (uint64_t)R, (uint64_t)d, kBM) ||
-        !make_tmap_bf16_2d(&tm_wg, w_gate, (uint64_t)E * I, (uint64_t)d, 128) ||
-        !make_tmap_bf16_2d(&tm_wu, w_up, (uint64_t)E * I, (uint64_t)d, 128) ||
-        !make_tmap_bf16_2d(&tm_h, h, (uint64_t)R, (uint64_t)I, kBM) ||
-        !make_tmap_bf16_2d(&tm_wd, w_down, (uint64_t)E * d, (uint64_t)I, 128))
+    // weights are the UMMA M operand (64 gate + 64 up rows, or 128 down rows
+    // per CTA), dispatched tokens the N operand (128-row boxes, 16-row boxes
+    // for tiles of at most 32 tokens)
+    CUtensorMap tm_wg, tm_wu, tm_wd, tm_xp, tm_xp_s, tm_h, tm_h_s;
+    if (!make_tmap_bf16_2d(&tm_wg, w_gate, (uint64_t)E * I, (uint64_t)d, 64) ||
+        !make_tmap_bf16_2d(&tm_wu, w_up, (uint64_t)E * I, (uint64_t)d, 64) ||
+        !make_tmap_bf16_2d(&tm_wd, w_down, (uint64_t)E * d, (uint64_t)I, 128) ||
+        !make_tmap_bf16_2d(&tm_xp, xp, (uint64_t)R, (uint64_t)d, 128) ||
+        !make_tmap_bf16_2d(&tm_xp_s, xp, (uint64_t)R, (uint64_t)d, 16) ||
+        !make_tmap_bf16_2d(&tm_h, h, (uint64_t)R, (uint64_t)I, 128) ||
+        !make_tmap_bf16_2d(&tm_h_s, h, (uint64_t)R, (uint64_t)I, 16))
       return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point unavailable or bad pointer)");
     marks.mark(stream);
-    err = launch_gemm_gateup_tc2(tm_xp, tm_wg, tm_wu, offsets, mtile, R, E, I, d, h, status, stream);
+    err = launch_gemm_gateup_tc2(tm_wg, tm_wu, tm_xp, tm_xp_s, offsets, mtile, R, E, I, d, h, status, stream);
     if (err != cudaSuccess) return fail_cuda(err, "gate/up grouped GEMM");
     marks.mark(stream);
-    err = launch_gemm_down_tc2(tm_h, tm_wd, offsets, mtile, R, E, I, d, y, status, stream);
+    err = launch_gemm_down_tc2(tm_wd, tm_h, tm_h_s, offsets, mtile, R, E, I, d, y, status, stream);
     if (err != cudaSuccess) return fail_cuda(err, "down grouped GEMM");
   } else {
     marks.mark(stream);

@@ -89,14 +89,15 @@ cudaError_t launch_permute(moe_dtype dtype, const void* x, int T, int d, int E, 
 cudaError_t launch_combine(int T, int d, int k, const float* y, const int32_t* inv, const float* topk_gate,
                            float* out, int32_t* status, cudaStream_t stream);
 
-// tcgen05 grouped GEMMs (bf16), one CTA pair per 256 x 256 tile. mode 0:
-// H = SiLU(Xp Wg^T) * (Xp Wu^T) per expert; mode 1: Y = H Wd^T per expert.
-cudaError_t launch_gemm_gateup_tc2(const CUtensorMap& tm_xp, const CUtensorMap& tm_wg, const CUtensorMap& tm_wu,
-                                   const int32_t* offsets, const int32_t* mtile, int R, int E, int I, int d, void* h,
-                                   int32_t* status, cudaStream_t stream);
-cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_h, const CUtensorMap& tm_wd, const int32_t* offsets,
-                                 const int32_t* mtile, int R, int E, int I, int d, float* y, int32_t* status,
-                                 cudaStream_t stream);
+// tcgen05 grouped GEMMs (bf16) on CTA pairs: 256 weight rows x up to 256
+// dispatched tokens per tile. mode 0: H = SiLU(Xp Wg^T) * (Xp Wu^T) per
+// expert; mode 1: Y = H Wd^T per expert.
+cudaError_t launch_gemm_gateup_tc2(const CUtensorMap& tm_wg, const CUtensorMap& tm_wu, const CUtensorMap& tm_xp,
+                                   const CUtensorMap& tm_xp_small, const int32_t* offsets, const int32_t* mtile,
+                                   int R, int E, int I, int d, void* h, int32_t* status, cudaStream_t stream);
+cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_wd, const CUtensorMap& tm_h, const CUtensorMap& tm_h_small,
+                                 const int32_t* offsets, const int32_t* mtile, int R, int E, int I, int d, float* y,
+                                 int32_t* status, cudaStream_t stream);
 
 // fp32 SIMT grouped GEMMs.
 cudaError_t launch_gemm_gateup_simt(const float* xp, const float* wg, const float* wu, const int32_t* offsets,
