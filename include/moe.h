@@ -153,6 +153,37 @@ moe_status moe_get_permutation(const void* workspace, size_t workspace_bytes, in
                                int32_t* inv, void* stream);
 
 /*
+ * moe_forward_noalloc — moe_forward for callers that cannot allocate device
+ * memory: the same layer, arguments and results, but the scratch lives in a
+ * static array of MOE_NOALLOC_SCRATCH_BYTES inside the library's device image
+ * instead of a caller workspace. The pages have no counterpart; it exists for
+ * callers that run inside an engine or plugin whose host framework owns every
+ * device allocation, or a serving loop that forbids allocation after warm-up.
+ *
+ *   - Shapes whose moe_workspace_size() exceeds MOE_NOALLOC_SCRATCH_BYTES are
+ *     rejected with MOE_ERR_WORKSPACE and a message (nothing is launched);
+ *     16 MiB covers, for example, a 32-token decode batch of the Mixtral
+ *     shape (d=4096, E=8, k=2, I=14336), which needs about 3.3 MB.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture. The call allocates nothing: no cudaMalloc,
+ *     no cudaFree.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind; the library rewrites everything it reads on each call, and
+ *     clears its own status word when status_dev is NULL. Calls that overlap
+ *     on the GPU (concurrent streams, or other threads) race on the array:
+ *     serialise them.
+ *   - Every GPU that loads the library holds the array until the process
+ *     exits.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES (16u << 20)
+moe_status moe_forward_noalloc(const void* x, const void* w_router, const float* b_router,
+                               const void* w_gate, const void* w_up, const void* w_down,
+                               int T, int d, int E, int k, int I, int renorm, moe_dtype dtype,
+                               float* out, int32_t* topk_idx, float* topk_gate, int32_t* counts,
+                               float* aux, int32_t* status_dev, void* stream);
+
+/*
  * moe_last_error_detail — the reason for the calling thread's last non-OK
  * status, NUL-terminated into buf (truncated to n bytes). Returns the full
  * length of the message.

@@ -74,6 +74,15 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 
 }  // namespace
 
+void set_error_detail(const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+}
+
 Workspace workspace_layout(int T, int d, int E, int k, int I, moe_dtype dtype) {
   const size_t R = (size_t)T * k;
   const size_t nb = (size_t)router_blocks(T, MOE_F32);  // the finer blocking of the two routers

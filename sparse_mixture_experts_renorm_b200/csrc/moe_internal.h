@@ -59,6 +59,9 @@ struct Workspace {
 
 Workspace workspace_layout(int T, int d, int E, int k, int I, moe_dtype dtype);
 
+// Sets the calling thread's moe_last_error_detail() message (printf format).
+void set_error_detail(const char* fmt, ...);
+
 inline int router_block_tokens(moe_dtype dtype) { return dtype == MOE_BF16 ? kRouterTokensTc : kRouterTokensSimt; }
 inline int router_blocks(int T, moe_dtype dtype) {
   const int rb = router_block_tokens(dtype);
