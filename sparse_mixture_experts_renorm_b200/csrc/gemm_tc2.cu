@@ -34,7 +34,9 @@ constexpr int kStages2 = 6;
 constexpr int kHalfBytes = 128 * kBK * 2;          // 16 KB: 128 rows x 64 bf16
 constexpr int kStage2Bytes = 2 * kHalfBytes;       // A half + B half per CTA
 constexpr int kSmallRows = 16;                     // B box for tiles of <= 32 tokens
-constexpr int kEpiBytes = 2 * 64 * 33 * 4;  // gate and up halves of a 32-token chunk (mode 0)
+// epilogue staging: gate and up halves of a 32-token chunk (mode 0, 2 x 64 x 33
+// fp32) or one 32 x 32 fp32 transpose tile per epilogue warp (mode 1, 4 x 32 x 36)
+constexpr int kEpiBytes = 4 * 32 * 36 * 4 > 2 * 64 * 33 * 4 ? 4 * 32 * 36 * 4 : 2 * 64 * 33 * 4;
 constexpr int kGemm2SmemBytes = kStages2 * kStage2Bytes + kEpiBytes + 1024 + 4096;
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -147,6 +149,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint8_t* sB = smem + kStages2 * kHalfBytes;   // [stages][<=128 token rows x 64]
   float* sG = reinterpret_cast<float*>(smem + kStages2 * kStage2Bytes);  // [64][33] gate chunk (mode 0)
   float* sU = sG + 64 * 33;                                              // [64][33] up chunk (mode 0)
+  float* sY = sG;                                                        // [4][32][36] (mode 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages2 * kStage2Bytes + kEpiBytes);
   uint64_t* full = bars;                 // leader: A+B bytes of both CTAs
   uint64_t* empty = bars + kStages2;     // both: stage consumed by the pair's UMMAs
@@ -350,19 +353,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
         }
       } else {
-        // lane = output feature
-        const int o = tc.n * 256 + (int)rank * 128 + q * 32 + lane;
-        float* ybase = static_cast<float*>(out) + row0 * N + o;
+        // lane = output feature. Each warp turns its 32 features x 32 tokens
+        // of a chunk around in shared memory and writes token rows of Y as
+        // 16-byte vectors (8 lanes per 128-byte row, 4 rows per instruction).
+        const int o0 = tc.n * 256 + (int)rank * 128 + q * 32;
+        float* tw = sY + (warp - 2) * (32 * 36);
+        const int vr = lane >> 3, vc = (lane & 7) * 4;
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
           uint32_t v[32];
           __syncwarp();
           tmem_ld_x32(tbase + c * 32, v);
           tmem_ld_wait();
-          if (o < N) {
 #pragma unroll
-            for (int t = 0; t < 32; ++t)
-              if (c * 32 + t < ntok) ybase[(size_t)(c * 32 + t) * N] = __uint_as_float(v[t]);
+          for (int t = 0; t < 32; ++t) tw[t * 36 + lane] = __uint_as_float(v[t]);
+          __syncwarp();
+          if (o0 < N) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int t = vr + 4 * i;
+              const int tok = c * 32 + t;
+              if (tok < ntok) {
+                const float4 val = *reinterpret_cast<const float4*>(tw + t * 36 + vc);
+                *reinterpret_cast<float4*>(static_cast<float*>(out) + (row0 + tok) * N + o0 + vc) = val;
+              }
+            }
           }
         }
       }
