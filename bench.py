@@ -94,7 +94,23 @@ def algorithmic(wl, counts):
                                            bytes=2 * used * I * d * el + R * d * el + R * I * el),
         "grouped_gemm_down": dict(flops=2.0 * R * d * I, bytes=used * d * I * el + R * I * el + R * d * 4),
         "combine": dict(flops=2.0 * R * d, bytes=R * d * 4 + T * d * 4 + R * 8),
+    } if not fused_combine(wl) else {
+        "router_topk": dict(flops=2.0 * T * d * E, bytes=T * d * el + E * d * el + T * k * 12 + nb * E * 8),
+        "route_scan": dict(flops=0.0, bytes=nb * E * 12 + (E + 1) * 8 + E * 4),
+        "permute": dict(flops=0.0, bytes=T * d * el + R * d * el + R * 16 + T * d * 4),
+        "grouped_gemm_gateup_swiglu": dict(flops=4.0 * R * d * I,
+                                           bytes=2 * used * I * d * el + R * d * el + R * I * el),
+        # down projection with the combine folded in: weights, H, and the fp32
+        # output accumulated in place (read + write)
+        "grouped_gemm_down": dict(flops=2.0 * R * d * I + 2.0 * R * d,
+                                  bytes=used * d * I * el + R * I * el + 2 * T * d * 4 + R * 8),
+        "combine": dict(flops=0.0, bytes=0),
     }
+
+
+def fused_combine(wl):
+    """k = 2 on the bf16 path: the combine runs inside the down GEMM's epilogue."""
+    return wl.dtype == "bf16" and wl.k == 2
 
 
 # --------------------------------------------------------------------- clocks
@@ -378,7 +394,8 @@ def main():
     for j, name in enumerate(KERNELS):
         w = work[name]
         t_s = avg[j] / 1e3
-        ent = {"name": name, "avg_us": float(avg[j] * 1e3), "share": float(avg[j] / avg.sum()),
+        ent = {"name": name if not (name == "combine" and fused_combine(wl)) else "combine (in grouped_gemm_down)",
+               "avg_us": float(avg[j] * 1e3), "share": float(avg[j] / avg.sum()),
                "tflops": w["flops"] / t_s / 1e12 if t_s > 0 else None,
                "gbs": w["bytes"] / t_s / 1e9 if t_s > 0 else None}
         kern.append(ent)
@@ -412,7 +429,7 @@ def main():
         "e2e": {"value": wl.T * world * e2e_steps / (ms_e2e / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x.numel() * x.element_size()),
                 "d2h_bytes_per_step": int(wl.T * wl.d * 4 + 4)},
-        "gpu_launches": nk * args.steps,
+        "gpu_launches": (nk - (1 if fused_combine(wl) else 0)) * args.steps,
         "clocks": clocks,
         "counts": counts.tolist() if wl.E <= 16 else {"max": int(counts.max()), "min": int(counts.min()),
                                                       "mean": float(counts.mean())},

@@ -112,6 +112,10 @@ __device__ __forceinline__ void tc_commit_pair_local(uint64_t* bar) {
                : "memory");
 }
 
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
 struct TileCoord {
   int e, m, n;
 };
@@ -142,7 +146,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                             const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBs,
                             const int32_t* __restrict__ offsets, const int32_t* __restrict__ mtile256, int E,
-                            int N, int K, void* __restrict__ out, int32_t* status, uint64_t limit_ns) {
+                            int N, int K, void* __restrict__ out, const int32_t* __restrict__ perm_tok,
+                            const float* __restrict__ rgate, float* __restrict__ comb_out, int32_t* status,
+                            uint64_t limit_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;                           // [stages][128 weight rows x 64]
@@ -375,7 +381,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               const int tok = c * 32 + t;
               if (tok < ntok) {
                 const float4 val = *reinterpret_cast<const float4*>(tw + t * 36 + vc);
-                *reinterpret_cast<float4*>(static_cast<float*>(out) + (row0 + tok) * N + o0 + vc) = val;
+                if (comb_out) {
+                  // combine folded in: out[token] += gate * y (two adds per
+                  // element into a zeroed row, so the order cannot matter)
+                  const size_t r = row0 + tok;
+                  const float g = rgate[r];
+                  red_add_v4(comb_out + (size_t)perm_tok[r] * N + o0 + vc, g * val.x, g * val.y, g * val.z,
+                             g * val.w);
+                } else {
+                  *reinterpret_cast<float4*>(static_cast<float*>(out) + (row0 + tok) * N + o0 + vc) = val;
+                }
               }
             }
           }
@@ -427,7 +442,8 @@ int max_active_pairs(const void* kern, int smem) {
 template <int kMode>
 cudaError_t launch_tc2(const CUtensorMap& tmA0, const CUtensorMap& tmA1, const CUtensorMap& tmB,
                        const CUtensorMap& tmBs, const int32_t* offsets, const int32_t* mtile256, int R, int E, int N,
-                       int K, void* out, int32_t* status, cudaStream_t stream) {
+                       int K, void* out, const int32_t* perm_tok, const float* rgate, float* comb_out,
+                       int32_t* status, cudaStream_t stream) {
   auto kern = grouped_gemm_tc2_kernel<kMode>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemm2SmemBytes);
   if (err != cudaSuccess) return err;
@@ -438,7 +454,7 @@ cudaError_t launch_tc2(const CUtensorMap& tmA0, const CUtensorMap& tmA1, const C
   const int clusters = (int)(max_tiles < pairs ? max_tiles : pairs);
   if (clusters <= 0) return cudaSuccess;
   kern<<<2 * clusters, kGemmThreads, kGemm2SmemBytes, stream>>>(tmA0, tmA1, tmB, tmBs, offsets, mtile256, E, N, K,
-                                                               out, status, kWaitLimitNs);
+                                                               out, perm_tok, rgate, comb_out, status, kWaitLimitNs);
   return cudaGetLastError();
 }
 
@@ -447,13 +463,16 @@ cudaError_t launch_tc2(const CUtensorMap& tmA0, const CUtensorMap& tmA1, const C
 cudaError_t launch_gemm_gateup_tc2(const CUtensorMap& tm_wg, const CUtensorMap& tm_wu, const CUtensorMap& tm_xp,
                                    const CUtensorMap& tm_xp_small, const int32_t* offsets, const int32_t* mtile256,
                                    int R, int E, int I, int d, void* h, int32_t* status, cudaStream_t stream) {
-  return launch_tc2<0>(tm_wg, tm_wu, tm_xp, tm_xp_small, offsets, mtile256, R, E, I, d, h, status, stream);
+  return launch_tc2<0>(tm_wg, tm_wu, tm_xp, tm_xp_small, offsets, mtile256, R, E, I, d, h, nullptr, nullptr, nullptr,
+                       status, stream);
 }
 
 cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_wd, const CUtensorMap& tm_h, const CUtensorMap& tm_h_small,
                                  const int32_t* offsets, const int32_t* mtile256, int R, int E, int I, int d, float* y,
-                                 int32_t* status, cudaStream_t stream) {
-  return launch_tc2<1>(tm_wd, tm_wd, tm_h, tm_h_small, offsets, mtile256, R, E, d, I, y, status, stream);
+                                 const int32_t* perm_tok, const float* rgate, float* comb_out, int32_t* status,
+                                 cudaStream_t stream) {
+  return launch_tc2<1>(tm_wd, tm_wd, tm_h, tm_h_small, offsets, mtile256, R, E, d, I, y, perm_tok, rgate, comb_out,
+                       status, stream);
 }
 
 }  // namespace moe

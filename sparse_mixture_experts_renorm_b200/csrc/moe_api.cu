@@ -99,6 +99,7 @@ Workspace workspace_layout(int T, int d, int E, int k, int I, moe_dtype dtype) {
   w.lrank = o;    o = align256(o + 4 * R);
   w.perm_tok = o; o = align256(o + 4 * R);
   w.inv = o;      o = align256(o + 4 * R);
+  w.rgate = o;    o = align256(o + 4 * R);
   w.xp = o;       o = align256(o + el * R * (size_t)d);
   w.h = o;        o = align256(o + el * R * (size_t)I);
   w.y = o;        o = align256(o + 4 * R * (size_t)d);
@@ -213,7 +214,13 @@ moe_status forward_impl(const void* x, const void* w_router, const float* b_rout
   err = launch_route_scan(router_blocks(T, dtype), T, E, k, blk_cnt, blk_psum, cnt, offsets, mtile, aux_p, stream);
   if (err != cudaSuccess) return fail_cuda(err, "routing scan kernel");
   marks.mark(stream);
-  err = launch_permute(dtype, x, T, d, E, k, router_block_tokens(dtype), topk_idx, lrank, blk_cnt, perm_tok, inv, xp, status, stream);
+  // With k = 2 the bf16 path folds the combine into the down GEMM's epilogue
+  // (two fp32 adds into a zeroed row commute, so the result stays
+  // deterministic); otherwise a separate combine kernel sums the k rows.
+  const bool fused_combine = dtype == MOE_BF16 && k == 2;
+  float* rgate = reinterpret_cast<float*>(ws + w.rgate);
+  err = launch_permute(dtype, x, T, d, E, k, router_block_tokens(dtype), topk_idx, lrank, blk_cnt, perm_tok, inv, xp,
+                       topk_gate, rgate, fused_combine ? out : nullptr, status, stream);
   if (err != cudaSuccess) return fail_cuda(err, "permute kernel");
 
   if (dtype == MOE_BF16) {
@@ -233,7 +240,8 @@ moe_status forward_impl(const void* x, const void* w_router, const float* b_rout
     err = launch_gemm_gateup_tc2(tm_wg, tm_wu, tm_xp, tm_xp_s, offsets, mtile, R, E, I, d, h, status, stream);
     if (err != cudaSuccess) return fail_cuda(err, "gate/up grouped GEMM");
     marks.mark(stream);
-    err = launch_gemm_down_tc2(tm_wd, tm_h, tm_h_s, offsets, mtile, R, E, I, d, y, status, stream);
+    err = launch_gemm_down_tc2(tm_wd, tm_h, tm_h_s, offsets, mtile, R, E, I, d, y, perm_tok, rgate,
+                               fused_combine ? out : nullptr, status, stream);
     if (err != cudaSuccess) return fail_cuda(err, "down grouped GEMM");
   } else {
     marks.mark(stream);
@@ -246,8 +254,10 @@ moe_status forward_impl(const void* x, const void* w_router, const float* b_rout
     if (err != cudaSuccess) return fail_cuda(err, "down grouped GEMM (fp32)");
   }
   marks.mark(stream);
-  err = launch_combine(T, d, k, y, inv, topk_gate, out, status, stream);
-  if (err != cudaSuccess) return fail_cuda(err, "combine kernel");
+  if (!fused_combine) {
+    err = launch_combine(T, d, k, y, inv, topk_gate, out, status, stream);
+    if (err != cudaSuccess) return fail_cuda(err, "combine kernel");
+  }
   err = marks.mark(stream);
   if (err != cudaSuccess) return fail_cuda(err, "recording a timing event");
   return MOE_OK;

@@ -51,6 +51,7 @@ struct Workspace {
   size_t lrank;       // int32 [T*k]   rank of (t,j) among its block's tokens of that expert
   size_t perm_tok;    // int32 [T*k]
   size_t inv;         // int32 [T*k]
+  size_t rgate;       // fp32  [T*k]   gate of every dispatched row
   size_t xp;          // dtype [T*k, d] expert-contiguous copy of x
   size_t h;           // dtype [T*k, I] SwiGLU hidden activations
   size_t y;           // fp32  [T*k, d] expert outputs
@@ -85,9 +86,12 @@ cudaError_t launch_router_tc(const void* x, const void* w_router, const float* b
 cudaError_t launch_route_scan(int nb, int T, int E, int k, int32_t* blk_cnt, const float* blk_psum, int32_t* counts,
                               int32_t* offsets, int32_t* mtile, float* aux, cudaStream_t stream);
 
+// Also records the gate of every dispatched row (rgate) and, when zero_out is
+// given, clears out[T, d] for a combine done by the down GEMM's epilogue.
 cudaError_t launch_permute(moe_dtype dtype, const void* x, int T, int d, int E, int k, int rb, const int32_t* topk_idx,
                            const int32_t* lrank, const int32_t* blk_base, int32_t* perm_tok, int32_t* inv,
-                           void* xp, int32_t* status, cudaStream_t stream);
+                           void* xp, const float* topk_gate, float* rgate, float* zero_out, int32_t* status,
+                           cudaStream_t stream);
 
 cudaError_t launch_combine(int T, int d, int k, const float* y, const int32_t* inv, const float* topk_gate,
                            float* out, int32_t* status, cudaStream_t stream);
@@ -98,9 +102,12 @@ cudaError_t launch_combine(int T, int d, int k, const float* y, const int32_t* i
 cudaError_t launch_gemm_gateup_tc2(const CUtensorMap& tm_wg, const CUtensorMap& tm_wu, const CUtensorMap& tm_xp,
                                    const CUtensorMap& tm_xp_small, const int32_t* offsets, const int32_t* mtile,
                                    int R, int E, int I, int d, void* h, int32_t* status, cudaStream_t stream);
+// comb_out != nullptr: instead of storing Y, add gate * y of every dispatched
+// row into comb_out[token] (used when k = 2, where the two adds commute).
 cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_wd, const CUtensorMap& tm_h, const CUtensorMap& tm_h_small,
                                  const int32_t* offsets, const int32_t* mtile, int R, int E, int I, int d, float* y,
-                                 int32_t* status, cudaStream_t stream);
+                                 const int32_t* perm_tok, const float* rgate, float* comb_out, int32_t* status,
+                                 cudaStream_t stream);
 
 // fp32 SIMT grouped GEMMs.
 cudaError_t launch_gemm_gateup_simt(const float* xp, const float* wg, const float* wu, const int32_t* offsets,

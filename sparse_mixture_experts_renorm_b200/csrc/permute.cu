@@ -20,7 +20,9 @@ __global__ void __launch_bounds__(kCopyThreads) permute_kernel(const uint4* __re
                                                               const int32_t* __restrict__ lrank,
                                                               const int32_t* __restrict__ blk_base,
                                                               int32_t* __restrict__ perm_tok, int32_t* __restrict__ inv,
-                                                              uint4* __restrict__ xp, int32_t* status) {
+                                                              uint4* __restrict__ xp, const float* __restrict__ gate,
+                                                              float* __restrict__ rgate, float4* __restrict__ zero_out,
+                                                              int nout4, int32_t* status) {
   const int t = blockIdx.x;
   __shared__ int s_rows[kMaxTopK];
   if (threadIdx.x < k) {
@@ -34,10 +36,16 @@ __global__ void __launch_bounds__(kCopyThreads) permute_kernel(const uint4* __re
     } else if (blockIdx.y == 0) {
       perm_tok[row] = t;
       inv[(size_t)t * k + j] = row;
+      rgate[row] = gate[(size_t)t * k + j];
     }
     s_rows[j] = row;
   }
   __syncthreads();
+  if (zero_out) {  // the output row this block's x chunk maps to, for a combine done by atomics
+    const int per = (nout4 + gridDim.y - 1) / gridDim.y;
+    for (int o = blockIdx.y * per + threadIdx.x; o < min(nout4, (int)(blockIdx.y + 1) * per); o += kCopyThreads)
+      zero_out[(size_t)t * nout4 + o] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   const int i = blockIdx.y * kCopyThreads + threadIdx.x;
   if (i >= nvec) return;
   const uint4 v = __ldg(x + (size_t)t * nvec + i);
@@ -92,12 +100,14 @@ __global__ void __launch_bounds__(kCopyThreads) combine_kernel(const float4* __r
 
 cudaError_t launch_permute(moe_dtype dtype, const void* x, int T, int d, int E, int k, int rb, const int32_t* topk_idx,
                            const int32_t* lrank, const int32_t* blk_base, int32_t* perm_tok, int32_t* inv, void* xp,
-                           int32_t* status, cudaStream_t stream) {
+                           const float* topk_gate, float* rgate, float* zero_out, int32_t* status,
+                           cudaStream_t stream) {
   const int elem = dtype == MOE_BF16 ? 2 : 4;
   const int nvec = d * elem / 16;
   const dim3 grid(T, (nvec + kCopyThreads - 1) / kCopyThreads);
   permute_kernel<<<grid, kCopyThreads, 0, stream>>>(static_cast<const uint4*>(x), nvec, E, k, rb, T * k, topk_idx, lrank,
-                                                    blk_base, perm_tok, inv, static_cast<uint4*>(xp), status);
+                                                    blk_base, perm_tok, inv, static_cast<uint4*>(xp), topk_gate, rgate,
+                                                    reinterpret_cast<float4*>(zero_out), d / 4, status);
   return cudaGetLastError();
 }
 
