@@ -316,11 +316,6 @@ def main():
         raise RuntimeError(f"device status word {status:#x} after warm-up")
 
     nk = B.MOE_NUM_KERNELS
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
-    for row in evs:  # create the events outside the timed region
-        for ev in row:
-            ev.record(stream)
-    torch.cuda.synchronize()
     sampler = ClockSampler(dev)
     time.sleep(0.3)
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -328,19 +323,31 @@ def main():
     torch.cuda.synchronize()
     t_wall0 = time.time()
     start.record(stream)
-    for i in range(args.steps):
-        layer(x, events=evs[i])
+    for _ in range(args.steps):
+        layer(x)
     stop.record(stream)
     torch.cuda.synchronize()
     barrier()
     t_wall1 = time.time()
     clocks = sampler.stop(t_wall0, t_wall1)
     ms = start.elapsed_time(stop)
-    per_kernel = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(nk)] for i in range(args.steps)])
     if world > 1:
         t = torch.tensor([ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
+
+    # ---- per-kernel device times: the same steps again, with an event recorded
+    # before each kernel and after the last (events between the kernels also
+    # stop the next kernel's set-up from overlapping the previous one's tail)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
+    for row in evs:  # create the events outside the timed loop
+        for ev in row:
+            ev.record(stream)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        layer(x, events=evs[i])
+    torch.cuda.synchronize()
+    per_kernel = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(nk)] for i in range(args.steps)])
     status = int(layer.status.item())
     if status:
         raise RuntimeError(f"device status word {status:#x} after the timed region")

@@ -24,6 +24,14 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
+// Programmatic dependent launch: every kernel of the library is launched so
+// that it may start while the previous kernel in the stream is finishing. It
+// sets up what needs no input (barriers, TMEM, descriptor prefetch), then
+// passes pdl_wait() before it reads or writes any global memory the previous
+// kernel may touch; pdl_trigger() lets the next kernel begin its own set-up.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier --
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

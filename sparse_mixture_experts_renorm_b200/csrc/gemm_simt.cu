@@ -20,6 +20,7 @@ __global__ void __launch_bounds__(256) grouped_gemm_simt_kernel(const float* __r
                                                                 const int32_t* __restrict__ offsets, int E, int N,
                                                                 int K, float* __restrict__ out) {
   __shared__ int s_info[3];  // expert, first row, rows in this tile
+  pdl_wait();
   if (threadIdx.x == 0) {
     int mt = blockIdx.y, cum = 0, e = -1, row0 = 0, rows = 0;
     for (int ee = 0; ee < E; ++ee) {
@@ -101,8 +102,7 @@ cudaError_t launch_simt(const float* A, const float* B0, const float* B1, const 
                         int K, float* out, cudaStream_t stream) {
   const int max_mtiles = R / kSimtBM + E;
   dim3 grid((N + kSimtBN - 1) / kSimtBN, max_mtiles);
-  grouped_gemm_simt_kernel<kMode><<<grid, 256, 0, stream>>>(A, B0, B1, offsets, E, N, K, out);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_simt_kernel<kMode>, grid, dim3(256), 0, stream, A, B0, B1, offsets, E, N, K, out);
 }
 
 }  // namespace

@@ -176,10 +176,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const int n_wb = kMode == 0 ? (N + 127) / 128 : (N + 255) / 256;
   const int KB = K / kBK;
 
-  for (int i = threadIdx.x; i <= E; i += blockDim.x) {
-    s_off[i] = offsets[i];
-    s_mt[i] = mtile256[i];
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages2; ++s) {
       mbar_init(&full[s], 1);
@@ -202,6 +198,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     tmem_alloc_pair(s_tmem, 2 * kBN);
     tmem_relinquish_pair();
+  }
+  pdl_wait();  // the routing tables and the A/B operands come from the kernels before
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) {
+    s_off[i] = offsets[i];
+    s_mt[i] = mtile256[i];
   }
   tc_fence_before();
   __syncthreads();
@@ -406,6 +407,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
   }
 
+  pdl_trigger();
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // no CTA leaves while its peer may still touch its shared memory or TMEM
@@ -453,9 +455,8 @@ cudaError_t launch_tc2(const CUtensorMap& tmA0, const CUtensorMap& tmA1, const C
   const long long max_tiles = (long long)(R / 256 + E) * n_wb;
   const int clusters = (int)(max_tiles < pairs ? max_tiles : pairs);
   if (clusters <= 0) return cudaSuccess;
-  kern<<<2 * clusters, kGemmThreads, kGemm2SmemBytes, stream>>>(tmA0, tmA1, tmB, tmBs, offsets, mtile256, E, N, K,
-                                                               out, perm_tok, rgate, comb_out, status, kWaitLimitNs);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(2 * clusters), dim3(kGemmThreads), kGemm2SmemBytes, stream, tmA0, tmA1, tmB, tmBs,
+                    offsets, mtile256, E, N, K, out, perm_tok, rgate, comb_out, status, kWaitLimitNs);
 }
 
 }  // namespace

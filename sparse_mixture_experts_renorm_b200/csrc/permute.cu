@@ -25,6 +25,7 @@ __global__ void __launch_bounds__(kCopyThreads) permute_kernel(const uint4* __re
                                                               int nout4, int32_t* status) {
   const int t = blockIdx.x;
   __shared__ int s_rows[kMaxTopK];
+  pdl_wait();
   if (threadIdx.x < k) {
     const int j = threadIdx.x;
     const int e = topk_idx[(size_t)t * k + j];
@@ -63,6 +64,7 @@ __global__ void __launch_bounds__(kCopyThreads) combine_kernel(const float4* __r
   const int t = blockIdx.x;
   __shared__ int s_rows[kMaxTopK];
   __shared__ float s_g[kMaxTopK];
+  pdl_wait();
   if (threadIdx.x < k) {
     const int j = threadIdx.x;
     int row = inv[(size_t)t * k + j];
@@ -105,19 +107,17 @@ cudaError_t launch_permute(moe_dtype dtype, const void* x, int T, int d, int E, 
   const int elem = dtype == MOE_BF16 ? 2 : 4;
   const int nvec = d * elem / 16;
   const dim3 grid(T, (nvec + kCopyThreads - 1) / kCopyThreads);
-  permute_kernel<<<grid, kCopyThreads, 0, stream>>>(static_cast<const uint4*>(x), nvec, E, k, rb, T * k, topk_idx, lrank,
-                                                    blk_base, perm_tok, inv, static_cast<uint4*>(xp), topk_gate, rgate,
-                                                    reinterpret_cast<float4*>(zero_out), d / 4, status);
-  return cudaGetLastError();
+  return launch_pdl(permute_kernel, grid, dim3(kCopyThreads), 0, stream, static_cast<const uint4*>(x), nvec, E, k, rb,
+                    T * k, topk_idx, lrank, blk_base, perm_tok, inv, static_cast<uint4*>(xp), topk_gate, rgate,
+                    reinterpret_cast<float4*>(zero_out), d / 4, status);
 }
 
 cudaError_t launch_combine(int T, int d, int k, const float* y, const int32_t* inv, const float* topk_gate, float* out,
                            int32_t* status, cudaStream_t stream) {
   const int nvec4 = d / 4;
   const dim3 grid(T, (nvec4 + kCopyThreads - 1) / kCopyThreads);
-  combine_kernel<<<grid, kCopyThreads, 0, stream>>>(reinterpret_cast<const float4*>(y), nvec4, k, T * k, inv,
-                                                    topk_gate, reinterpret_cast<float4*>(out), status);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, grid, dim3(kCopyThreads), 0, stream, reinterpret_cast<const float4*>(y), nvec4, k,
+                    T * k, inv, topk_gate, reinterpret_cast<float4*>(out), status);
 }
 
 }  // namespace moe

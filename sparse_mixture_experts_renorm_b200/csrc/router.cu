@@ -49,6 +49,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(
   const int ntok = min(kRouterTokensSimt, T - tok0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  pdl_wait();
   router_logits_f32(x, wr, T, d, E, tok0, s_p, ld);
 
   // ---- softmax, top-k and gates: one warp per token --------------------
@@ -194,6 +195,7 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int nb, int T, int E, 
   const bool active = sl < S;
   const int chunk = (nb + S - 1) / S;
   const int b0 = min(nb, sl * chunk), b1 = min(nb, b0 + chunk);
+  pdl_wait();
   if (active) {
     int c = 0;
     double ps = 0.0;
@@ -259,16 +261,15 @@ cudaError_t launch_router(moe_dtype dtype, const void* x, const void* w_router, 
   const size_t smem = (size_t)kRouterTokensSimt * (E + 1) * sizeof(float);
   cudaError_t err = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  router_kernel<<<nb, kRouterThreads, smem, stream>>>(static_cast<const float*>(x), static_cast<const float*>(w_router),
-                                                      b_router, T, d, E, k, renorm, topk_idx, topk_gate, lrank, blk_cnt,
-                                                      blk_psum, status);
-  return cudaGetLastError();
+  return launch_pdl(router_kernel, dim3(nb), dim3(kRouterThreads), smem, stream, static_cast<const float*>(x),
+                    static_cast<const float*>(w_router), b_router, T, d, E, k, renorm, topk_idx, topk_gate, lrank,
+                    blk_cnt, blk_psum, status);
 }
 
 cudaError_t launch_route_scan(int nb, int T, int E, int k, int32_t* blk_cnt, const float* blk_psum, int32_t* counts,
                               int32_t* offsets, int32_t* mtile, float* aux, cudaStream_t stream) {
-  route_scan_kernel<<<1, 1024, 0, stream>>>(nb, T, E, k, blk_cnt, blk_psum, counts, offsets, mtile, aux);
-  return cudaGetLastError();
+  return launch_pdl(route_scan_kernel, dim3(1), dim3(1024), 0, stream, nb, T, E, k, blk_cnt, blk_psum, counts, offsets,
+                    mtile, aux);
 }
 
 }  // namespace moe

@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
+  pdl_wait();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -289,6 +290,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   }
 
+  pdl_trigger();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -311,11 +313,9 @@ cudaError_t launch_router_tc(const void* x, const void* w_router, const float* b
   cudaError_t err = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, c.smem_bytes);
   if (err != cudaSuccess) return err;
   const int nb = (T + kRB - 1) / kRB;
-  router_tc_kernel<<<nb, kGemmThreads, c.smem_bytes, stream>>>(tmX, tmW, b_router, T, d, E, k, renorm, c.npad,
-                                                               c.stages, c.stage_bytes, c.tmem_cols, topk_idx,
-                                                               topk_gate, lrank, blk_cnt, blk_psum, status,
-                                                               kWaitLimitNs);
-  return cudaGetLastError();
+  return launch_pdl(router_tc_kernel, dim3(nb), dim3(kGemmThreads), c.smem_bytes, stream, tmX, tmW, b_router, T, d, E,
+                    k, renorm, c.npad, c.stages, c.stage_bytes, c.tmem_cols, topk_idx, topk_gate, lrank, blk_cnt,
+                    blk_psum, status, kWaitLimitNs);
 }
 
 }  // namespace moe
