@@ -116,6 +116,22 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 
+// 32 accumulator columns of this warp's lanes, summed over the tile's
+// accumulators in order (a tile with one accumulator is a plain load).
+__device__ __forceinline__ void ld_chunk_sum(uint32_t taddr, int nacc, int stride, uint32_t (&v)[32]) {
+  __syncwarp();
+  tmem_ld_x32(taddr, v);
+  tmem_ld_wait();
+  for (int a = 1; a < nacc; ++a) {
+    uint32_t w[32];
+    __syncwarp();
+    tmem_ld_x32(taddr + a * stride, w);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(w[i]));
+  }
+}
+
 struct TileCoord {
   int e, m, n;
 };
@@ -274,7 +290,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       for (int tile = cid; ok && tile < total; tile += ncl) {
         const TileCoord tc = decode_tile(tile, n_wb, s_mt, E);
         const int ntok = min(256, s_off[tc.e + 1] - s_off[tc.e] - tc.m * 256);
-        const uint32_t idesc = idesc_bf16_f32(256, (ntok + 15) & ~15);
+        const int nt16 = (ntok + 15) & ~15;
+        const uint32_t idesc = idesc_bf16_f32(256, nt16);
+        // narrow tiles spread their K loop over independent accumulators
+        const int nacc = nt16 <= 64 ? 4 : (nt16 <= 128 ? 2 : 1);
+        const int acc_stride = kBN / nacc;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, s_abort, status, limit_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kBN);
@@ -287,9 +307,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const uint64_t adesc = sw128_kmajor_desc(smem_u32(sA + stage * kHalfBytes));
           const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sB + stage * kHalfBytes));
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            tc_mma_bf16_pair(d_tmem, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2),
-                             idesc, (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const int a = kk % nacc;
+            tc_mma_bf16_pair(d_tmem + static_cast<uint32_t>(a * acc_stride), adesc + static_cast<uint64_t>(kk * 2),
+                             bdesc + static_cast<uint64_t>(kk * 2), idesc, (kb > 0 || kk >= nacc) ? 1u : 0u);
+          }
           tc_commit_pair_both(&empty[stage]);
           if (++stage == kStages2) {
             stage = 0;
@@ -323,6 +345,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kBN);
       const int nchunks = (ntok + 31) >> 5;
+      const int nt16 = (ntok + 15) & ~15;
+      const int nacc = nt16 <= 64 ? 4 : (nt16 <= 128 ? 2 : 1);
+      const int acc_stride = kBN / nacc;
       if (kMode == 0) {
         // TMEM lanes 0-63 hold the gate rows, 64-127 the up rows of this
         // CTA's 64 hidden units. Per 32-token chunk both halves go to shared
@@ -337,9 +362,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
           uint32_t v[32];
-          __syncwarp();
-          tmem_ld_x32(tbase + c * 32, v);
-          tmem_ld_wait();
+          ld_chunk_sum(tbase + c * 32, nacc, acc_stride, v);
 #pragma unroll
           for (int t = 0; t < 32; ++t) sdst[t] = __uint_as_float(v[t]);
           epi_bar();
@@ -369,9 +392,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < nchunks; ++c) {
           uint32_t v[32];
-          __syncwarp();
-          tmem_ld_x32(tbase + c * 32, v);
-          tmem_ld_wait();
+          ld_chunk_sum(tbase + c * 32, nacc, acc_stride, v);
 #pragma unroll
           for (int t = 0; t < 32; ++t) tw[t * 36 + lane] = __uint_as_float(v[t]);
           __syncwarp();

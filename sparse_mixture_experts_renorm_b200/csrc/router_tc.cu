@@ -9,12 +9,16 @@
 // load_balancing_loss (E * sum_i f_i * P_i); Model Architecture Patterns,
 // "Top-K Router" (raw top-k softmax gates when not renormalised).
 //
-// Each CTA owns 128 tokens (the UMMA M); N is E rounded up to a multiple of 16
-// (TMA zero-fills the missing router rows). Warp 0 streams x and W_r through a
-// shared-memory ring by TMA, warp 1 issues 128 x N x 16 UMMAs into TMEM, and
-// warps 2-5 read each token's logits row from its own TMEM lane, so softmax and
-// top-k need no cross-thread reduction. After the MMAs the ring is reused for
-// the [128][E+1] probability tile that the per-block statistics read.
+// A block of 128 tokens (the UMMA M) is owned by a cluster of S CTAs that
+// split the d-long K loop (S = 1 when the grid already fills the GPU): each
+// CTA's warp 0 streams its share of x and W_r through a shared-memory ring by
+// TMA, warp 1 issues 128 x N x 16 UMMAs (N = E rounded up to 16; TMA zero-fills
+// the missing router rows), and warps 2-5 read each token's logits from their
+// own TMEM lane. The other CTAs of the cluster add their partial logits into
+// the leading CTA's shared memory, which finishes the block: one thread per
+// token does the softmax, top-k and gates without cross-thread reductions
+// (logits in registers for E <= 64), then the block's histogram, ranks and
+// probability sums.
 #include <math.h>
 
 #include "common.cuh"
@@ -22,25 +26,38 @@
 namespace moe {
 namespace {
 
-constexpr int kRB = kRouterTokensTc;  // 128 tokens per CTA
+constexpr int kRB = kRouterTokensTc;  // 128 tokens per block
+constexpr int kRegE = 64;             // up to this many experts a token's logits stay in registers
 
 struct RouterCfg {
-  int npad;        // UMMA N
-  int stages;      // ring depth
-  int stage_bytes; // x tile + W_r tile
-  int tmem_cols;   // power of two >= max(32, npad)
-  int smem_bytes;  // dynamic shared memory
+  int npad;         // UMMA N
+  int S;            // CTAs per token block (split of the K loop)
+  int stages;       // ring depth
+  int stage_bytes;  // x tile + W_r tile
+  int part_bytes;   // partial-logit buffer of the leading CTA
+  int tmem_cols;    // power of two >= max(32, columns read)
+  int smem_bytes;   // dynamic shared memory
 };
 
-RouterCfg router_cfg(int E) {
+RouterCfg router_cfg(int T, int d, int E, int num_sms) {
   RouterCfg c;
   c.npad = ((E + 15) / 16) * 16;
   c.stage_bytes = kRB * kBK * 2 + c.npad * kBK * 2;
-  c.stages = (192 * 1024) / c.stage_bytes;
+  const int nb = (T + kRB - 1) / kRB;
+  const int KB = d / kBK;
+  // split K only while the grid leaves SMs idle, the partial logits stay
+  // small, and each CTA keeps at least two k-blocks
+  c.S = 1;
+  if (E <= kRegE)
+    while (c.S < 8 && nb * c.S * 2 <= num_sms && (c.S * 2 - 1) * kRB * E * 4 <= 64 * 1024 && KB / (c.S * 2) >= 2)
+      c.S *= 2;
+  c.part_bytes = (c.S - 1) * kRB * E * 4;
+  c.stages = (192 * 1024 - c.part_bytes) / c.stage_bytes;
   if (c.stages > 8) c.stages = 8;
+  const int cols = 32 * ((E + 31) / 32);
   c.tmem_cols = 32;
-  while (c.tmem_cols < c.npad) c.tmem_cols <<= 1;
-  c.smem_bytes = c.stages * c.stage_bytes + 1024 + 12288;
+  while (c.tmem_cols < cols) c.tmem_cols <<= 1;
+  c.smem_bytes = c.stages * c.stage_bytes + c.part_bytes + 1024 + 12288;
   return c;
 }
 
@@ -49,16 +66,51 @@ __device__ __forceinline__ bool ahead(float v, int e, float bv, int be) { return
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+__device__ __forceinline__ uint32_t cta_rank_in_cluster() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Store to the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ void st_cluster_f32(const void* local_in_leader_layout, uint32_t rank, float v) {
+  uint32_t addr;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(addr) : "r"(smem_u32(local_in_leader_layout)), "r"(rank));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+// Insert (v, e) into the list of the kMaxTopK best, kept sorted best first.
+__device__ __forceinline__ void topk_insert(float (&bv)[kMaxTopK], int (&be)[kMaxTopK], float v, int e) {
+  if (!ahead(v, e, bv[kMaxTopK - 1], be[kMaxTopK - 1])) return;
+  bv[kMaxTopK - 1] = v;
+  be[kMaxTopK - 1] = e;
+#pragma unroll
+  for (int j = kMaxTopK - 1; j > 0; --j) {
+    if (ahead(bv[j], be[j], bv[j - 1], be[j - 1])) {
+      const float tv = bv[j];
+      bv[j] = bv[j - 1];
+      bv[j - 1] = tv;
+      const int te = be[j];
+      be[j] = be[j - 1];
+      be[j - 1] = te;
+    }
+  }
+}
+
+template <int kE>  // E <= kE: logits in registers; kE == 0: E > kRegE, logits in shared memory
 __global__ void __launch_bounds__(kGemmThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                     const float* __restrict__ br, int T, int d, int E, int k, int renorm, int npad, int stages,
-                     int stage_bytes, int tmem_cols, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate,
-                     int32_t* __restrict__ lrank, int32_t* __restrict__ blk_cnt, float* __restrict__ blk_psum,
-                     int32_t* status, uint64_t limit_ns) {
+                     const float* __restrict__ br, int T, int d, int E, int k, int renorm, int npad, int S,
+                     int stages, int stage_bytes, int tmem_cols, int32_t* __restrict__ topk_idx,
+                     float* __restrict__ topk_gate, int32_t* __restrict__ lrank, int32_t* __restrict__ blk_cnt,
+                     float* __restrict__ blk_psum, int32_t* status, uint64_t limit_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes);
+  float* part = reinterpret_cast<float*>(smem + stages * stage_bytes);  // [S-1][128][E] (leading CTA)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes + (S - 1) * kRB * E * 4);
   uint64_t* full = bars;           // [stages]
   uint64_t* empty = bars + 8;      // [stages]
   uint64_t* tfull = bars + 16;
@@ -69,8 +121,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   int* s_wcnt = s_idx + kRB * kMaxTopK;              // [4][E] per-warp counts, then exclusive prefix
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tok0 = blockIdx.x * kRB;
+  const uint32_t rank = S > 1 ? cta_rank_in_cluster() : 0u;
+  const int blk = blockIdx.x / S;
+  const int tok0 = blk * kRB;
   const int KB = d / kBK;
+  const int kb0 = (int)rank * KB / S, kb1 = ((int)rank + 1) * KB / S;
   const int a_bytes = kRB * kBK * 2;
 
   if (threadIdx.x == 0) {
@@ -97,12 +152,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem_base = *s_tmem;
   pdl_wait();
 
+  constexpr int kL = kE > 0 ? kE : 1;
+  float lg[kL];  // this token's logits (register path)
   if (warp == 0) {
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, s_abort, status, limit_ns)) break;
         mbar_arrive_expect_tx(&full[stage], stage_bytes);
         uint8_t* st = ring + stage * stage_bytes;
@@ -130,10 +187,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t idesc = idesc_bf16_f32(kRB, npad);
       int stage = 0;
       uint32_t phase = 0;
-      bool ok = true;
-      for (int kb = 0; kb < KB; ++kb) {
+      bool mok = true;
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&full[stage], phase, s_abort, status, limit_ns)) {
-          ok = false;
+          mok = false;
           break;
         }
         tc_fence_after();
@@ -143,34 +200,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk)
           tc_mma_bf16(tmem_base, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2), idesc,
-                      (kb | kk) != 0 ? 1u : 0u);
+                      (kb > kb0 || kk > 0) ? 1u : 0u);
         tc_commit(&empty[stage]);
         if (++stage == stages) {
           stage = 0;
           phase ^= 1u;
         }
       }
-      if (ok) tc_commit(tfull);
+      if (mok) tc_commit(tfull);
       tc_commit(done);
       mbar_wait(done, 0, nullptr, status, limit_ns);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------ one thread per token --
+    // -------------------------- read this CTA's partial logits from TMEM --
     const int q = warp & 3;
     const int r = q * 32 + lane;
-    const int t = tok0 + r;
-    const bool valid = t < T;
-    const int ld = E + 1;
-    float* s_p = reinterpret_cast<float*>(ring);  // [128][E+1], reuses the ring after the MMAs
     const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull, 0, s_abort, status, limit_ns));
     tc_fence_after();
     const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const int nchunks = (E + 31) >> 5;
-
-    // pass 1: logits (+ bias) into the probability tile, row maximum
-    float m = -INFINITY;
-    bool finite = true;
+    float* s_p = reinterpret_cast<float*>(ring);  // [128][E+1] when E > kRegE (ring free after the MMAs)
     for (int c = 0; c < nchunks; ++c) {
       uint32_t v[32];
       __syncwarp();
@@ -181,26 +231,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = 0u;
       }
+      if (kE > 0) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int e = c * 32 + i;
-        if (e < E) {
-          float l = __uint_as_float(v[i]);
-          if (br) l += br[e];
-          finite = finite && isfinite(l);
-          m = fmaxf(m, l);
-          s_p[r * ld + e] = l;
-        }
+        for (int i = 0; i < 32; ++i)
+#pragma unroll
+          for (int cc = 0; cc * 32 < kL; ++cc)
+            if (c == cc && cc * 32 + i < kL) lg[cc * 32 + i] = __uint_as_float(v[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (c * 32 + i < E) s_p[r * (E + 1) + c * 32 + i] = __uint_as_float(v[i]);
       }
     }
-    // pass 2: exponentials and their sum (expert order)
-    float s = 0.f;
-    for (int e = 0; e < E; ++e) {
-      const float ex = expf(s_p[r * ld + e] - m);
-      s_p[r * ld + e] = ex;
-      s += ex;
+    if (S > 1 && rank > 0) {  // this CTA's share of the K loop goes to the leader
+      float* dst = part + ((size_t)(rank - 1) * kRB + r) * E;
+#pragma unroll
+      for (int e = 0; e < kL; ++e)
+        if (e < E) st_cluster_f32(dst + e, 0, lg[e]);
     }
-    // pass 3: probabilities and the k best under (p descending, index ascending)
+  }
+
+  if (S > 1) cluster_sync_all();  // every partial has landed in the leading CTA
+
+  if (rank == 0 && warp >= 2) {
+    // ------------------------------------------------ one thread per token --
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const int t = tok0 + r;
+    const bool valid = t < T;
+    const int ld = E + 1;
+    float* s_p = reinterpret_cast<float*>(ring);  // [128][E+1] probabilities
     float bv[kMaxTopK];
     int be[kMaxTopK];
 #pragma unroll
@@ -208,24 +268,58 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bv[j] = -INFINITY;
       be[j] = 0x7fffffff;
     }
-    for (int e = 0; e < E; ++e) {
-      const float p = s_p[r * ld + e] / s;
-      s_p[r * ld + e] = valid ? p : 0.f;
-      const float pv = (p != p) ? -INFINITY : p;
-      if (ahead(pv, e, bv[kMaxTopK - 1], be[kMaxTopK - 1])) {
-        bv[kMaxTopK - 1] = pv;
-        be[kMaxTopK - 1] = e;
+    bool finite = true;
+    if (kE > 0) {
+      // the other CTAs' partial logits in rank order, the bias, the maximum
+      for (int s2 = 0; s2 < S - 1; ++s2) {
+        const float* src = part + ((size_t)s2 * kRB + r) * E;
 #pragma unroll
-        for (int j = kMaxTopK - 1; j > 0; --j) {
-          if (ahead(bv[j], be[j], bv[j - 1], be[j - 1])) {
-            const float tv = bv[j];
-            bv[j] = bv[j - 1];
-            bv[j - 1] = tv;
-            const int te = be[j];
-            be[j] = be[j - 1];
-            be[j - 1] = te;
-          }
+        for (int e = 0; e < kL; ++e)
+          if (e < E) lg[e] += src[e];
+      }
+      float m = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < kL; ++e)
+        if (e < E) {
+          if (br) lg[e] += br[e];
+          finite = finite && isfinite(lg[e]);
+          m = fmaxf(m, lg[e]);
         }
+      float s = 0.f;
+#pragma unroll
+      for (int e = 0; e < kL; ++e)
+        if (e < E) {
+          lg[e] = __expf(lg[e] - m);
+          s += lg[e];
+        }
+      const float inv_s = 1.0f / s;
+#pragma unroll
+      for (int e = 0; e < kL; ++e)
+        if (e < E) {
+          const float p = lg[e] * inv_s;
+          s_p[r * ld + e] = valid ? p : 0.f;
+          topk_insert(bv, be, (p != p) ? -INFINITY : p, e);
+        }
+    } else {
+      float m = -INFINITY;
+      for (int e = 0; e < E; ++e) {
+        float l = s_p[r * ld + e];
+        if (br) l += br[e];
+        finite = finite && isfinite(l);
+        m = fmaxf(m, l);
+        s_p[r * ld + e] = l;
+      }
+      float s = 0.f;
+      for (int e = 0; e < E; ++e) {
+        const float ex = __expf(s_p[r * ld + e] - m);
+        s_p[r * ld + e] = ex;
+        s += ex;
+      }
+      const float inv_s = 1.0f / s;
+      for (int e = 0; e < E; ++e) {
+        const float p = s_p[r * ld + e] * inv_s;
+        s_p[r * ld + e] = valid ? p : 0.f;
+        topk_insert(bv, be, (p != p) ? -INFINITY : p, e);
       }
     }
     if (valid && !finite) atomicOr(status, MOE_DEV_NONFINITE);
@@ -254,13 +348,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     // per-warp histogram and in-warp rank of each assignment
     uint32_t myrank[kMaxTopK];
+    int mine[kMaxTopK];
 #pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) myrank[j] = 0;
+    for (int j = 0; j < kMaxTopK; ++j) {
+      myrank[j] = 0;
+      mine[j] = j < k ? s_idx[r * kMaxTopK + j] : -1;
+    }
+#pragma unroll 4
     for (int e = 0; e < E; ++e) {
       int jhit = -1;
 #pragma unroll
       for (int j = 0; j < kMaxTopK; ++j)
-        if (j < k && s_idx[r * kMaxTopK + j] == e) jhit = j;
+        if (mine[j] == e) jhit = j;
       const uint32_t mask = __ballot_sync(0xffffffffu, jhit >= 0);
       const uint32_t rk = __popc(mask & ((1u << lane) - 1u));
 #pragma unroll
@@ -277,10 +376,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         s_wcnt[qq * E + e] = run;
         run += c;
       }
-      blk_cnt[(size_t)blockIdx.x * E + e] = run;
+      blk_cnt[(size_t)blk * E + e] = run;
       float ps = 0.f;
       for (int rr = 0; rr < kRB; ++rr) ps += s_p[rr * ld + e];
-      blk_psum[(size_t)blockIdx.x * E + e] = ps;
+      blk_psum[(size_t)blk * E + e] = ps;
     }
     epi_bar();
     if (valid) {
@@ -300,22 +399,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 }  // namespace
 
 cudaError_t launch_router_tc(const void* x, const void* w_router, const float* b_router, int T, int d, int E, int k,
                              int renorm, int32_t* topk_idx, float* topk_gate, int32_t* lrank, int32_t* blk_cnt,
                              float* blk_psum, int32_t* status, cudaStream_t stream) {
-  const RouterCfg c = router_cfg(E);
+  const RouterCfg c = router_cfg(T, d, E, sm_count());
   CUtensorMap tmX, tmW;
   if (!make_tmap_bf16_2d(&tmX, x, (uint64_t)T, (uint64_t)d, kRB) ||
       !make_tmap_bf16_2d(&tmW, w_router, (uint64_t)E, (uint64_t)d, (uint32_t)c.npad))
     return cudaErrorInvalidValue;
-  cudaError_t err = cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, c.smem_bytes);
+  auto kern = E <= 16 ? router_tc_kernel<16> : E <= 32 ? router_tc_kernel<32> : E <= kRegE ? router_tc_kernel<kRegE>
+                                                                                           : router_tc_kernel<0>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, c.smem_bytes);
   if (err != cudaSuccess) return err;
   const int nb = (T + kRB - 1) / kRB;
-  return launch_pdl(router_tc_kernel, dim3(nb), dim3(kGemmThreads), c.smem_bytes, stream, tmX, tmW, b_router, T, d, E,
-                    k, renorm, c.npad, c.stages, c.stage_bytes, c.tmem_cols, topk_idx, topk_gate, lrank, blk_cnt,
-                    blk_psum, status, kWaitLimitNs);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nb * c.S);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = c.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  attrs[1].id = cudaLaunchAttributeClusterDimension;
+  attrs[1].val.clusterDim.x = c.S;
+  attrs[1].val.clusterDim.y = 1;
+  attrs[1].val.clusterDim.z = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = c.S > 1 ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, tmX, tmW, b_router, T, d, E, k, renorm, c.npad, c.S, c.stages,
+                            c.stage_bytes, c.tmem_cols, topk_idx, topk_gate, lrank, blk_cnt, blk_psum, status,
+                            kWaitLimitNs);
 }
 
 }  // namespace moe
