@@ -288,25 +288,19 @@ def main():
 
     from sparse_mixture_experts_renorm_b200 import MoELayer
     from sparse_mixture_experts_renorm_b200 import _binding as B
+    from sparse_mixture_experts_renorm_b200 import parallel as par
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = par.env_ranks()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
-        from datetime import timedelta
-
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        par.init("nccl", 120.0, device=dev)
 
     inp = make_inputs(wl, dev, seed=0)  # same weights on every rank
-    x = make_tokens(wl, wl.T, dev, seed=1000 + rank) if world > 1 else inp.x
+    x = make_tokens(wl, wl.T, dev, seed=par.batch_seed(rank)) if world > 1 else inp.x
     layer = MoELayer(inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k, wl.renorm, wl.T)
     stream = torch.cuda.current_stream(dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
+    barrier = par.barrier
 
     for _ in range(args.warmup):
         layer(x)
@@ -330,11 +324,7 @@ def main():
     barrier()
     t_wall1 = time.time()
     clocks = sampler.stop(t_wall0, t_wall1)
-    ms = start.elapsed_time(stop)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = par.max_over_ranks(start.elapsed_time(stop), dev)
 
     # ---- per-kernel device times: the same steps again, with an event recorded
     # before each kernel and after the last (events between the kernels also
@@ -375,11 +365,7 @@ def main():
     pipe.synchronize()
     torch.cuda.synchronize()
     barrier()
-    ms_e2e = s2.elapsed_time(e2)
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = par.max_over_ranks(s2.elapsed_time(e2), dev)
 
     counts = layer.counts.cpu().numpy()
     if world > 1:
@@ -387,7 +373,7 @@ def main():
     if rank != 0:
         return 0
 
-    tokens = wl.T * world * args.steps
+    tokens = par.job_tokens(wl.T, world, args.steps)
     tok_s = tokens / (ms / 1e3)
     tflops = wl.active_flops * world * args.steps / (ms / 1e3) / 1e12
     peaks, peak_src = load_peaks()
@@ -433,7 +419,7 @@ def main():
         "config": config_of(wl, world),
         "roofline": roof,
         "kernels": kern,
-        "e2e": {"value": wl.T * world * e2e_steps / (ms_e2e / 1e3), "unit": "tokens/s",
+        "e2e": {"value": par.job_tokens(wl.T, world, e2e_steps) / (ms_e2e / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x.numel() * x.element_size()),
                 "d2h_bytes_per_step": int(wl.T * wl.d * 4 + 4)},
         "gpu_launches": (nk - (1 if fused_combine(wl) else 0)) * args.steps,
