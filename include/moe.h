@@ -184,6 +184,17 @@ moe_status moe_forward_noalloc(const void* x, const void* w_router, const float*
                                float* aux, int32_t* status_dev, void* stream);
 
 /*
+ * moe_selftest_wait_timeout — a diagnostic of the failure handling every
+ * kernel of the library shares: it launches one warp on `stream` that waits
+ * on a shared-memory barrier phase nothing will complete, through the same
+ * bounded wait the kernels use, with a limit of limit_ns nanoseconds
+ * (1e6 .. 1e9*5). The wait gives up, OR-s MOE_DEV_TIMEOUT into *status_dev
+ * (device int32, not cleared here) and the kernel returns; the context stays
+ * usable. The pages have no counterpart (their Rust layer panics instead).
+ */
+moe_status moe_selftest_wait_timeout(int32_t* status_dev, long long limit_ns, void* stream);
+
+/*
  * moe_last_error_detail — the reason for the calling thread's last non-OK
  * status, NUL-terminated into buf (truncated to n bytes). Returns the full
  * length of the message.

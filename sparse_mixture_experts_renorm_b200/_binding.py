@@ -26,7 +26,7 @@ STATUS_NAMES = {
 }
 
 EXPORTED = ("moe_workspace_size", "moe_forward", "moe_forward_events", "moe_kernel_name", "moe_get_permutation",
-            "moe_last_error_detail", "moe_forward_noalloc")
+            "moe_last_error_detail", "moe_forward_noalloc", "moe_selftest_wait_timeout")
 MOE_NOALLOC_SCRATCH_BYTES = 16 << 20
 MOE_NUM_KERNELS = 6
 
@@ -64,6 +64,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.moe_kernel_name.restype = ctypes.c_char_p
     lib.moe_forward_noalloc.argtypes = [P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, P, P, P, P, P, P, P]
     lib.moe_forward_noalloc.restype = I32
+    lib.moe_selftest_wait_timeout.argtypes = [P, ctypes.c_longlong, P]
+    lib.moe_selftest_wait_timeout.restype = I32
     lib.moe_get_permutation.argtypes = [P, SZ, I32, I32, I32, I32, I32, I32, P, P, P, P]
     lib.moe_get_permutation.restype = I32
     lib.moe_last_error_detail.argtypes = [ctypes.c_char_p, SZ]

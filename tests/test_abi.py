@@ -120,3 +120,9 @@ def test_get_permutation_validation(lib):
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(RuntimeError, match="missing"):
         B.load_library(str(tmp_path / "nope.so"))
+
+
+def test_selftest_argument_checks(lib):
+    assert lib.moe_selftest_wait_timeout(None, 50_000_000, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_selftest_wait_timeout(ctypes.c_void_p(4096), 10, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_selftest_wait_timeout(ctypes.c_void_p(4096), 10**10, None) == B.MOE_ERR_INVALID_ARG

@@ -164,3 +164,25 @@ def test_mixtral_decode_all_tokens():
     wl = WORKLOADS["mixtral_decode"]
     inp, res, perm = run(wl)
     check(wl, inp, res, perm)
+
+
+# ---------------------------------------------------------- failure handling --
+
+def test_bounded_wait_gives_up_and_reports():
+    """A barrier wait that can never complete gives up after its limit and sets
+    MOE_DEV_TIMEOUT; the context stays usable (a forward runs afterwards)."""
+    import ctypes
+    import time
+
+    lib = B.load_library()
+    status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    st = lib.moe_selftest_wait_timeout(ctypes.c_void_p(status.data_ptr()), 50_000_000,
+                                       ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == B.MOE_OK
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 5.0
+    assert int(status.item()) & B.MOE_DEV_TIMEOUT
+    wl = Workload("after_timeout", T=40, d=128, E=4, k=2, I=128, renorm=True, dtype="bf16", router_std=0.3)
+    inp, res, perm = run(wl, seed=11)
+    check(wl, inp, res, perm)
