@@ -8,7 +8,10 @@ lives in ``moe_oracle.c`` and this module only marshals arguments.
 Parity status: every function here is pinned by ``tests/test_oracle.py``
 (brute force on tiny inputs, a dense library SwiGLU for E=1/k=1 and k=E,
 zero-router ties, uniform-routing aux values, the stable-sort dispatch order,
-and the Mixtral parameter count).
+the Mixtral parameter count; for the options: torch's rms_norm and worked
+values of the other RMSNorm form, scipy's logsumexp and closed forms of the
+z-loss, hand-worked capacity cases, and shared experts against a dense torch
+SwiGLU).
 """
 from __future__ import annotations
 
@@ -23,7 +26,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 
-F32, BF16 = 0, 1
+F32, BF16, F64 = 0, 1, 2
 
 _lib = None
 
@@ -41,16 +44,23 @@ def build(force: bool = False) -> str:
 
 
 def _bind(lib):
-    P, I64, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    P, I64, I32, D = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double
     lib.oracle_num_threads.restype = I32
     lib.oracle_set_num_threads.argtypes = [I32]
-    lib.oracle_router_probs.argtypes = [P, P, P, I32, I64, I64, I32, P]
+    lib.oracle_rmsnorm.argtypes = [P, I32, P, I32, I64, I64, D, I32, P]
+    lib.oracle_router_logits.argtypes = [P, I32, P, I32, P, I64, I64, I32, P]
+    lib.oracle_softmax.argtypes = [P, I64, I32, P]
+    lib.oracle_z_loss.argtypes = [P, I64, I32]
+    lib.oracle_z_loss.restype = D
     lib.oracle_gates.argtypes = [P, I64, I32, I32, P, I32, P]
     lib.oracle_topk.argtypes = [P, I64, I32, I32, I32, P, P, P]
     lib.oracle_stats.argtypes = [P, P, I64, I32, I32, P, P, P]
-    lib.oracle_dispatch.argtypes = [P, I64, I32, I32, P, P, P]
-    lib.oracle_expert_rows.argtypes = [P, P, P, P, I32, I64, I64, I64, P, P, I32, P]
-    lib.oracle_moe_tokens.argtypes = [P, P, P, P, I32, I64, I64, I32, I64, P, P, P, I32, P]
+    lib.oracle_capacity.argtypes = [D, I64, I32, I32]
+    lib.oracle_capacity.restype = I64
+    lib.oracle_dispatch.argtypes = [P, I64, I32, I32, I64, P, P, P]
+    lib.oracle_dispatch.restype = I64
+    lib.oracle_expert_rows.argtypes = [P, I32, P, P, P, I32, I64, I64, I64, P, P, I32, P]
+    lib.oracle_moe_tokens.argtypes = [P, I32, P, P, P, I32, I64, I64, I32, I64, P, P, P, P, I32, P, P, P, I32, P]
     return lib
 
 
@@ -91,15 +101,19 @@ def _as_stored(a):
                 return a.view(torch.int16).numpy().view(np.uint16), BF16
             if a.dtype == torch.float32:
                 return a.numpy(), F32
-            raise TypeError(f"oracle takes fp32 or bf16 tensors, got {a.dtype}")
+            if a.dtype == torch.float64:
+                return a.numpy(), F64
+            raise TypeError(f"oracle takes fp32, bf16 or fp64 tensors, got {a.dtype}")
     except ImportError:  # pragma: no cover - torch is always present here
         pass
     a = np.ascontiguousarray(a)
     if a.dtype == np.float32:
         return a, F32
+    if a.dtype == np.float64:
+        return a, F64
     if a.dtype == np.uint16:
         return a, BF16
-    raise TypeError(f"oracle takes float32 or bf16-bit (uint16) arrays, got {a.dtype}")
+    raise TypeError(f"oracle takes float32, float64 or bf16-bit (uint16) arrays, got {a.dtype}")
 
 
 def _ptr(a: np.ndarray | None):
@@ -114,18 +128,56 @@ def set_num_threads(n: int) -> None:
     _load().oracle_set_num_threads(int(n))
 
 
-def router_probs(x, w_router, b_router=None) -> np.ndarray:
-    """Softmax router probabilities ``[T, E]`` in fp64."""
+def rmsnorm(x, weight=None, eps: float = 1e-5, form: int = 1) -> np.ndarray:
+    """The pre-MoE RMSNorm of every token in fp64: form 1 is torch's
+    nn.RMSNorm (eps under the root), form 2 the page's w*x/(rms+eps)."""
     lib = _load()
     xs, dt = _as_stored(x)
-    ws, dt2 = _as_stored(w_router)
-    assert dt == dt2, "x and router weight must share a dtype"
+    T, d = xs.shape
+    ws, wdt = (None, 0) if weight is None else _as_stored(weight)
+    out = np.empty((T, d), dtype=np.float64)
+    lib.oracle_rmsnorm(_ptr(xs), dt, _ptr(ws), wdt, T, d, float(eps), int(form), _ptr(out))
+    return out
+
+
+def router_logits(x, w_router, b_router=None) -> np.ndarray:
+    """Router logits ``[T, E]`` in fp64 (bias included)."""
+    lib = _load()
+    xs, dt = _as_stored(x)
+    ws, wdt = _as_stored(w_router)
     T, d = xs.shape
     E = ws.shape[0]
     b = None if b_router is None else np.ascontiguousarray(np.asarray(b_router, dtype=np.float32))
+    logits = np.empty((T, E), dtype=np.float64)
+    lib.oracle_router_logits(_ptr(xs), dt, _ptr(ws), wdt, _ptr(b), T, d, E, _ptr(logits))
+    return logits
+
+
+def softmax(logits: np.ndarray) -> np.ndarray:
+    lib = _load()
+    logits = np.ascontiguousarray(logits, dtype=np.float64)
+    T, E = logits.shape
     probs = np.empty((T, E), dtype=np.float64)
-    lib.oracle_router_probs(_ptr(xs), _ptr(ws), _ptr(b), dt, T, d, E, _ptr(probs))
+    lib.oracle_softmax(_ptr(logits), T, E, _ptr(probs))
     return probs
+
+
+def router_probs(x, w_router, b_router=None) -> np.ndarray:
+    """Softmax router probabilities ``[T, E]`` in fp64."""
+    return softmax(router_logits(x, w_router, b_router))
+
+
+def z_loss(logits: np.ndarray) -> float:
+    """Router z-loss statistic: mean over tokens of logsumexp(logits)^2."""
+    lib = _load()
+    logits = np.ascontiguousarray(logits, dtype=np.float64)
+    T, E = logits.shape
+    return float(lib.oracle_z_loss(_ptr(logits), T, E))
+
+
+def capacity(capacity_factor: float, T: int, k: int, E: int) -> int:
+    """Assignments an expert may keep, or -1 (no limit) when the factor is <= 0."""
+    return int(_load().oracle_capacity(float(capacity_factor), T, k, E))
 
 
 def topk(probs: np.ndarray, k: int, renorm: bool):
@@ -166,23 +218,24 @@ def stats(probs: np.ndarray, idx: np.ndarray):
     return counts, mean_prob, float(aux[0])
 
 
-def dispatch(idx: np.ndarray, E: int):
-    """(offsets int64 [E+1], perm_tok int32 [T*k], inv int32 [T,k])."""
+def dispatch(idx: np.ndarray, E: int, cap: int = -1):
+    """(offsets int64 [E+1], perm_tok int32 [R], inv int32 [T,k], dropped):
+    R kept rows; inv is -1 for a dropped slot; cap < 0 keeps everything."""
     lib = _load()
     idx = np.ascontiguousarray(idx, dtype=np.int32)
     T, k = idx.shape
     offsets = np.zeros((E + 1,), dtype=np.int64)
     perm = np.zeros((T * k,), dtype=np.int32)
     inv = np.zeros((T, k), dtype=np.int32)
-    lib.oracle_dispatch(_ptr(idx), T, k, E, _ptr(offsets), _ptr(perm), _ptr(inv))
-    return offsets, perm, inv
+    dropped = lib.oracle_dispatch(_ptr(idx), T, k, E, int(cap), _ptr(offsets), _ptr(perm), _ptr(inv))
+    return offsets, perm[:int(offsets[E])].copy(), inv, int(dropped)
 
 
 def expert_rows(x, w_gate, w_up, w_down, tok, expert, h_round: bool = False) -> np.ndarray:
     """``SwiGLU_e(x[t])`` in fp64 for each requested (token, expert) row."""
     lib = _load()
-    xs, dt = _as_stored(x)
-    g, _ = _as_stored(w_gate)
+    xs, xdt = _as_stored(x)
+    g, dt = _as_stored(w_gate)
     u, _ = _as_stored(w_up)
     dn, _ = _as_stored(w_down)
     d = xs.shape[1]
@@ -191,16 +244,19 @@ def expert_rows(x, w_gate, w_up, w_down, tok, expert, h_round: bool = False) -> 
     expert = np.ascontiguousarray(expert, dtype=np.int32)
     n = tok.shape[0]
     y = np.empty((n, d), dtype=np.float64)
-    lib.oracle_expert_rows(_ptr(xs), _ptr(g), _ptr(u), _ptr(dn), dt, d, I, n, _ptr(tok), _ptr(expert),
+    lib.oracle_expert_rows(_ptr(xs), xdt, _ptr(g), _ptr(u), _ptr(dn), dt, d, I, n, _ptr(tok), _ptr(expert),
                            int(h_round), _ptr(y))
     return y
 
 
-def moe_tokens(x, w_gate, w_up, w_down, tok, idx, gate, h_round: bool = False) -> np.ndarray:
-    """``out[i] = sum_j gate[i,j] * SwiGLU_{idx[i,j]}(x[tok[i]])`` in fp64."""
+def moe_tokens(x, w_gate, w_up, w_down, tok, idx, gate, h_round: bool = False, keep=None,
+               shared=None) -> np.ndarray:
+    """``out[i] = sum_j keep[i,j] gate[i,j] SwiGLU_{idx[i,j]}(x[tok[i]])
+    + sum_s SharedSwiGLU_s(x[tok[i]])`` in fp64. ``shared`` is None or the
+    (gate [S,I,d], up [S,I,d], down [S,d,I]) weights of the shared experts."""
     lib = _load()
-    xs, dt = _as_stored(x)
-    g, _ = _as_stored(w_gate)
+    xs, xdt = _as_stored(x)
+    g, dt = _as_stored(w_gate)
     u, _ = _as_stored(w_up)
     dn, _ = _as_stored(w_down)
     d = xs.shape[1]
@@ -209,9 +265,19 @@ def moe_tokens(x, w_gate, w_up, w_down, tok, idx, gate, h_round: bool = False) -
     idx = np.ascontiguousarray(idx, dtype=np.int32)
     gate = np.ascontiguousarray(gate, dtype=np.float64)
     ntok, k = idx.shape
+    kp = None if keep is None else np.ascontiguousarray(keep, dtype=np.int8)
+    if shared is not None:
+        sg, sgdt = _as_stored(shared[0])
+        su, _ = _as_stored(shared[1])
+        sd, _ = _as_stored(shared[2])
+        assert sgdt == dt, "shared and routed experts must share a dtype"
+        ns = sg.shape[0]
+    else:
+        sg = su = sd = None
+        ns = 0
     out = np.empty((ntok, d), dtype=np.float64)
-    lib.oracle_moe_tokens(_ptr(xs), _ptr(g), _ptr(u), _ptr(dn), dt, d, I, k, ntok, _ptr(tok), _ptr(idx),
-                          _ptr(gate), int(h_round), _ptr(out))
+    lib.oracle_moe_tokens(_ptr(xs), xdt, _ptr(g), _ptr(u), _ptr(dn), dt, d, I, k, ntok, _ptr(tok), _ptr(idx),
+                          _ptr(gate), _ptr(kp), ns, _ptr(sg), _ptr(su), _ptr(sd), int(h_round), _ptr(out))
     return out
 
 
@@ -221,27 +287,48 @@ class OracleResult:
     topk_idx: np.ndarray  # [T, k] int32
     topk_gate: np.ndarray  # [T, k] fp64
     gap: np.ndarray  # [T] fp64, p_(k) - p_(k+1)
-    counts: np.ndarray  # [E] int64
+    counts: np.ndarray  # [E] int64, assignments before any capacity drop
     mean_prob: np.ndarray  # [E] fp64
     aux: float
-    offsets: np.ndarray  # [E+1] int64
-    perm_tok: np.ndarray  # [T*k] int32
-    inv: np.ndarray  # [T, k] int32
+    offsets: np.ndarray  # [E+1] int64, of the kept rows
+    perm_tok: np.ndarray  # [R] int32, R kept rows
+    inv: np.ndarray  # [T, k] int32, -1 for a dropped slot
     tokens: np.ndarray  # [n] int32, the tokens whose output rows were evaluated
     out: np.ndarray  # [n, d] fp64
+    logits: np.ndarray = None  # [T, E] fp64
+    z_loss: float = 0.0
+    capacity: int = -1  # assignments an expert may keep, -1 = no limit
+    dropped: int = 0  # assignments dropped by the capacity
+    xhat: np.ndarray = None  # [T, d] fp64 normalised input, when a norm was applied
 
 
 def forward(x, w_router, b_router, w_gate, w_up, w_down, k: int, renorm: bool, tokens=None,
-            h_round: bool = False) -> OracleResult:
+            h_round: bool = False, *, norm_form: int = 0, norm_weight=None, norm_eps: float = 1e-5,
+            capacity_factor: float = 0.0, shared=None) -> OracleResult:
     """The whole layer. Routing, statistics and dispatch cover every token;
-    the expert output is evaluated for ``tokens`` (all tokens if None)."""
-    probs = router_probs(x, w_router, b_router)
+    the expert output is evaluated for ``tokens`` (all tokens if None).
+
+    Options: ``norm_form`` 1 or 2 applies the pre-MoE RMSNorm (weight
+    ``norm_weight`` or ones, ``norm_eps``) before the router and the experts;
+    ``capacity_factor`` > 0 caps every expert at ceil(cf*T*k/E) assignments;
+    ``shared`` = (gate, up, down) adds shared experts with weight 1."""
+    xin = x
+    xhat = None
+    if norm_form:
+        xhat = rmsnorm(x, norm_weight, norm_eps, norm_form)
+        xin = xhat
+    logits = router_logits(xin, w_router, b_router)
+    probs = softmax(logits)
     T, E = probs.shape
     idx, gate, gap = topk(probs, k, renorm)
     counts, mean_prob, aux = stats(probs, idx)
-    offsets, perm, inv = dispatch(idx, E)
+    cap = capacity(capacity_factor, T, k, E)
+    offsets, perm, inv, dropped = dispatch(idx, E, cap)
     if tokens is None:
         tokens = np.arange(T, dtype=np.int32)
     tokens = np.asarray(tokens, dtype=np.int32)
-    out = moe_tokens(x, w_gate, w_up, w_down, tokens, idx[tokens], gate[tokens], h_round=h_round)
-    return OracleResult(probs, idx, gate, gap, counts, mean_prob, aux, offsets, perm, inv, tokens, out)
+    keep = (inv[tokens] >= 0) if cap >= 0 else None
+    out = moe_tokens(xin, w_gate, w_up, w_down, tokens, idx[tokens], gate[tokens], h_round=h_round, keep=keep,
+                     shared=shared)
+    return OracleResult(probs, idx, gate, gap, counts, mean_prob, aux, offsets, perm, inv, tokens, out,
+                        logits=logits, z_loss=z_loss(logits), capacity=cap, dropped=dropped, xhat=xhat)

@@ -46,6 +46,29 @@
  *                 MoELayer::forward ("Scatter weighted outputs back");
  *                 Mixtral MoE Block markdown, _moe_forward.
  *
+ * Options of the layer that the pages name as configuration knobs:
+ *
+ *   RMSNorm       the block applies RMSNorm before the MoE layer (Mixtral MoE
+ *                 Block, layer table "post_attn_norm", nn.RMSNorm). Form 1 is
+ *                 torch's nn.RMSNorm, x / sqrt(mean(x^2) + eps) * w; form 2 is
+ *                 the one printed under Model Architecture Patterns, "RMSNorm
+ *                 (no bias, no mean centering)": w * x / (||x|| / sqrt(d) + eps).
+ *                 The router and every expert then see the normalised x.
+ *   z-loss        the router z-loss statistic of ST-MoE that the training
+ *                 config enables ("moe_router_z_loss_weight"; the Mixtral
+ *                 page's note on the router z-loss): mean over tokens of
+ *                 (logsumexp_e logits[t,e])^2, on the logits with their bias.
+ *   capacity      "moe_capacity_factor: 0 = no drop, > 0 = cap tokens per
+ *                 expert": capacity C = ceil(cf * T * k / E) assignments per
+ *                 expert; an expert keeps its first C assignments in dispatch
+ *                 order (tokens ascending) and drops the rest, whose slots
+ *                 then contribute nothing to the output. Routing, gates,
+ *                 counts and the balance statistic are those before dropping.
+ *   shared        "moe_shared_experts: shared experts that process all
+ *                 tokens", each the same SwiGLU MLP as a routed expert
+ *                 (the parameter count adds n_shared * expert_mlp); their
+ *                 outputs are added to every token with weight 1.
+ *
  * Inputs are read as stored (fp32, or bf16 bit patterns widened exactly to
  * fp64). All arithmetic is fp64. OpenMP parallelises over independent tokens
  * or rows only; no step is blocked, fused or reordered beyond the definition.
@@ -58,10 +81,11 @@
 #include <omp.h>
 #endif
 
-enum { ORACLE_F32 = 0, ORACLE_BF16 = 1 };
+enum { ORACLE_F32 = 0, ORACLE_BF16 = 1, ORACLE_F64 = 2 };
 
 /* Exact widening of one stored element to fp64. */
 static double load_elem(const void* base, int dtype, int64_t i) {
+  if (dtype == ORACLE_F64) return ((const double*)base)[i];
   if (dtype == ORACLE_F32) return (double)((const float*)base)[i];
   uint32_t bits = ((uint32_t)((const uint16_t*)base)[i]) << 16;
   float f;
@@ -102,31 +126,78 @@ void oracle_set_num_threads(int n) {
 #endif
 }
 
-/* ---- router: logits and softmax ------------------------------------------ */
+/* ---- pre-MoE RMSNorm ------------------------------------------------------ */
 
-/* probs[t*E + e] for every token. */
-void oracle_router_probs(const void* x, const void* w_router, const float* b_router,
-                         int dtype, int64_t T, int64_t d, int E, double* probs) {
+/* xhat[t*d + c] = x[t,c] * r_t * w[c] with r_t = 1 / sqrt(mean_c x^2 + eps)
+ * (form 1) or 1 / (sqrt(mean_c x^2) + eps) (form 2); w = 1 when NULL. */
+void oracle_rmsnorm(const void* x, int x_dtype, const void* weight, int w_dtype, int64_t T, int64_t d,
+                    double eps, int form, double* xhat) {
 #pragma omp parallel for schedule(static)
   for (int64_t t = 0; t < T; ++t) {
-    double* p = probs + t * E;
+    double ss = 0.0;
+    for (int64_t c = 0; c < d; ++c) {
+      const double v = load_elem(x, x_dtype, t * d + c);
+      ss += v * v;
+    }
+    const double ms = ss / (double)d;
+    const double r = form == 1 ? 1.0 / sqrt(ms + eps) : 1.0 / (sqrt(ms) + eps);
+    for (int64_t c = 0; c < d; ++c) {
+      const double w = weight ? load_elem(weight, w_dtype, c) : 1.0;
+      xhat[t * d + c] = load_elem(x, x_dtype, t * d + c) * r * w;
+    }
+  }
+}
+
+/* ---- router: logits, softmax, z-loss ---------------------------------------- */
+
+/* logits[t*E + e] = sum_c x[t,c] * Wr[e,c] (+ b[e]). */
+void oracle_router_logits(const void* x, int x_dtype, const void* w_router, int w_dtype, const float* b_router,
+                          int64_t T, int64_t d, int E, double* logits) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
     for (int e = 0; e < E; ++e) {
       double acc = 0.0;
       for (int64_t c = 0; c < d; ++c)
-        acc += load_elem(x, dtype, t * d + c) * load_elem(w_router, dtype, (int64_t)e * d + c);
+        acc += load_elem(x, x_dtype, t * d + c) * load_elem(w_router, w_dtype, (int64_t)e * d + c);
       if (b_router) acc += (double)b_router[e];
-      p[e] = acc; /* logit for now */
+      logits[t * E + e] = acc;
     }
-    double m = p[0];
+  }
+}
+
+/* probs[t*E + e] = exp(l - max l) / sum exp(l - max l), per token. */
+void oracle_softmax(const double* logits, int64_t T, int E, double* probs) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
+    const double* l = logits + t * E;
+    double* p = probs + t * E;
+    double m = l[0];
     for (int e = 1; e < E; ++e)
-      if (p[e] > m) m = p[e];
+      if (l[e] > m) m = l[e];
     double s = 0.0;
     for (int e = 0; e < E; ++e) {
-      p[e] = exp(p[e] - m);
+      p[e] = exp(l[e] - m);
       s += p[e];
     }
     for (int e = 0; e < E; ++e) p[e] /= s;
   }
+}
+
+/* mean_t (log sum_e exp logits[t,e])^2; 0 when T = 0. */
+double oracle_z_loss(const double* logits, int64_t T, int E) {
+  if (T == 0) return 0.0;
+  double acc = 0.0;
+  for (int64_t t = 0; t < T; ++t) {
+    const double* l = logits + t * E;
+    double m = l[0];
+    for (int e = 1; e < E; ++e)
+      if (l[e] > m) m = l[e];
+    double s = 0.0;
+    for (int e = 0; e < E; ++e) s += exp(l[e] - m);
+    const double lse = m + log(s);
+    acc += lse * lse;
+  }
+  return acc / (double)T;
 }
 
 /* ---- top-k ---------------------------------------------------------------- */
@@ -207,33 +278,51 @@ void oracle_stats(const double* probs, const int32_t* topk_idx, int64_t T, int E
   *aux = (double)E * s;
 }
 
-/* ---- dispatch order ------------------------------------------------------- */
+/* ---- dispatch order and capacity ------------------------------------------- */
+
+/* Assignments an expert may keep: ceil(cf * T * k / E), or -1 (no limit) when
+ * cf <= 0. */
+int64_t oracle_capacity(double cf, int64_t T, int k, int E) {
+  if (!(cf > 0.0)) return -1;
+  return (int64_t)ceil(cf * (double)T * (double)k / (double)E);
+}
 
 /* offsets[E+1]; perm_tok[R] = token of each dispatched row; inv[T*k] = row of
- * each (token, slot). Rows are expert-contiguous, tokens ascending within an
- * expert. */
-void oracle_dispatch(const int32_t* topk_idx, int64_t T, int k, int E, int64_t* offsets,
-                     int32_t* perm_tok, int32_t* inv) {
-  int64_t row = 0;
+ * each (token, slot), or -1 when the slot was dropped. Rows are
+ * expert-contiguous, tokens ascending within an expert; with capacity >= 0 an
+ * expert keeps only its first `capacity` assignments in that order. Returns
+ * the number of dropped assignments. */
+int64_t oracle_dispatch(const int32_t* topk_idx, int64_t T, int k, int E, int64_t capacity, int64_t* offsets,
+                        int32_t* perm_tok, int32_t* inv) {
+  int64_t row = 0, dropped = 0;
   for (int e = 0; e < E; ++e) {
     offsets[e] = row;
+    int64_t taken = 0;
     for (int64_t t = 0; t < T; ++t)
       for (int j = 0; j < k; ++j)
         if (topk_idx[t * k + j] == e) {
+          if (capacity >= 0 && taken >= capacity) {
+            inv[t * k + j] = -1;
+            ++dropped;
+            continue;
+          }
           perm_tok[row] = (int32_t)t;
           inv[t * k + j] = (int32_t)row;
           ++row;
+          ++taken;
         }
   }
   offsets[E] = row;
+  return dropped;
 }
 
 /* ---- expert SwiGLU MLP ---------------------------------------------------- */
 
 /* y[r, :] = down_e(SiLU(gate_e(x_t)) * up_e(x_t)) for each requested row
- * (t = tok[r], e = expert[r]). h_round = 1 rounds the hidden activation to
+ * (t = tok[r], e = expert[r]); x is read as x_dtype, the weights as dtype.
+ * h_round = 1 rounds the hidden activation to
  * bf16 (a diagnostic mode; parity is judged with h_round = 0). */
-void oracle_expert_rows(const void* x, const void* w_gate, const void* w_up, const void* w_down,
+void oracle_expert_rows(const void* x, int x_dtype, const void* w_gate, const void* w_up, const void* w_down,
                         int dtype, int64_t d, int64_t I, int64_t n, const int32_t* tok,
                         const int32_t* expert, int h_round, double* y) {
 #pragma omp parallel
@@ -244,7 +333,7 @@ void oracle_expert_rows(const void* x, const void* w_gate, const void* w_up, con
     for (int64_t r = 0; r < n; ++r) {
       const int64_t t = tok[r];
       const int64_t e = expert[r];
-      for (int64_t c = 0; c < d; ++c) xv[c] = load_elem(x, dtype, t * d + c);
+      for (int64_t c = 0; c < d; ++c) xv[c] = load_elem(x, x_dtype, t * d + c);
       for (int64_t i = 0; i < I; ++i) {
         const int64_t wrow = (e * I + i) * d;
         double g = 0.0, u = 0.0;
@@ -270,23 +359,42 @@ void oracle_expert_rows(const void* x, const void* w_gate, const void* w_up, con
 
 /* ---- combine -------------------------------------------------------------- */
 
-/* out[i, :] = sum_j gate[i,j] * expert_{idx[i,j]}(x[tok[i]]) for a list of
- * tokens with their chosen experts and gates. */
-void oracle_moe_tokens(const void* x, const void* w_gate, const void* w_up, const void* w_down,
+/* out[i, :] = sum_j keep[i,j] * gate[i,j] * expert_{idx[i,j]}(x[tok[i]])
+ *           + sum_s shared_s(x[tok[i]])
+ * for a list of tokens with their chosen experts and gates. keep == NULL keeps
+ * every slot; n_shared shared experts (weights [n_shared, I, d] and
+ * [n_shared, d, I]) are added with weight 1. */
+void oracle_moe_tokens(const void* x, int x_dtype, const void* w_gate, const void* w_up, const void* w_down,
                        int dtype, int64_t d, int64_t I, int k, int64_t ntok, const int32_t* tok,
-                       const int32_t* idx, const double* gate, int h_round, double* out) {
+                       const int32_t* idx, const double* gate, const int8_t* keep, int n_shared,
+                       const void* s_gate, const void* s_up, const void* s_down, int h_round, double* out) {
   const int64_t n = ntok * k;
+  const int64_t ns = ntok * n_shared;
   int32_t* rtok = (int32_t*)malloc(sizeof(int32_t) * (size_t)(n > 0 ? n : 1));
   double* y = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n * d : 1));
+  int32_t* stok = (int32_t*)malloc(sizeof(int32_t) * (size_t)(ns > 0 ? ns : 1));
+  int32_t* sexp = (int32_t*)malloc(sizeof(int32_t) * (size_t)(ns > 0 ? ns : 1));
+  double* ys = (double*)malloc(sizeof(double) * (size_t)(ns > 0 ? ns * d : 1));
   for (int64_t i = 0; i < ntok; ++i)
     for (int j = 0; j < k; ++j) rtok[i * k + j] = tok[i];
-  oracle_expert_rows(x, w_gate, w_up, w_down, dtype, d, I, n, rtok, idx, h_round, y);
+  oracle_expert_rows(x, x_dtype, w_gate, w_up, w_down, dtype, d, I, n, rtok, idx, h_round, y);
+  for (int64_t i = 0; i < ntok; ++i)
+    for (int s = 0; s < n_shared; ++s) {
+      stok[i * n_shared + s] = tok[i];
+      sexp[i * n_shared + s] = s;
+    }
+  if (ns > 0) oracle_expert_rows(x, x_dtype, s_gate, s_up, s_down, dtype, d, I, ns, stok, sexp, h_round, ys);
   for (int64_t i = 0; i < ntok; ++i)
     for (int64_t c = 0; c < d; ++c) {
       double acc = 0.0;
-      for (int j = 0; j < k; ++j) acc += gate[i * k + j] * y[(i * k + j) * d + c];
+      for (int j = 0; j < k; ++j)
+        if (!keep || keep[i * k + j]) acc += gate[i * k + j] * y[(i * k + j) * d + c];
+      for (int s = 0; s < n_shared; ++s) acc += ys[(i * n_shared + s) * d + c];
       out[i * d + c] = acc;
     }
   free(rtok);
   free(y);
+  free(stok);
+  free(sexp);
+  free(ys);
 }

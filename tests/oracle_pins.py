@@ -254,7 +254,7 @@ def pin_dispatch_stable_sort():
     T, E, k = 37, 6, 3
     rng = np.random.default_rng(5)
     idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
-    offsets, perm, inv = oracle.dispatch(idx, E)
+    offsets, perm, inv, _ = oracle.dispatch(idx, E)
     order = np.argsort(idx.reshape(-1), kind="stable")
     np.testing.assert_array_equal(perm, order // k)
     expect_inv = np.empty(T * k, dtype=np.int64)
@@ -332,6 +332,152 @@ def pin_gap_definition():
     assert np.all(np.isinf(gapE))
 
 
+# ---------------------------------------------------------------------------
+# pins of the layer's options: pre-MoE RMSNorm, z-loss, capacity, shared experts
+# ---------------------------------------------------------------------------
+
+def pin_rmsnorm_torch_form():
+    """Form 1 is torch's nn.RMSNorm: against torch.nn.functional.rms_norm in
+    fp64 (a library routine), with and without a weight, two eps values."""
+    g = torch.Generator().manual_seed(31)
+    x = torch.randn((9, 24), generator=g).to(torch.bfloat16)
+    w = (1.0 + 0.3 * torch.randn((24,), generator=g)).to(torch.bfloat16)
+    for eps in (1e-5, 0.5):
+        ref = F.rms_norm(x.double(), (24,), w.double(), eps).numpy()
+        np.testing.assert_allclose(oracle.rmsnorm(x, w, eps, form=1), ref, rtol=0, atol=1e-14)
+        ref1 = F.rms_norm(x.double(), (24,), None, eps).numpy()
+        np.testing.assert_allclose(oracle.rmsnorm(x, None, eps, form=1), ref1, rtol=0, atol=1e-14)
+
+
+def pin_rmsnorm_worked_values():
+    """x = (3, 4), w = (1, 2), eps = 0.5, worked by hand.
+    Form 2 (eps outside the root, as printed under Model Architecture
+    Patterns): rms = 5/sqrt(2) = 3.5355..., x_hat = w*x / 4.0355... =
+    (0.74339..., 1.98238...). Form 1 (torch): 1/sqrt(12.5 + 0.5) = 0.27735...,
+    x_hat = (0.83205..., 2.21880...). With eps = 0 and unit weight both forms
+    give mean(x_hat^2) = 1 and are invariant to scaling x."""
+    x = torch.tensor([[3.0, 4.0]])
+    w = torch.tensor([1.0, 2.0])
+    np.testing.assert_allclose(oracle.rmsnorm(x, w, 0.5, form=2)[0], [0.7433960585957724, 1.9823894895887266],
+                               rtol=1e-15)
+    np.testing.assert_allclose(oracle.rmsnorm(x, w, 0.5, form=1)[0], [0.8320502943378437, 2.2188007849009166],
+                               rtol=1e-15)
+    g = torch.Generator().manual_seed(32)
+    xr = torch.randn((5, 16), generator=g)
+    for form in (1, 2):
+        a = oracle.rmsnorm(xr, None, 0.0, form=form)
+        np.testing.assert_allclose((a * a).mean(axis=1), 1.0, rtol=1e-14)
+        np.testing.assert_allclose(oracle.rmsnorm(xr * 4.0, None, 0.0, form=form), a, rtol=1e-14)
+
+
+def pin_norm_feeds_router_and_experts():
+    """With the norm on, the whole layer equals the brute-force layer applied
+    to torch's rms_norm(x) (fp64), router and experts alike."""
+    T, d, E, k, I = 8, 16, 4, 2, 12
+    x, wr, b, wg, wu, wd = _rand_case(T, d, E, k, I, "bf16", 33, bias=True)
+    w = (1.0 + 0.2 * torch.randn((d,), generator=torch.Generator().manual_seed(34))).to(torch.bfloat16)
+    xh = F.rms_norm(x.double(), (d,), w.double(), 1e-5)
+    bp, bidx, bg, bout = brute_force(xh, wr, b, wg, wu, wd, k, True)
+    r = oracle.forward(x, wr, b, wg, wu, wd, k, True, norm_form=1, norm_weight=w, norm_eps=1e-5)
+    np.testing.assert_allclose(r.probs, bp, rtol=0, atol=1e-13)
+    np.testing.assert_array_equal(r.topk_idx, bidx)
+    np.testing.assert_allclose(r.out, bout, rtol=0, atol=1e-11 * max(1.0, float(np.abs(bout).max())))
+
+
+def pin_z_loss_closed_forms():
+    """Zero logits: (ln E)^2. Router weights zero and bias (0, ln 3): every
+    token's logsumexp is ln 4, so z = (ln 4)^2. Two tokens with logits
+    (a, a, a, a) and (L, L, L, L): z = ((a + ln 4)^2 + (L + ln 4)^2) / 2, a mean
+    over tokens, not a sum."""
+    np.testing.assert_allclose(oracle.z_loss(np.zeros((7, 8))), 4.324077125263812, rtol=1e-15)
+    x = torch.randn((6, 4), generator=torch.Generator().manual_seed(35))
+    wr = torch.zeros((2, 4))
+    b = torch.tensor([0.0, math.log(3.0)])
+    w3 = torch.zeros((2, 1, 4))
+    wd3 = torch.zeros((2, 4, 1))
+    r = oracle.forward(x, wr, b, w3, w3, wd3, 1, True)
+    np.testing.assert_allclose(r.z_loss, 1.9218120556728056, rtol=1e-7)  # b is stored in fp32
+    a, L = -1.5, 30.0
+    lg = np.array([[a] * 4, [L] * 4])
+    np.testing.assert_allclose(oracle.z_loss(lg), ((a + math.log(4)) ** 2 + (L + math.log(4)) ** 2) / 2, rtol=1e-15)
+    assert oracle.z_loss(np.zeros((0, 3))) == 0.0
+
+
+def pin_z_loss_scipy():
+    """Against scipy.special.logsumexp on random logits with a bias."""
+    from scipy.special import logsumexp
+
+    x, wr, b, *_ = _rand_case(33, 12, 6, 2, 4, "f32", 36, bias=True)
+    lg = oracle.router_logits(x, wr, b)
+    ref = _f64(x) @ _f64(wr).T + _f64(b)
+    np.testing.assert_allclose(lg, ref, rtol=0, atol=1e-12)
+    lse = logsumexp(ref, axis=1)
+    np.testing.assert_allclose(oracle.z_loss(lg), np.mean(lse * lse), rtol=1e-14)
+
+
+def pin_capacity_values():
+    """C = ceil(cf * T * k / E): 10 tokens, k = 1, E = 4, cf = 1 gives 3 (2.5
+    rounded up); cf = 1.25 at T = 4096, k = 2, E = 8 gives 1280; cf = 0.5 at
+    T = 7, k = 2, E = 3 gives 3 (2.33 rounded up); cf = 0 means no limit."""
+    assert oracle.capacity(1.0, 10, 1, 4) == 3
+    assert oracle.capacity(1.25, 4096, 2, 8) == 1280
+    assert oracle.capacity(0.5, 7, 2, 3) == 3
+    assert oracle.capacity(0.0, 10, 1, 4) == -1
+
+
+def pin_capacity_dispatch_worked():
+    """A hand-worked drop with C = 2. Assignments per expert in token order:
+    e0: t0 t1 t2 t3 t5 -> keeps t0 t1; e1: t0 t2 t4 t5 -> keeps t0 t2;
+    e2: t1 t3 t4 -> keeps t1 t3. Six slots are dropped."""
+    idx = np.array([[0, 1], [0, 2], [1, 0], [2, 0], [1, 2], [0, 1]], dtype=np.int32)
+    offsets, perm, inv, dropped = oracle.dispatch(idx, 3, cap=2)
+    np.testing.assert_array_equal(offsets, [0, 2, 4, 6])
+    np.testing.assert_array_equal(perm, [0, 1, 0, 2, 1, 3])
+    np.testing.assert_array_equal(inv, [[0, 2], [1, 4], [3, -1], [5, -1], [-1, -1], [-1, -1]])
+    assert dropped == 6
+    # no limit: the plain dispatch
+    offsets, perm, inv, dropped = oracle.dispatch(idx, 3)
+    np.testing.assert_array_equal(offsets, [0, 5, 9, 12])
+    assert dropped == 0 and inv.min() == 0
+
+
+def pin_capacity_layer():
+    """Every token routed to expert 0 (bias), k = 1, cf = 1 over E = 4 with
+    T = 10: C = 3, so tokens 0-2 get gate * SwiGLU_0(x) (dense torch) and the
+    other 7 get zero; counts and the statistic are those before dropping.
+    A factor large enough to keep everything gives the plain layer."""
+    T, d, E, I = 10, 8, 4, 6
+    x, wr, _, wg, wu, wd = _rand_case(T, d, E, 1, I, "f32", 37, router_std=0.01)
+    b = torch.tensor([20.0, 0.0, 0.0, 0.0])
+    r = oracle.forward(x, wr, b, wg, wu, wd, 1, False, capacity_factor=1.0)
+    assert r.capacity == 3 and r.dropped == 7
+    np.testing.assert_array_equal(r.counts, [10, 0, 0, 0])
+    dense = dense_swiglu_torch(x, wg[0], wu[0], wd[0]).numpy() * r.topk_gate[:, :1]
+    np.testing.assert_allclose(r.out[:3], dense[:3], rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(r.out[3:], 0.0)
+    np.testing.assert_array_equal(r.inv[:, 0], [0, 1, 2] + [-1] * 7)
+    plain = oracle.forward(x, wr, b, wg, wu, wd, 1, False)
+    big = oracle.forward(x, wr, b, wg, wu, wd, 1, False, capacity_factor=4.0)
+    assert big.dropped == 0
+    np.testing.assert_array_equal(big.out, plain.out)
+
+
+def pin_shared_experts():
+    """Shared experts add sum_s SwiGLU_s(x) (dense torch, fp64) to every
+    token, with weight 1, on top of the routed output."""
+    T, d, E, k, I, S = 9, 12, 4, 2, 10, 2
+    x, wr, b, wg, wu, wd = _rand_case(T, d, E, k, I, "bf16", 38, bias=True)
+    g = torch.Generator().manual_seed(39)
+    sg = (torch.randn((S, I, d), generator=g) * 0.3).to(torch.bfloat16)
+    su = (torch.randn((S, I, d), generator=g) * 0.3).to(torch.bfloat16)
+    sd = (torch.randn((S, d, I), generator=g) * 0.3).to(torch.bfloat16)
+    plain = oracle.forward(x, wr, b, wg, wu, wd, k, True)
+    r = oracle.forward(x, wr, b, wg, wu, wd, k, True, shared=(sg, su, sd))
+    extra = sum(dense_swiglu_torch(x, sg[s], su[s], sd[s]) for s in range(S)).numpy()
+    np.testing.assert_allclose(r.out - plain.out, extra, rtol=0, atol=1e-11 * max(1.0, float(np.abs(extra).max())))
+    np.testing.assert_array_equal(r.topk_idx, plain.topk_idx)
+
+
 ALL_PINS = [
     pin_brute_force,
     pin_gates_sum_to_one,
@@ -346,4 +492,13 @@ ALL_PINS = [
     pin_axonml_unit_tests,
     pin_mixtral_parameter_count,
     pin_gap_definition,
+    pin_rmsnorm_torch_form,
+    pin_rmsnorm_worked_values,
+    pin_norm_feeds_router_and_experts,
+    pin_z_loss_closed_forms,
+    pin_z_loss_scipy,
+    pin_capacity_values,
+    pin_capacity_dispatch_worked,
+    pin_capacity_layer,
+    pin_shared_experts,
 ]

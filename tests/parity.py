@@ -47,7 +47,7 @@ def check(inp, res, perm, k, renorm, dtype, tokens=None, h_round=False, report=N
     probs = oracle.router_probs(x, wr, b)
     idx_o, gate_o, gap = oracle.topk(probs, k, renorm)
     counts_o, _, aux_o = oracle.stats(probs, idx_o)
-    offs_o, perm_o, inv_o = oracle.dispatch(idx_o, E)
+    offs_o, perm_o, inv_o, _ = oracle.dispatch(idx_o, E)
 
     idx_g = _np(res.topk_idx).astype(np.int32)
     gate_g = _np(res.topk_gate).astype(np.float64)
@@ -81,7 +81,7 @@ def check(inp, res, perm, k, renorm, dtype, tokens=None, h_round=False, report=N
     rep["aux"] = aux_g
     rep["aux_oracle"] = aux_o
     assert abs(aux_g - aux_ref) <= 1e-4, f"aux {aux_g} vs {aux_ref}"
-    offs_r, perm_r, inv_r = oracle.dispatch(idx_g, E)
+    offs_r, perm_r, inv_r, _ = oracle.dispatch(idx_g, E)
     np.testing.assert_array_equal(offs_g, offs_r)
     np.testing.assert_array_equal(perm_g, perm_r)
     np.testing.assert_array_equal(inv_g.reshape(T, k), inv_r)

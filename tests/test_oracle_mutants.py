@@ -31,12 +31,30 @@ MUTANTS = [
     ("aux_no_E", "*aux = (double)E * s;", "*aux = s;"),
     ("gap_wrong_slot", "gap[t] = (k < E) ? r[k - 1].p - r[k].p : INFINITY;",
      "gap[t] = (k < E) ? r[0].p - r[k].p : INFINITY;"),
-    ("dispatch_token_descending", "if (topk_idx[t * k + j] == e) {\n          perm_tok[row] = (int32_t)t;",
-     "if (topk_idx[t * k + j] == E - 1 - e) {\n          perm_tok[row] = (int32_t)t;"),
-    ("combine_gate_sum", "for (int j = 0; j < k; ++j) acc += gate[i * k + j] * y[(i * k + j) * d + c];",
-     "for (int j = 0; j < k; ++j) { double gs = 0.0; for (int jj = 0; jj < k; ++jj) gs += gate[i * k + jj];"
+    ("dispatch_token_descending", "if (topk_idx[t * k + j] == e) {", "if (topk_idx[t * k + j] == E - 1 - e) {"),
+    ("combine_gate_sum", "if (!keep || keep[i * k + j]) acc += gate[i * k + j] * y[(i * k + j) * d + c];",
+     "if (!keep || keep[i * k + j]) { double gs = 0.0; for (int jj = 0; jj < k; ++jj) gs += gate[i * k + jj];"
      " acc += gs * y[(i * k + j) * d + c]; }"),
-    ("router_transposed", "load_elem(w_router, dtype, (int64_t)e * d + c)", "load_elem(w_router, dtype, c * E + e)"),
+    ("router_transposed", "load_elem(w_router, w_dtype, (int64_t)e * d + c)",
+     "load_elem(w_router, w_dtype, c * E + e)"),
+    # options: RMSNorm, z-loss, capacity, shared experts
+    ("rms_eps_outside_in_torch_form", "form == 1 ? 1.0 / sqrt(ms + eps) : 1.0 / (sqrt(ms) + eps)",
+     "form == 1 ? 1.0 / (sqrt(ms) + eps) : 1.0 / (sqrt(ms) + eps)"),
+    ("rms_eps_inside_in_page_form", "form == 1 ? 1.0 / sqrt(ms + eps) : 1.0 / (sqrt(ms) + eps)",
+     "form == 1 ? 1.0 / sqrt(ms + eps) : 1.0 / sqrt(ms + eps)"),
+    ("rms_sum_not_mean", "const double ms = ss / (double)d;", "const double ms = ss;"),
+    ("rms_no_weight", "const double w = weight ? load_elem(weight, w_dtype, c) : 1.0;", "const double w = 1.0;"),
+    ("z_not_squared", "acc += lse * lse;", "acc += lse;"),
+    ("z_max_not_lse", "const double lse = m + log(s);", "const double lse = m;"),
+    ("z_sum_not_mean", "return acc / (double)T;", "return acc;"),
+    ("capacity_floor", "return (int64_t)ceil(cf * (double)T * (double)k / (double)E);",
+     "return (int64_t)floor(cf * (double)T * (double)k / (double)E);"),
+    ("capacity_per_token_not_assignment", "return (int64_t)ceil(cf * (double)T * (double)k / (double)E);",
+     "return (int64_t)ceil(cf * (double)T / (double)E);"),
+    ("capacity_off_by_one", "if (capacity >= 0 && taken >= capacity) {", "if (capacity >= 0 && taken > capacity) {"),
+    ("dropped_slot_still_combined", "if (!keep || keep[i * k + j]) acc", "if (1) acc"),
+    ("shared_not_added", "acc += ys[(i * n_shared + s) * d + c];", "acc += 0.0 * ys[(i * n_shared + s) * d + c];"),
+    ("shared_half_weight", "acc += ys[(i * n_shared + s) * d + c];", "acc += 0.5 * ys[(i * n_shared + s) * d + c];"),
 ]
 
 
