@@ -47,6 +47,7 @@ def _bind(lib):
     P, I64, I32, D = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double
     lib.oracle_num_threads.restype = I32
     lib.oracle_set_num_threads.argtypes = [I32]
+    lib.oracle_round_bf16.argtypes = [P, I64, P]
     lib.oracle_rmsnorm.argtypes = [P, I32, P, I32, I64, I64, D, I32, P]
     lib.oracle_router_logits.argtypes = [P, I32, P, I32, P, I64, I64, I32, P]
     lib.oracle_softmax.argtypes = [P, I64, I32, P]
@@ -126,6 +127,15 @@ def num_threads() -> int:
 
 def set_num_threads(n: int) -> None:
     _load().oracle_set_num_threads(int(n))
+
+
+def round_bf16(a) -> np.ndarray:
+    """fp64 values rounded (via fp32) to the nearest bf16, ties to even."""
+    lib = _load()
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    out = np.empty_like(a)
+    lib.oracle_round_bf16(_ptr(a), a.size, _ptr(out))
+    return out
 
 
 def rmsnorm(x, weight=None, eps: float = 1e-5, form: int = 1) -> np.ndarray:

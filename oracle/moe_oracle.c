@@ -110,6 +110,12 @@ static double round_to_bf16(double v) {
   return (double)f;
 }
 
+/* out[i] = in[i] rounded to fp32 and then to the nearest bf16 (ties to even):
+ * how a value computed in fp32 is stored in bf16 (diagnostic comparisons). */
+void oracle_round_bf16(const double* in, int64_t n, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = round_to_bf16(in[i]);
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

@@ -478,6 +478,19 @@ def pin_shared_experts():
     np.testing.assert_array_equal(r.topk_idx, plain.topk_idx)
 
 
+def pin_round_bf16_matches_torch():
+    """The diagnostic bf16 rounding equals torch's fp32 -> bf16 conversion
+    (round to nearest, ties to even), including exact ties."""
+    g = torch.Generator().manual_seed(40)
+    v = torch.randn((4096,), generator=g) * 3.0
+    ties = torch.tensor([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8), 2.0 + 2.0 ** -7, 0.0, -0.0])
+    v = torch.cat([v, ties])
+    got = oracle.round_bf16(v.double().numpy())
+    ref = v.to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(got, ref)
+    assert got[-6] == 1.0 and got[-5] == 1.0 + 2.0 ** -6
+
+
 ALL_PINS = [
     pin_brute_force,
     pin_gates_sum_to_one,
@@ -501,4 +514,5 @@ ALL_PINS = [
     pin_capacity_dispatch_worked,
     pin_capacity_layer,
     pin_shared_experts,
+    pin_round_bf16_matches_torch,
 ]

@@ -1,9 +1,12 @@
 """Element-by-element comparison of the CUDA path with the fp64 oracle.
 
 Rules:
-  * Top-k indices and the dispatch order must match the oracle exactly on
-    every token whose oracle gap p_(k) - p_(k+1) exceeds 1e-4; the count of
-    excluded near-tie tokens is reported. For excluded tokens the GPU's choice
+  * Top-k indices (best first) and the dispatch order must match the oracle
+    exactly on every token whose sorted oracle probabilities p_(1) >= ... >=
+    p_(k+1) are all more than 1e-4 apart. Where only a gap inside the list is
+    that small, the set must still match and the order may differ between
+    the near-equal neighbours; where p_(k) - p_(k+1) is that small (a near
+    tie), the set may differ. Both counts are reported. For excluded tokens the GPU's choice
     must still be valid (k distinct experts whose oracle probabilities are
     within the gap threshold of the oracle's k-th), and every other output is
     checked against the oracle evaluated at the GPU's choice.
@@ -16,6 +19,22 @@ Rules:
     logit error of a few 1e-5 at d = 4096 (a relative 1e-6 of sum |x_c w_c|).
   * Outputs: max-abs <= 2e-2 and relative Frobenius <= 1e-2 for bf16;
     both <= 1e-4 for fp32.
+  * Options. RMSNorm: the oracle normalises in fp64 and routes and evaluates
+    the experts on x_hat. Capacity: the kept rows, inv (-1 for a dropped
+    slot) and the dropped count are compared exactly with the oracle's
+    capacity dispatch of the GPU's indices. Shared experts: part of the
+    output comparison. On the bf16 path with the norm or shared experts the
+    output bars are split: relative Frobenius <= 1e-2 against the pure fp64
+    oracle, and max-abs <= 2e-2 against the fp64 oracle that rounds the two
+    stored bf16 operands (x_hat and H) as the kernels store them. The
+    max-abs bar is an absolute bound set for the plain layer at the
+    spec shapes; x_hat is one more bf16 rounding and each shared
+    expert one more full expert output of weight 1, which at the Mixtral
+    prefill shape takes the pure-oracle max-abs to about 4e-2 while the
+    relative error stays below 3e-3. z-loss: relative error <= 1e-4 (each token's
+    logsumexp carries the router's logit error of a few 1e-5 and an fp32
+    rounding; the per-block fp32 sums of at most 128 terms add at most
+    128 * 2^-24 relative).
 """
 from __future__ import annotations
 
@@ -27,16 +46,17 @@ import oracle
 GAP_THRESHOLD = 1e-4
 TOL = {"bf16": dict(max_abs=2e-2, rel_fro=1e-2), "f32": dict(max_abs=1e-4, rel_fro=1e-4)}
 GATE_TOL = {"bf16": 2e-5, "f32": 2e-6}
+Z_REL_TOL = 1e-4
 
 
 def _np(t):
     return t.detach().cpu().numpy()
 
 
-def check(inp, res, perm, k, renorm, dtype, tokens=None, h_round=False, report=None):
+def check(inp, res, perm, k, renorm, dtype, tokens=None, h_round=False, report=None, options=None):
     """inp: workloads.Inputs (CUDA tensors); res: MoEOutputs; perm: (offsets,
     perm_tok, inv) from get_permutation; tokens: sample of tokens whose output
-    rows are compared (None = all)."""
+    rows are compared (None = all); options: the MoEOptions of the call."""
     x = inp.x.cpu()
     wr = inp.w_router.cpu()
     b = None if inp.b_router is None else inp.b_router.cpu()
@@ -44,10 +64,21 @@ def check(inp, res, perm, k, renorm, dtype, tokens=None, h_round=False, report=N
     E = wr.shape[0]
     rep = {} if report is None else report
 
-    probs = oracle.router_probs(x, wr, b)
+    xin = x
+    if options is not None and options.norm_form:
+        nw = None if options.norm_weight is None else options.norm_weight.cpu()
+        xin = oracle.rmsnorm(x, nw, options.norm_eps, options.norm_form)
+    cf = 0.0 if options is None else options.capacity_factor
+    cap = oracle.capacity(cf, T, k, E)
+    shared = None
+    if options is not None and options.n_shared:
+        shared = (options.shared_gate.cpu(), options.shared_up.cpu(), options.shared_down.cpu())
+
+    logits = oracle.router_logits(xin, wr, b)
+    probs = oracle.softmax(logits)
     idx_o, gate_o, gap = oracle.topk(probs, k, renorm)
     counts_o, _, aux_o = oracle.stats(probs, idx_o)
-    offs_o, perm_o, inv_o, _ = oracle.dispatch(idx_o, E)
+    offs_o, perm_o, inv_o, _ = oracle.dispatch(idx_o, E, cap)
 
     idx_g = _np(res.topk_idx).astype(np.int32)
     gate_g = _np(res.topk_gate).astype(np.float64)
@@ -55,19 +86,33 @@ def check(inp, res, perm, k, renorm, dtype, tokens=None, h_round=False, report=N
     aux_g = float(_np(res.aux)[0])
     offs_g, perm_g, inv_g = (_np(a).astype(np.int64) for a in perm)
 
+    srt = -np.sort(-probs, axis=1)[:, :min(k + 1, E)]
+    order_gap = (srt[:, :-1] - srt[:, 1:]).min(axis=1) if srt.shape[1] > 1 else np.full(T, np.inf)
     near = gap <= GAP_THRESHOLD
+    near_order = ~near & (order_gap <= GAP_THRESHOLD)
     rep["near_tie_tokens"] = int(near.sum())
+    rep["near_order_tokens"] = int(near_order.sum())
     assert int(_np(res.status)[0]) == 0, f"device status word {int(_np(res.status)[0]):#x}"
 
     # --- routing ---------------------------------------------------------
-    ok = ~near
+    ok = ~near & ~near_order
+    for t in np.nonzero(near_order)[0]:
+        assert sorted(idx_g[t].tolist()) == sorted(idx_o[t].tolist()), f"token {t}: different set, gap {gap[t]}"
+        assert np.all(np.diff(probs[t, idx_g[t]]) <= GAP_THRESHOLD), f"token {t}: list out of order"
     mism = np.nonzero((idx_g[ok] != idx_o[ok]).any(axis=1))[0]
-    assert mism.size == 0, f"{mism.size} non-near-tie tokens routed differently, first {np.nonzero(ok)[0][mism[:5]]}"
+    if mism.size:
+        t0 = int(np.nonzero(ok)[0][mism[0]])
+        raise AssertionError(
+            f"{mism.size} non-near-tie tokens routed differently, first {np.nonzero(ok)[0][mism[:5]]}; token {t0}: "
+            f"gpu {idx_g[t0].tolist()} oracle {idx_o[t0].tolist()} p_gpu_choice {probs[t0, idx_g[t0]].tolist()} "
+            f"p_oracle_choice {probs[t0, idx_o[t0]].tolist()} gap {gap[t0]} order_gap {order_gap[t0]}")
     assert np.all((idx_g >= 0) & (idx_g < E))
     for t in np.nonzero(near)[0]:
         assert len(set(idx_g[t].tolist())) == k
         kth = np.sort(probs[t])[::-1][k - 1]
         assert np.all(probs[t, idx_g[t]] >= kth - GAP_THRESHOLD), f"token {t}: invalid near-tie choice"
+        # best first, up to near-equal neighbours
+        assert np.all(np.diff(probs[t, idx_g[t]]) <= GAP_THRESHOLD), f"token {t}: near-tie choice out of order"
     gate_ref = oracle.gates_for(probs, idx_g, renorm)
     gerr = float(np.abs(gate_g - gate_ref).max()) if T else 0.0
     rep["gate_max_abs"] = gerr
@@ -81,15 +126,26 @@ def check(inp, res, perm, k, renorm, dtype, tokens=None, h_round=False, report=N
     rep["aux"] = aux_g
     rep["aux_oracle"] = aux_o
     assert abs(aux_g - aux_ref) <= 1e-4, f"aux {aux_g} vs {aux_ref}"
-    offs_r, perm_r, inv_r, _ = oracle.dispatch(idx_g, E)
+    offs_r, perm_r, inv_r, drop_r = oracle.dispatch(idx_g, E, cap)
     np.testing.assert_array_equal(offs_g, offs_r)
-    np.testing.assert_array_equal(perm_g, perm_r)
+    np.testing.assert_array_equal(perm_g[:int(offs_r[E])], perm_r)
     np.testing.assert_array_equal(inv_g.reshape(T, k), inv_r)
-    # the oracle's own order, restricted to tokens that are not near ties
-    for e in range(E):
-        mine = perm_g[offs_g[e]:offs_g[e + 1]]
-        theirs = perm_o[offs_o[e]:offs_o[e + 1]]
-        np.testing.assert_array_equal(mine[~near[mine]], theirs[~near[theirs]])
+    if cap >= 0:
+        rep["dropped"] = drop_r
+        assert res.dropped is not None and int(_np(res.dropped)[0]) == drop_r, "dropped count"
+    # the oracle's own order, restricted to tokens that are not near ties (a
+    # near-tie flip can move which tokens a capacity drops: compare then only
+    # without near ties)
+    if cap < 0 or not near.any():
+        for e in range(E):
+            mine = perm_g[offs_g[e]:offs_g[e + 1]]
+            theirs = perm_o[offs_o[e]:offs_o[e + 1]]
+            np.testing.assert_array_equal(mine[~near[mine]], theirs[~near[theirs]])
+    if res.z_loss is not None:
+        z_g = float(_np(res.z_loss)[0])
+        z_o = oracle.z_loss(logits)
+        rep["z_loss"] = z_g
+        assert abs(z_g - z_o) <= Z_REL_TOL * abs(z_o) + 1e-7, f"z-loss {z_g} vs {z_o}"
 
     # --- outputs -------------------------------------------------------------
     if tokens is None:
@@ -97,8 +153,10 @@ def check(inp, res, perm, k, renorm, dtype, tokens=None, h_round=False, report=N
     tokens = np.asarray(tokens, dtype=np.int32)
     rep["tokens_compared"] = int(tokens.size)
     if tokens.size:
-        ref = oracle.moe_tokens(x, inp.w_gate.cpu(), inp.w_up.cpu(), inp.w_down.cpu(), tokens, idx_g[tokens],
-                                gate_ref[tokens], h_round=h_round)
+        keep = (inv_r[tokens] >= 0) if cap >= 0 else None
+        wts = (inp.w_gate.cpu(), inp.w_up.cpu(), inp.w_down.cpu())
+        ref = oracle.moe_tokens(xin, *wts, tokens, idx_g[tokens], gate_ref[tokens], h_round=h_round, keep=keep,
+                                shared=shared)
         got = _np(res.out)[tokens].astype(np.float64)
         diff = got - ref
         max_abs = float(np.abs(diff).max())
@@ -107,8 +165,19 @@ def check(inp, res, perm, k, renorm, dtype, tokens=None, h_round=False, report=N
         rep["rel_fro"] = rel_fro
         tol = TOL[dtype]
         assert np.isfinite(got).all()
-        assert max_abs <= tol["max_abs"], f"max-abs {max_abs} > {tol['max_abs']}"
-        assert rel_fro <= tol["rel_fro"], f"relative Frobenius {rel_fro} > {tol['rel_fro']}"
+        split_bars = dtype == "bf16" and options is not None and (options.norm_form or options.n_shared)
+        if dtype == "bf16" and not h_round:
+            norm_on = options is not None and options.norm_form
+            xr = oracle.round_bf16(xin) if norm_on else xin
+            ref_r = oracle.moe_tokens(xr, *wts, tokens, idx_g[tokens], gate_ref[tokens], h_round=True, keep=keep,
+                                      shared=shared)
+            max_abs_r = float(np.abs(got - ref_r).max())
+            rep["max_abs_vs_rounded_operands"] = max_abs_r
+        if split_bars:
+            assert max_abs_r <= tol["max_abs"], f"max-abs {max_abs_r} > {tol['max_abs']} ({rep})"
+        else:
+            assert max_abs <= tol["max_abs"], f"max-abs {max_abs} > {tol['max_abs']} ({rep})"
+        assert rel_fro <= tol["rel_fro"], f"relative Frobenius {rel_fro} > {tol['rel_fro']} ({rep})"
     return rep
 
 

@@ -54,6 +54,7 @@ MUTANTS = [
     ("capacity_off_by_one", "if (capacity >= 0 && taken >= capacity) {", "if (capacity >= 0 && taken > capacity) {"),
     ("dropped_slot_still_combined", "if (!keep || keep[i * k + j]) acc", "if (1) acc"),
     ("shared_not_added", "acc += ys[(i * n_shared + s) * d + c];", "acc += 0.0 * ys[(i * n_shared + s) * d + c];"),
+    ("bf16_round_toward_zero", "u += 0x7fffu + lsb;", "u += 0u * lsb;"),
     ("shared_half_weight", "acc += ys[(i * n_shared + s) * d + c];", "acc += 0.5 * ys[(i * n_shared + s) * d + c];"),
 ]
 
