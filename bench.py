@@ -3,7 +3,11 @@ TFLOP/s, with the dominant kernel's roofline fraction, the end-to-end number
 through the host API and the fp64 oracle timed on the host cores.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--norm {1,2}] [--shared S] [--capacity CF] [--zloss]
     python bench.py --impl reference ...   (the fp64 CPU oracle, timed alone)
+
+The options time the layer with the pre-MoE RMSNorm (with a weight), S shared
+experts, a capacity factor and the router z-loss.
 
 N > 1 runs under torchrun: every rank processes its own batch of tokens with
 the same (replicated) weights and no collective on the data path (weak
@@ -78,28 +82,40 @@ def load_traffic(workload, kernel):
 
 # ------------------------------------------------------------ algorithmic work
 
-def algorithmic(wl, counts):
+def algorithmic(wl, counts, opts=None):
     """Algorithmic FLOPs and DRAM bytes per launch of each kernel (the minimum
-    traffic: every input read once, every output written once)."""
+    traffic: every input read once, every output written once). Rows are the
+    kept assignments (all of them without a capacity) plus T per shared
+    expert."""
+    o = opts or {}
     T, d, E, k, I = wl.T, wl.d, wl.E, wl.k, wl.I
-    R = T * k
+    S = o.get("shared", 0)
+    counts = np.asarray(counts)
+    cap = o.get("cap", -1)
+    kept = int(np.minimum(counts, cap).sum()) if cap >= 0 else T * k
+    R = kept + S * T  # GEMM rows
     el = 2 if wl.dtype == "bf16" else 4
-    used = int((np.asarray(counts) > 0).sum())
+    used = int((counts > 0).sum()) + S  # weight sets streamed
     nb = (T + 127) // 128 if wl.dtype == "bf16" else (T + 31) // 32
+    norm_w = o.get("norm", 0) and wl.dtype == "bf16"
+    router = dict(flops=2.0 * T * d * E * (2 if norm_w else 1),
+                  bytes=T * d * el + E * d * el * (5 if norm_w else 1) + d * el * (1 if norm_w else 0)
+                  + T * k * 12 + nb * E * 8 + (T * 4 if o.get("norm", 0) else 0))
+    scan = dict(flops=0.0, bytes=nb * E * 12 + (E + 1) * 8 + E * 4)
+    xrows = kept + (T if S else 0)
+    gate_up = dict(flops=4.0 * R * d * I, bytes=2 * used * I * d * el + R * d * el + R * I * el)
+    if not fused_combine(wl, S):
+        return {
+            "router_topk": router, "route_scan": scan,
+            "permute": dict(flops=0.0, bytes=T * d * el + xrows * d * el + T * k * 12),
+            "grouped_gemm_gateup_swiglu": gate_up,
+            "grouped_gemm_down": dict(flops=2.0 * R * d * I, bytes=used * d * I * el + R * I * el + R * d * 4),
+            "combine": dict(flops=2.0 * R * d, bytes=R * d * 4 + T * d * 4 + T * k * 8),
+        }
     return {
-        "router_topk": dict(flops=2.0 * T * d * E, bytes=T * d * el + E * d * el + T * k * 12 + nb * E * 8),
-        "route_scan": dict(flops=0.0, bytes=nb * E * 12 + (E + 1) * 8 + E * 4),
-        "permute": dict(flops=0.0, bytes=T * d * el + R * d * el + R * 12),
-        "grouped_gemm_gateup_swiglu": dict(flops=4.0 * R * d * I,
-                                           bytes=2 * used * I * d * el + R * d * el + R * I * el),
-        "grouped_gemm_down": dict(flops=2.0 * R * d * I, bytes=used * d * I * el + R * I * el + R * d * 4),
-        "combine": dict(flops=2.0 * R * d, bytes=R * d * 4 + T * d * 4 + R * 8),
-    } if not fused_combine(wl) else {
-        "router_topk": dict(flops=2.0 * T * d * E, bytes=T * d * el + E * d * el + T * k * 12 + nb * E * 8),
-        "route_scan": dict(flops=0.0, bytes=nb * E * 12 + (E + 1) * 8 + E * 4),
-        "permute": dict(flops=0.0, bytes=T * d * el + R * d * el + R * 16 + T * d * 4),
-        "grouped_gemm_gateup_swiglu": dict(flops=4.0 * R * d * I,
-                                           bytes=2 * used * I * d * el + R * d * el + R * I * el),
+        "router_topk": router, "route_scan": scan,
+        "permute": dict(flops=0.0, bytes=T * d * el + xrows * d * el + T * k * 16 + T * d * 4),
+        "grouped_gemm_gateup_swiglu": gate_up,
         # down projection with the combine folded in: weights, H, and the fp32
         # output accumulated in place (read + write)
         "grouped_gemm_down": dict(flops=2.0 * R * d * I + 2.0 * R * d,
@@ -108,9 +124,10 @@ def algorithmic(wl, counts):
     }
 
 
-def fused_combine(wl):
-    """k = 2 on the bf16 path: the combine runs inside the down GEMM's epilogue."""
-    return wl.dtype == "bf16" and wl.k == 2
+def fused_combine(wl, n_shared=0):
+    """k = 2 on the bf16 path without shared experts: the combine runs inside
+    the down GEMM's epilogue."""
+    return wl.dtype == "bf16" and wl.k == 2 and n_shared == 0
 
 
 # --------------------------------------------------------------------- clocks
@@ -258,8 +275,8 @@ def run_reference(args, wl):
     return 0
 
 
-def config_of(wl, n_gpus):
-    return {"workload": wl.name, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "I": wl.I, "renorm": wl.renorm,
+def config_of(wl, n_gpus, opts=None):
+    return {"workload": wl.name, "options": opts or None, "T": wl.T, "d": wl.d, "E": wl.E, "k": wl.k, "I": wl.I, "renorm": wl.renorm,
             "router_bias": "zipf" if wl.zipf_bias else None, "global_batch_tokens": wl.T * n_gpus,
             "parallelism": f"dp{n_gpus} (replicated weights, independent token batches, no collective)",
             "l2": "inputs larger than L2: every step streams all expert weights "
@@ -277,6 +294,11 @@ def main():
     ap.add_argument("--workload", default="mixtral_prefill", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--norm", type=int, default=0, choices=[0, 1, 2],
+                    help="pre-MoE RMSNorm: 1 torch nn.RMSNorm form, 2 eps outside the root (with a weight)")
+    ap.add_argument("--shared", type=int, default=0, help="shared experts (each the routed experts' shape)")
+    ap.add_argument("--capacity", type=float, default=0.0, help="capacity factor (0: no dropping)")
+    ap.add_argument("--zloss", action="store_true", help="also compute the router z-loss statistic")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     wl = WORKLOADS[args.workload]
@@ -298,7 +320,23 @@ def main():
 
     inp = make_inputs(wl, dev, seed=0)  # same weights on every rank
     x = make_tokens(wl, wl.T, dev, seed=par.batch_seed(rank)) if world > 1 else inp.x
-    layer = MoELayer(inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k, wl.renorm, wl.T)
+    opts = {}
+    options = None
+    if args.norm or args.shared or args.capacity > 0 or args.zloss:
+        from sparse_mixture_experts_renorm_b200 import MoEOptions
+        from sparse_mixture_experts_renorm_b200.workloads import make_option_inputs
+
+        oi = make_option_inputs(wl, dev, seed=0, n_shared=args.shared, norm_weight=bool(args.norm))
+        options = MoEOptions(norm_form=args.norm, norm_eps=1e-5, norm_weight=oi.norm_weight,
+                             shared_gate=oi.shared_gate, shared_up=oi.shared_up, shared_down=oi.shared_down,
+                             capacity_factor=args.capacity, z_loss=args.zloss)
+        opts = {"norm": args.norm, "shared": args.shared, "capacity_factor": args.capacity, "z_loss": args.zloss}
+        if args.capacity > 0:
+            import math
+
+            opts["cap"] = min(wl.T, int(math.ceil(args.capacity * wl.T * wl.k / wl.E)))
+    layer = MoELayer(inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k, wl.renorm, wl.T,
+                     options=options)
     stream = torch.cuda.current_stream(dev)
     barrier = par.barrier
 
@@ -373,21 +411,25 @@ def main():
     if rank != 0:
         return 0
 
+    work = algorithmic(wl, counts, opts)
     tokens = par.job_tokens(wl.T, world, args.steps)
     tok_s = tokens / (ms / 1e3)
-    tflops = wl.active_flops * world * args.steps / (ms / 1e3) / 1e12
+    # active FLOPs: the three projections of every computed row plus the router
+    rows = work["grouped_gemm_gateup_swiglu"]["flops"] / (4.0 * wl.d * wl.I)
+    step_flops = 6.0 * wl.d * wl.I * rows + 2.0 * wl.d * wl.E * wl.T
+    tflops = step_flops * world * args.steps / (ms / 1e3) / 1e12
     peaks, peak_src = load_peaks()
     region_s = ms / 1e3
     sustained = region_s >= 1.0
     tc_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     hbm_peak = peaks["hbm_gbs"]
-    work = algorithmic(wl, counts)
     avg = per_kernel.mean(axis=0)
     kern = []
     for j, name in enumerate(KERNELS):
         w = work[name]
         t_s = avg[j] / 1e3
-        ent = {"name": name if not (name == "combine" and fused_combine(wl)) else "combine (in grouped_gemm_down)",
+        ent = {"name": name if not (name == "combine" and fused_combine(wl, args.shared))
+               else "combine (in grouped_gemm_down)",
                "avg_us": float(avg[j] * 1e3), "share": float(avg[j] / avg.sum()),
                "tflops": w["flops"] / t_s / 1e12 if t_s > 0 else None,
                "gbs": w["bytes"] / t_s / 1e9 if t_s > 0 else None}
@@ -406,7 +448,7 @@ def main():
         achieved = w["bytes"] / t_dom / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak}
     roof["kernel"] = dname
-    roof["traffic"] = load_traffic(wl.name, dname)
+    roof["traffic"] = load_traffic(wl.name, dname) if not opts else None
     roof["peak_source"] = (f"{peak_src} ({'sustained' if sustained and tensor_bound else 'burst'}"
                            f"{' bf16' if tensor_bound else ' HBM copy'})")
     roof["algorithmic_per_launch"] = w["flops"] if tensor_bound else w["bytes"]
@@ -416,18 +458,22 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded, random-init weights)",
         "tflops_active": tflops,
-        "config": config_of(wl, world),
+        "config": config_of(wl, world, opts),
         "roofline": roof,
         "kernels": kern,
         "e2e": {"value": par.job_tokens(wl.T, world, e2e_steps) / (ms_e2e / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x.numel() * x.element_size()),
                 "d2h_bytes_per_step": int(wl.T * wl.d * 4 + 4)},
-        "gpu_launches": (nk - (1 if fused_combine(wl) else 0)) * args.steps,
+        "gpu_launches": (nk - (1 if fused_combine(wl, args.shared) else 0)
+                         + (1 if args.norm and wl.dtype == "bf16" else 0)) * args.steps,
         "clocks": clocks,
         "counts": counts.tolist() if wl.E <= 16 else {"max": int(counts.max()), "min": int(counts.min()),
                                                       "mean": float(counts.mean())},
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if opts:
+        line["metric_extra"] = {"z_loss": float(layer.z_loss.item()) if args.zloss else None,
+                                "dropped": int(layer.dropped.item()) if args.capacity > 0 else None}
+    if world == 1 and not args.no_cpu_baseline and not opts:
         inp_cpu = inputs_to_cpu(inp)
         rate, n, dt, threads = cpu_oracle_rate(inp_cpu, wl, args.cpu_budget_s)
         line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",

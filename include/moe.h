@@ -153,6 +153,82 @@ moe_status moe_get_permutation(const void* workspace, size_t workspace_bytes, in
                                int32_t* inv, void* stream);
 
 /*
+ * Options of the layer that the pages name as configuration knobs. A zeroed
+ * struct (with struct_bytes set) is the plain layer of moe_forward.
+ *
+ * Pre-MoE RMSNorm (the block normalises x before this layer: Mixtral MoE
+ * Block, "post_attn_norm", nn.RMSNorm; Model Architecture Patterns,
+ * "RMSNorm (no bias, no mean centering)"):
+ *   MOE_NORM_RMS              x_hat = x / sqrt(mean_c x^2 + eps) * w
+ *   MOE_NORM_RMS_EPS_OUTSIDE  x_hat = w * x / (sqrt(mean_c x^2) + eps)
+ * The router and every expert then see x_hat instead of x. The router folds
+ * the per-token scale into its logits (exact x, w * W_r split into two bf16
+ * terms), and the experts read x_hat rounded once to the layer dtype.
+ *
+ * Shared experts ("moe_shared_experts: shared experts that process all
+ * tokens", KempnerForge ModelConfig): n_shared SwiGLU MLPs of the routed
+ * experts' shape, applied to every token and added with weight 1:
+ *   out[t] += sum_s W_sdown[s] (SiLU(W_sgate[s] x_t) * (W_sup[s] x_t))
+ *
+ * Capacity ("moe_capacity_factor: 0 = no drop, > 0 = cap tokens per
+ * expert"): every expert keeps at most C = ceil(cf * T * k / E) assignments,
+ * its first C in dispatch order (tokens ascending); a dropped slot adds
+ * nothing to out. topk_idx, topk_gate, counts and aux are those before
+ * dropping; moe_get_permutation reports the kept rows and inv = -1 for a
+ * dropped slot.
+ *
+ * Router z-loss (the ST-MoE statistic of "moe_router_z_loss_weight"):
+ *   z = (1/T) sum_t ( log sum_e exp(logit[t,e]) )^2, logits with their bias.
+ */
+typedef enum {
+  MOE_NORM_NONE = 0,
+  MOE_NORM_RMS = 1,
+  MOE_NORM_RMS_EPS_OUTSIDE = 2
+} moe_norm_form;
+
+#define MOE_MAX_SHARED 8
+
+typedef struct moe_options {
+  size_t struct_bytes;       /* sizeof(moe_options) */
+  int norm_form;             /* moe_norm_form */
+  float norm_eps;            /* >= 0 and finite */
+  const void* norm_weight;   /* device, [d] in the layer dtype, or NULL for ones */
+  int n_shared;              /* 0 .. MOE_MAX_SHARED */
+  const void* shared_gate;   /* device, [n_shared, I, d], dtype */
+  const void* shared_up;     /* device, [n_shared, I, d], dtype */
+  const void* shared_down;   /* device, [n_shared, d, I], dtype */
+  double capacity_factor;    /* 0: no dropping; > 0 and finite: the cap above */
+  int32_t* dropped;          /* device, [1] int32, or NULL: assignments dropped */
+  float* z_loss;             /* device, [1] fp32, or NULL: the z-loss statistic */
+} moe_options;
+
+/*
+ * moe_workspace_size_ex — moe_workspace_size for a layer with options (opt
+ * may be NULL: the plain layer). Shared experts add T rows to the dispatched
+ * input and n_shared * T rows to the hidden and output scratch. Returns 0 for
+ * an invalid shape or invalid options.
+ */
+size_t moe_workspace_size_ex(int T, int d, int E, int k, int I, moe_dtype dtype, const moe_options* opt);
+
+/*
+ * moe_forward_ex — moe_forward with options (opt may be NULL) and optional
+ * per-kernel timing events (events may be NULL with n_events = 0; otherwise
+ * as moe_forward_events). The workspace must hold moe_workspace_size_ex()
+ * bytes for the same options. Invalid options (unknown norm form, negative
+ * or non-finite eps or capacity factor, n_shared outside 0..MOE_MAX_SHARED,
+ * a NULL or misaligned shared weight, struct_bytes smaller than the struct)
+ * give MOE_ERR_INVALID_ARG before anything is launched. With the norm and
+ * a weight on the bf16 path, an extra small kernel that splits w * W_r runs
+ * before the router and is timed with it.
+ */
+moe_status moe_forward_ex(const void* x, const void* w_router, const float* b_router,
+                          const void* w_gate, const void* w_up, const void* w_down,
+                          int T, int d, int E, int k, int I, int renorm, moe_dtype dtype,
+                          const moe_options* opt, float* out, int32_t* topk_idx, float* topk_gate,
+                          int32_t* counts, float* aux, void* workspace, size_t workspace_bytes,
+                          int32_t* status_dev, void* stream, void* const* events, int n_events);
+
+/*
  * moe_forward_noalloc — moe_forward for callers that cannot allocate device
  * memory: the same layer, arguments and results, but the scratch lives in a
  * static array of MOE_NOALLOC_SCRATCH_BYTES inside the library's device image
@@ -188,7 +264,7 @@ moe_status moe_forward_noalloc(const void* x, const void* w_router, const float*
  * kernel of the library shares: it launches one warp on `stream` that waits
  * on a shared-memory barrier phase nothing will complete, through the same
  * bounded wait the kernels use, with a limit of limit_ns nanoseconds
- * (1e6 .. 1e9*5). The wait gives up, OR-s MOE_DEV_TIMEOUT into *status_dev
+ * (1e6 .. 5e9). The wait gives up, OR-s MOE_DEV_TIMEOUT into *status_dev
  * (device int32, not cleared here) and the kernel returns; the context stays
  * usable. The pages have no counterpart (their Rust layer panics instead).
  */

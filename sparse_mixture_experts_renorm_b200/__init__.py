@@ -17,8 +17,8 @@ import torch
 from . import _binding as B
 from ._binding import MoEError, load_library
 
-__all__ = ["MoEError", "MoEOutputs", "MoELayer", "HostPipeline", "moe_forward", "workspace_size", "get_permutation",
-           "load_library"]
+__all__ = ["MoEError", "MoEOptions", "MoEOutputs", "MoELayer", "HostPipeline", "moe_forward", "workspace_size",
+           "get_permutation", "load_library"]
 
 
 def _dtype_code(t: torch.dtype) -> int:
@@ -33,12 +33,72 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def workspace_size(T: int, d: int, E: int, k: int, I: int, dtype: torch.dtype) -> int:
+@dataclass
+class MoEOptions:
+    """Options of the layer (``moe_options`` in include/moe.h).
+
+    norm_form: 0 none, 1 torch's nn.RMSNorm x/sqrt(mean x^2 + eps)*w, 2 the
+    form w*x/(sqrt(mean x^2) + eps); norm_weight: [d] in the layer dtype or
+    None for ones. shared_*: weights of the shared experts ([S, I, d],
+    [S, I, d], [S, d, I]) or None. capacity_factor: 0 = no dropping.
+    z_loss: also compute the router z-loss statistic."""
+    norm_form: int = 0
+    norm_eps: float = 1e-5
+    norm_weight: torch.Tensor | None = None
+    shared_gate: torch.Tensor | None = None
+    shared_up: torch.Tensor | None = None
+    shared_down: torch.Tensor | None = None
+    capacity_factor: float = 0.0
+    z_loss: bool = False
+
+    @property
+    def n_shared(self) -> int:
+        return 0 if self.shared_gate is None else int(self.shared_gate.shape[0])
+
+    def to_c(self, dropped=None, z_loss=None) -> B.moe_options:
+        o = B.moe_options()
+        o.struct_bytes = ctypes.sizeof(B.moe_options)
+        o.norm_form = int(self.norm_form)
+        o.norm_eps = float(self.norm_eps)
+        o.norm_weight = None if self.norm_weight is None else self.norm_weight.data_ptr()
+        o.n_shared = self.n_shared
+        if self.n_shared:
+            o.shared_gate = self.shared_gate.data_ptr()
+            o.shared_up = self.shared_up.data_ptr()
+            o.shared_down = self.shared_down.data_ptr()
+        o.capacity_factor = float(self.capacity_factor)
+        o.dropped = None if dropped is None else dropped.data_ptr()
+        o.z_loss = None if z_loss is None else z_loss.data_ptr()
+        return o
+
+
+def workspace_size(T: int, d: int, E: int, k: int, I: int, dtype: torch.dtype,
+                   options: MoEOptions | None = None) -> int:
     lib = load_library()
-    n = lib.moe_workspace_size(T, d, E, k, I, _dtype_code(dtype))
+    if options is None:
+        n = lib.moe_workspace_size(T, d, E, k, I, _dtype_code(dtype))
+    else:
+        opt = options.to_c()
+        n = lib.moe_workspace_size_ex(T, d, E, k, I, _dtype_code(dtype), ctypes.byref(opt))
     if n == 0:
         raise MoEError(B.MOE_ERR_INVALID_ARG, B.last_error_detail(lib))
     return int(n)
+
+
+def _check_options(options: MoEOptions, x, E: int, I: int):
+    d = x.shape[1]
+    if options.norm_weight is not None:
+        w = options.norm_weight
+        if w.dtype != x.dtype or w.numel() != d or w.device != x.device or not w.is_contiguous():
+            raise ValueError(f"norm_weight must be a contiguous {x.dtype} CUDA tensor of {d} elements")
+    if options.n_shared:
+        S = options.n_shared
+        for name, t, shape in (("shared_gate", options.shared_gate, (S, I, d)),
+                               ("shared_up", options.shared_up, (S, I, d)),
+                               ("shared_down", options.shared_down, (S, d, I))):
+            if t is None or tuple(t.shape) != shape or t.dtype != x.dtype or t.device != x.device \
+                    or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous {x.dtype} CUDA tensor of shape {shape}")
 
 
 @dataclass
@@ -50,17 +110,20 @@ class MoEOutputs:
     aux: torch.Tensor  # [1] fp32
     status: torch.Tensor  # [1] int32, MOE_DEV_* bits
     workspace: torch.Tensor  # uint8, holds the dispatch order of this call
+    z_loss: torch.Tensor | None = None  # [1] fp32 when options.z_loss
+    dropped: torch.Tensor | None = None  # [1] int32 when options.capacity_factor > 0
 
 
 def moe_forward(x, w_router, b_router, w_gate, w_up, w_down, k: int, renorm: bool, *, out=None, topk_idx=None,
                 topk_gate=None, counts=None, aux=None, workspace=None, status=None, stream=None,
-                events=None) -> MoEOutputs:
+                events=None, options: MoEOptions | None = None, z_loss=None, dropped=None) -> MoEOutputs:
     """Run the layer on ``x`` ([T, d], CUDA) with stacked expert weights
     ``w_gate``/``w_up`` [E, I, d] and ``w_down`` [E, d, I]. Buffers that are
     not given are allocated with torch; the call is asynchronous on
     ``stream`` (default: torch's current stream). ``events``: optional list
     of MOE_NUM_KERNELS + 1 timing-enabled ``torch.cuda.Event`` recorded
-    around each kernel (see ``moe_forward_events`` in include/moe.h)."""
+    around each kernel (see ``moe_forward_events`` in include/moe.h).
+    ``options``: RMSNorm, shared experts, capacity, z-loss (``MoEOptions``)."""
     lib = load_library()
     T, d = x.shape
     E = w_router.shape[0]
@@ -89,26 +152,37 @@ def moe_forward(x, w_router, b_router, w_gate, w_up, w_down, k: int, renorm: boo
         aux = torch.empty((1,), dtype=torch.float32, device=dev)
     if status is None:
         status = torch.zeros((1,), dtype=torch.int32, device=dev)
+    if options is not None:
+        _check_options(options, x, E, I)
+        if options.z_loss and z_loss is None:
+            z_loss = torch.empty((1,), dtype=torch.float32, device=dev)
+        if options.capacity_factor > 0 and dropped is None:
+            dropped = torch.empty((1,), dtype=torch.int32, device=dev)
     if workspace is None:
-        n = lib.moe_workspace_size(T, d, E, k, I, dt)
-        if n == 0:
-            raise MoEError(B.MOE_ERR_INVALID_ARG, B.last_error_detail(lib))
-        workspace = torch.empty((n,), dtype=torch.uint8, device=dev)
+        workspace = torch.empty((workspace_size(T, d, E, k, I, x.dtype, options),), dtype=torch.uint8, device=dev)
     if stream is None:
         stream = torch.cuda.current_stream(dev).cuda_stream
-    args = (_ptr(x), _ptr(w_router), _ptr(b_router), _ptr(w_gate), _ptr(w_up), _ptr(w_down), T, d, E, k, I,
-            int(bool(renorm)), dt, _ptr(out), _ptr(topk_idx), _ptr(topk_gate), _ptr(counts), _ptr(aux),
-            _ptr(workspace), workspace.numel(), _ptr(status), ctypes.c_void_p(stream))
-    if events is None:
-        st = lib.moe_forward(*args)
-    else:
+    head = (_ptr(x), _ptr(w_router), _ptr(b_router), _ptr(w_gate), _ptr(w_up), _ptr(w_down), T, d, E, k, I,
+            int(bool(renorm)), dt)
+    tail = (_ptr(out), _ptr(topk_idx), _ptr(topk_gate), _ptr(counts), _ptr(aux), _ptr(workspace), workspace.numel(),
+            _ptr(status), ctypes.c_void_p(stream))
+    arr, n_ev = None, 0
+    if events is not None:
         for ev in events:
             if not ev.cuda_event:  # torch creates the event on its first record
                 ev.record(torch.cuda.current_stream(dev))
         arr = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
-        st = lib.moe_forward_events(*args, arr, len(events))
+        n_ev = len(events)
+    if options is not None:
+        opt = options.to_c(dropped=dropped, z_loss=z_loss if options.z_loss else None)
+        st = lib.moe_forward_ex(*head, ctypes.byref(opt), *tail, arr, n_ev)
+    elif events is None:
+        st = lib.moe_forward(*head, *tail)
+    else:
+        st = lib.moe_forward_events(*head, *tail, arr, n_ev)
     B.check(st, lib)
-    return MoEOutputs(out, topk_idx, topk_gate, counts, aux, status, workspace)
+    return MoEOutputs(out, topk_idx, topk_gate, counts, aux, status, workspace,
+                      z_loss if options is not None and options.z_loss else None, dropped)
 
 
 def get_permutation(res: MoEOutputs, T: int, d: int, E: int, k: int, I: int, dtype: torch.dtype, stream=None):
@@ -130,7 +204,9 @@ class MoELayer:
     """The layer with resident weights and preallocated outputs/workspace for a
     fixed number of tokens, for repeated calls (serving, benchmarking)."""
 
-    def __init__(self, w_router, b_router, w_gate, w_up, w_down, k: int, renorm: bool, max_tokens: int):
+    def __init__(self, w_router, b_router, w_gate, w_up, w_down, k: int, renorm: bool, max_tokens: int,
+                 options: MoEOptions | None = None):
+        self.options = options
         self.w_router, self.b_router = w_router, b_router
         self.w_gate, self.w_up, self.w_down = w_gate, w_up, w_down
         self.k, self.renorm = k, renorm
@@ -144,7 +220,9 @@ class MoELayer:
         self.counts = torch.empty((self.E,), dtype=torch.int32, device=dev)
         self.aux = torch.empty((1,), dtype=torch.float32, device=dev)
         self.status = torch.zeros((1,), dtype=torch.int32, device=dev)
-        self.workspace = torch.empty((workspace_size(max_tokens, self.d, self.E, k, self.I, self.dtype),),
+        self.z_loss = torch.empty((1,), dtype=torch.float32, device=dev)
+        self.dropped = torch.empty((1,), dtype=torch.int32, device=dev)
+        self.workspace = torch.empty((workspace_size(max_tokens, self.d, self.E, k, self.I, self.dtype, options),),
                                      dtype=torch.uint8, device=dev)
 
     def __call__(self, x, stream=None, events=None) -> MoEOutputs:
@@ -153,7 +231,8 @@ class MoELayer:
             raise ValueError(f"this layer was sized for {self.T} tokens")
         return moe_forward(x, self.w_router, self.b_router, self.w_gate, self.w_up, self.w_down, self.k, self.renorm,
                            out=self.out, topk_idx=self.topk_idx, topk_gate=self.topk_gate, counts=self.counts,
-                           aux=self.aux, workspace=self.workspace, status=self.status, stream=stream, events=events)
+                           aux=self.aux, workspace=self.workspace, status=self.status, stream=stream, events=events,
+                           options=self.options, z_loss=self.z_loss, dropped=self.dropped)
 
     def forward_host(self, x_host, out_host, aux_host, x_dev):
         """End-to-end call from host memory: copy ``x_host`` (pinned, [T, d])
@@ -202,7 +281,7 @@ class HostPipeline:
         moe_forward(self.x_dev[b], L.w_router, L.b_router, L.w_gate, L.w_up, L.w_down, L.k, L.renorm,
                     out=self.out_dev[b], topk_idx=L.topk_idx, topk_gate=L.topk_gate, counts=L.counts,
                     aux=self.aux_dev[b], workspace=L.workspace, status=L.status,
-                    stream=self.compute.cuda_stream)
+                    stream=self.compute.cuda_stream, options=L.options, z_loss=L.z_loss, dropped=L.dropped)
         self.computed[b].record(self.compute)
         self.d2h.wait_event(self.computed[b])
         with torch.cuda.stream(self.d2h):

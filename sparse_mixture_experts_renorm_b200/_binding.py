@@ -26,9 +26,30 @@ STATUS_NAMES = {
 }
 
 EXPORTED = ("moe_workspace_size", "moe_forward", "moe_forward_events", "moe_kernel_name", "moe_get_permutation",
-            "moe_last_error_detail", "moe_forward_noalloc", "moe_selftest_wait_timeout")
+            "moe_last_error_detail", "moe_forward_noalloc", "moe_selftest_wait_timeout", "moe_workspace_size_ex",
+            "moe_forward_ex")
+MOE_NORM_NONE, MOE_NORM_RMS, MOE_NORM_RMS_EPS_OUTSIDE = 0, 1, 2
+MOE_MAX_SHARED = 8
 MOE_NOALLOC_SCRATCH_BYTES = 16 << 20
 MOE_NUM_KERNELS = 6
+
+
+class moe_options(ctypes.Structure):
+    """The C struct ``moe_options`` of include/moe.h (same field order and types)."""
+
+    _fields_ = [
+        ("struct_bytes", ctypes.c_size_t),
+        ("norm_form", ctypes.c_int),
+        ("norm_eps", ctypes.c_float),
+        ("norm_weight", ctypes.c_void_p),
+        ("n_shared", ctypes.c_int),
+        ("shared_gate", ctypes.c_void_p),
+        ("shared_up", ctypes.c_void_p),
+        ("shared_down", ctypes.c_void_p),
+        ("capacity_factor", ctypes.c_double),
+        ("dropped", ctypes.c_void_p),
+        ("z_loss", ctypes.c_void_p),
+    ]
 
 
 class MoEError(RuntimeError):
@@ -60,6 +81,12 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.moe_forward.restype = I32
     lib.moe_forward_events.argtypes = lib.moe_forward.argtypes + [ctypes.POINTER(ctypes.c_void_p), I32]
     lib.moe_forward_events.restype = I32
+    OPT = ctypes.POINTER(moe_options)
+    lib.moe_workspace_size_ex.argtypes = [I32, I32, I32, I32, I32, I32, OPT]
+    lib.moe_workspace_size_ex.restype = SZ
+    lib.moe_forward_ex.argtypes = ([P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, OPT, P, P, P, P, P, P, SZ, P,
+                                    P, ctypes.POINTER(ctypes.c_void_p), I32])
+    lib.moe_forward_ex.restype = I32
     lib.moe_kernel_name.argtypes = [I32]
     lib.moe_kernel_name.restype = ctypes.c_char_p
     lib.moe_forward_noalloc.argtypes = [P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, P, P, P, P, P, P, P]

@@ -24,7 +24,10 @@
 //
 // Persistent: clusters walk a device-side tile list built from the routing
 // counts (experts in order; n-tile outer, m-tile inner inside an expert, so
-// clusters running together share weight tiles in L2). Every wait is bounded.
+// clusters running together share weight tiles in L2). Shared experts
+// ("moe_shared_experts", KempnerForge ModelConfig) are extra groups after the
+// routed experts, each over all T tokens, with their own weight tensor maps.
+// Every wait is bounded.
 #include "common.cuh"
 
 namespace moe {
@@ -133,8 +136,34 @@ __device__ __forceinline__ void ld_chunk_sum(uint32_t taddr, int nacc, int strid
 }
 
 struct TileCoord {
-  int e, m, n;
+  int e, m, n;  // group (routed expert, then shared experts), token tile, weight block
 };
+
+// Rows of group g: routed experts read and write their dispatched rows;
+// shared expert s reads sh.rows rows at sh.in0 + s * sh.in_step and writes
+// them at sh.out0 + s * sh.rows.
+struct GroupRows {
+  int in0, out0, cnt, widx;
+  bool shared;
+};
+
+__device__ __forceinline__ GroupRows group_rows(int g, const int* s_off, int E, const SharedGroups& sh) {
+  GroupRows r;
+  if (g < E) {
+    r.in0 = r.out0 = s_off[g];
+    r.cnt = s_off[g + 1] - s_off[g];
+    r.widx = g;
+    r.shared = false;
+  } else {
+    const int s = g - E;
+    r.in0 = sh.in0 + s * sh.in_step;
+    r.out0 = sh.out0 + s * sh.rows;
+    r.cnt = sh.rows;
+    r.widx = s;
+    r.shared = true;
+  }
+  return r;
+}
 
 __device__ __forceinline__ TileCoord decode_tile(int tile, int n_tiles, const int* s_mt, int E) {
   const int q = tile / n_tiles;
@@ -160,9 +189,11 @@ __device__ __forceinline__ float silu_f32(float z) { return __fdividef(z, 1.0f +
 template <int kMode>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                            const __grid_constant__ CUtensorMap tmS0, const __grid_constant__ CUtensorMap tmS1,
                             const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBs,
                             const int32_t* __restrict__ offsets, const int32_t* __restrict__ mtile256, int E,
-                            int N, int K, void* __restrict__ out, const int32_t* __restrict__ perm_tok,
+                            const SharedGroups sh, int N, int K, void* __restrict__ out,
+                            const int32_t* __restrict__ perm_tok,
                             const float* __restrict__ rgate, float* __restrict__ comb_out, int32_t* status,
                             uint64_t limit_ns) {
   extern __shared__ uint8_t smem_raw[];
@@ -181,7 +212,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_off = reinterpret_cast<int*>(s_tmem + 4);  // [E+1]
-  int* s_mt = s_off + (E + 1);                       // [E+1]
+  int* s_mt = s_off + (E + 1);                       // [G+1]
+  const int G = E + sh.n;                            // GEMM groups: routed, then shared experts
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -210,14 +242,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     if (kMode == 0) tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmBs);
+    if (sh.n > 0) {
+      tma_prefetch_desc(&tmS0);
+      if (kMode == 0) tma_prefetch_desc(&tmS1);
+    }
   }
   if (warp == 1) {
     tmem_alloc_pair(s_tmem, 2 * kBN);
     tmem_relinquish_pair();
   }
   pdl_wait();  // the routing tables and the A/B operands come from the kernels before
-  for (int i = threadIdx.x; i <= E; i += blockDim.x) {
-    s_off[i] = offsets[i];
+  for (int i = threadIdx.x; i <= G; i += blockDim.x) {
+    if (i <= E) s_off[i] = offsets[i];
     s_mt[i] = mtile256[i];
   }
   tc_fence_before();
@@ -225,7 +261,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   cluster_sync();  // the peer's barriers are initialised before any remote signal
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
-  const int total = s_mt[E] * n_wb;
+  const int total = s_mt[G] * n_wb;
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -235,12 +271,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int issued = 0;
       bool ok = true;
       for (int tile = cid; ok && tile < total; tile += ncl) {
-        const TileCoord tc = decode_tile(tile, n_wb, s_mt, E);
-        const int ntok = min(256, s_off[tc.e + 1] - s_off[tc.e] - tc.m * 256);
+        const TileCoord tc = decode_tile(tile, n_wb, s_mt, G);
+        const GroupRows gr = group_rows(tc.e, s_off, E, sh);
+        const int ntok = min(256, gr.cnt - tc.m * 256);
         const int half = ((ntok + 15) & ~15) >> 1;  // token rows of B held by each CTA
         const bool small = half <= kSmallRows;
-        const int brow = s_off[tc.e] + tc.m * 256 + (int)rank * half;
-        const int arow = kMode == 0 ? tc.e * N + tc.n * 128 + (int)rank * 64 : tc.e * N + tc.n * 256 + (int)rank * 128;
+        const int brow = gr.in0 + tc.m * 256 + (int)rank * half;
+        const int arow =
+            kMode == 0 ? gr.widx * N + tc.n * 128 + (int)rank * 64 : gr.widx * N + tc.n * 256 + (int)rank * 128;
+        const CUtensorMap* mA0 = gr.shared ? &tmS0 : &tmA0;
+        const CUtensorMap* mA1 = gr.shared ? &tmS1 : &tmA1;
         const uint32_t bytes = 2u * (uint32_t)(kHalfBytes + (small ? kSmallRows * 128 : kHalfBytes));
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, s_abort, status, limit_ns)) {
@@ -251,10 +291,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if (leader) mbar_arrive_expect_tx(&full[stage], bytes);
           if (kMode == 0) {
             // rows 0-63: gate rows of this CTA's 64 hidden units, 64-127: up rows
-            tma_load_2d_pair(sA + stage * kHalfBytes, &tmA0, fbar, kb * kBK, arow);
-            tma_load_2d_pair(sA + stage * kHalfBytes + kHalfBytes / 2, &tmA1, fbar, kb * kBK, arow);
+            tma_load_2d_pair(sA + stage * kHalfBytes, mA0, fbar, kb * kBK, arow);
+            tma_load_2d_pair(sA + stage * kHalfBytes + kHalfBytes / 2, mA1, fbar, kb * kBK, arow);
           } else {
-            tma_load_2d_pair(sA + stage * kHalfBytes, &tmA0, fbar, kb * kBK, arow);
+            tma_load_2d_pair(sA + stage * kHalfBytes, mA0, fbar, kb * kBK, arow);
           }
           tma_load_2d_pair(sB + stage * kHalfBytes, small ? &tmBs : &tmB, fbar, kb * kBK, brow);
           ++issued;
@@ -288,8 +328,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = cid; ok && tile < total; tile += ncl) {
-        const TileCoord tc = decode_tile(tile, n_wb, s_mt, E);
-        const int ntok = min(256, s_off[tc.e + 1] - s_off[tc.e] - tc.m * 256);
+        const TileCoord tc = decode_tile(tile, n_wb, s_mt, G);
+        const int ntok = min(256, group_rows(tc.e, s_off, E, sh).cnt - tc.m * 256);
         const int nt16 = (ntok + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(256, nt16);
         // narrow tiles spread their K loop over independent accumulators
@@ -338,9 +378,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = cid; tile < total; tile += ncl) {
-      const TileCoord tc = decode_tile(tile, n_wb, s_mt, E);
-      const int ntok = min(256, s_off[tc.e + 1] - s_off[tc.e] - tc.m * 256);
-      const size_t row0 = static_cast<size_t>(s_off[tc.e]) + static_cast<size_t>(tc.m * 256);
+      const TileCoord tc = decode_tile(tile, n_wb, s_mt, G);
+      const GroupRows gr = group_rows(tc.e, s_off, E, sh);
+      const int ntok = min(256, gr.cnt - tc.m * 256);
+      const size_t row0 = static_cast<size_t>(gr.out0) + static_cast<size_t>(tc.m * 256);
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, s_abort, status, limit_ns))) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * kBN);
@@ -403,7 +444,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
               const int tok = c * 32 + t;
               if (tok < ntok) {
                 const float4 val = *reinterpret_cast<const float4*>(tw + t * 36 + vc);
-                if (comb_out) {
+                if (comb_out && !gr.shared) {
                   // combine folded in: out[token] += gate * y (two adds per
                   // element into a zeroed row, so the order cannot matter)
                   const size_t r = row0 + tok;
@@ -463,38 +504,42 @@ int max_active_pairs(const void* kern, int smem) {
 }
 
 template <int kMode>
-cudaError_t launch_tc2(const CUtensorMap& tmA0, const CUtensorMap& tmA1, const CUtensorMap& tmB,
-                       const CUtensorMap& tmBs, const int32_t* offsets, const int32_t* mtile256, int R, int E, int N,
-                       int K, void* out, const int32_t* perm_tok, const float* rgate, float* comb_out,
-                       int32_t* status, cudaStream_t stream) {
+cudaError_t launch_tc2(const CUtensorMap& tmA0, const CUtensorMap& tmA1, const CUtensorMap& tmS0,
+                       const CUtensorMap& tmS1, const CUtensorMap& tmB, const CUtensorMap& tmBs, const int32_t* offsets,
+                       const int32_t* mtile256, int R_rows, int E, const SharedGroups& sh, int N, int K, void* out,
+                       const int32_t* perm_tok, const float* rgate, float* comb_out, int32_t* status,
+                       cudaStream_t stream) {
   auto kern = grouped_gemm_tc2_kernel<kMode>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemm2SmemBytes);
   if (err != cudaSuccess) return err;
   const int pairs = max_active_pairs(reinterpret_cast<const void*>(kern), kGemm2SmemBytes);
   if (pairs <= 0) return cudaErrorInvalidConfiguration;
   const int n_wb = kMode == 0 ? (N + 127) / 128 : (N + 255) / 256;
-  const long long max_tiles = (long long)(R / 256 + E) * n_wb;
+  const long long max_tiles = (long long)(R_rows / 256 + E + sh.n) * n_wb;
   const int clusters = (int)(max_tiles < pairs ? max_tiles : pairs);
   if (clusters <= 0) return cudaSuccess;
-  return launch_pdl(kern, dim3(2 * clusters), dim3(kGemmThreads), kGemm2SmemBytes, stream, tmA0, tmA1, tmB, tmBs,
-                    offsets, mtile256, E, N, K, out, perm_tok, rgate, comb_out, status, kWaitLimitNs);
+  return launch_pdl(kern, dim3(2 * clusters), dim3(kGemmThreads), kGemm2SmemBytes, stream, tmA0, tmA1, tmS0, tmS1,
+                    tmB, tmBs, offsets, mtile256, E, sh, N, K, out, perm_tok, rgate, comb_out, status, kWaitLimitNs);
 }
 
 }  // namespace
 
-cudaError_t launch_gemm_gateup_tc2(const CUtensorMap& tm_wg, const CUtensorMap& tm_wu, const CUtensorMap& tm_xp,
-                                   const CUtensorMap& tm_xp_small, const int32_t* offsets, const int32_t* mtile256,
-                                   int R, int E, int I, int d, void* h, int32_t* status, cudaStream_t stream) {
-  return launch_tc2<0>(tm_wg, tm_wu, tm_xp, tm_xp_small, offsets, mtile256, R, E, I, d, h, nullptr, nullptr, nullptr,
-                       status, stream);
+cudaError_t launch_gemm_gateup_tc2(const CUtensorMap& tm_wg, const CUtensorMap& tm_wu, const CUtensorMap& tm_sg,
+                                   const CUtensorMap& tm_su, const CUtensorMap& tm_xp, const CUtensorMap& tm_xp_small,
+                                   const int32_t* offsets, const int32_t* mtile, int R_rows, int E,
+                                   const SharedGroups& sh, int I, int d, void* h, int32_t* status,
+                                   cudaStream_t stream) {
+  return launch_tc2<0>(tm_wg, tm_wu, tm_sg, tm_su, tm_xp, tm_xp_small, offsets, mtile, R_rows, E, sh, I, d, h, nullptr,
+                       nullptr, nullptr, status, stream);
 }
 
-cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_wd, const CUtensorMap& tm_h, const CUtensorMap& tm_h_small,
-                                 const int32_t* offsets, const int32_t* mtile256, int R, int E, int I, int d, float* y,
+cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_wd, const CUtensorMap& tm_sd, const CUtensorMap& tm_h,
+                                 const CUtensorMap& tm_h_small, const int32_t* offsets, const int32_t* mtile,
+                                 int R_rows, int E, const SharedGroups& sh, int I, int d, float* y,
                                  const int32_t* perm_tok, const float* rgate, float* comb_out, int32_t* status,
                                  cudaStream_t stream) {
-  return launch_tc2<1>(tm_wd, tm_wd, tm_h, tm_h_small, offsets, mtile256, R, E, d, I, y, perm_tok, rgate, comb_out,
-                       status, stream);
+  return launch_tc2<1>(tm_wd, tm_wd, tm_sd, tm_sd, tm_h, tm_h_small, offsets, mtile, R_rows, E, sh, d, I, y, perm_tok,
+                       rgate, comb_out, status, stream);
 }
 
 }  // namespace moe

@@ -23,16 +23,10 @@ constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 8;
 
 // tcgen05 grouped GEMM tiling.
-constexpr int kTileM = 256;       // rows (dispatched tokens) per tile of the CTA pair
-constexpr int kBM = 128;          // rows per CTA
-constexpr int kBN = 256;          // UMMA N: 128 gate + 128 up columns, or 256 down columns
+constexpr int kTileM = 256;       // dispatched tokens per tile of the CTA pair (UMMA N)
+constexpr int kBN = 256;          // weight rows per tile of the CTA pair (UMMA M)
 constexpr int kBK = 64;           // K per pipeline stage (one 128-byte swizzle row of bf16)
-constexpr int kStages = 4;        // shared-memory pipeline depth
 constexpr int kGemmThreads = 192; // warp 0 TMA, warp 1 MMA + TMEM owner, warps 2-5 epilogue
-constexpr int kTileABytes = kBM * kBK * 2;
-constexpr int kTileBBytes = kBN * kBK * 2;
-constexpr int kStageBytes = kTileABytes + kTileBBytes;
-constexpr int kGemmSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 4096 /*barriers, tables*/;
 
 // fp32 SIMT grouped GEMM tiling.
 constexpr int kSimtBM = 64;
@@ -41,26 +35,57 @@ constexpr int kSimtBN = 64;
 // Bounded waits give up after this long (a healthy wait takes microseconds).
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
-// Byte offsets of every scratch array inside the caller's workspace.
+// Byte offsets of every scratch array inside the caller's workspace. The
+// arrays up to and including `inv` sit at offsets that depend on the shape
+// only (not on the options), so moe_get_permutation can find them.
 struct Workspace {
   size_t status;      // int32 [1]     device status word used when the caller passes none
-  size_t offsets;     // int32 [E+1]   first dispatched row of each expert
+  size_t offsets;     // int32 [E+1]   first dispatched (kept) row of each expert
   size_t counts;      // int32 [E]     assignments per expert (when the caller passes none)
-  size_t mtile;       // int32 [E+1]   prefix of ceil(count/kTileM) (tcgen05 tile schedule)
+  size_t mtile;       // int32 [E+1+kMaxShared] prefix of 256-token tiles over the GEMM groups
   size_t aux;         // fp32  [1]     statistic (when the caller passes none)
   size_t blk_cnt;     // int32 [nb*E]  per-router-block counts, then per-block base rows
   size_t blk_psum;    // fp32  [nb*E]  per-router-block sums of probabilities
   size_t lrank;       // int32 [T*k]   rank of (t,j) among its block's tokens of that expert
   size_t perm_tok;    // int32 [T*k]
-  size_t inv;         // int32 [T*k]
+  size_t inv;         // int32 [T*k]   row of each (token, slot), -1 when dropped
   size_t rgate;       // fp32  [T*k]   gate of every dispatched row
-  size_t xp;          // dtype [T*k, d] expert-contiguous copy of x
-  size_t h;           // dtype [T*k, I] SwiGLU hidden activations
-  size_t y;           // fp32  [T*k, d] expert outputs
+  size_t xp;          // dtype [T*k (+T), d] expert-contiguous (normalised) x; then x_hat for shared experts
+  size_t h;           // dtype [T*k + S*T, I] SwiGLU hidden activations (routed rows, then shared)
+  size_t y;           // fp32  [T*k + S*T, d] expert outputs
+  size_t blk_z;       // fp32  [nb]    per-router-block sums of logsumexp^2
+  size_t zloss;       // fp32  [1]     z-loss (when the caller passes none)
+  size_t dropped;     // int32 [1]     dropped assignments (when the caller passes none)
+  size_t rnorm;       // fp32  [T]     RMSNorm scale of every token
+  size_t wr_hi;       // bf16  [E, d]  high part of w * W_r (norm with a weight, bf16)
+  size_t wr_lo;       // bf16  [E, d]  low part of w * W_r
   size_t total;
 };
 
-Workspace workspace_layout(int T, int d, int E, int k, int I, moe_dtype dtype);
+constexpr int kMaxShared = MOE_MAX_SHARED;
+
+// The shared experts as extra groups of the grouped GEMMs: group E + s takes
+// `rows` (= T) rows starting at in0 + s * in_step of the input and writes them
+// at out0 + s * rows of the output.
+struct SharedGroups {
+  int n;        // number of shared experts (0: none)
+  int rows;     // T
+  int in0;      // first input row of shared expert 0
+  int in_step;  // input rows between shared experts (0: they all read the same rows)
+  int out0;     // first output row of shared expert 0
+};
+
+// Pre-MoE RMSNorm as the router applies it.
+struct RouterNorm {
+  int form;          // moe_norm_form (0: none)
+  float eps;
+  const void* w;     // fp32 path: the norm weight [d] (NULL: ones)
+  const void* w_hi;  // bf16 path: high part of w * W_r (NULL: no weight, plain W_r)
+  const void* w_lo;  // bf16 path: low part of w * W_r
+  float* rnorm;      // [T] out: the per-token scale
+};
+
+Workspace workspace_layout(int T, int d, int E, int k, int I, moe_dtype dtype, int n_shared = 0, bool norm = false);
 
 // Sets the calling thread's moe_last_error_detail() message (printf format).
 void set_error_detail(const char* fmt, ...);
@@ -94,44 +119,70 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 
 // ---- launchers (all asynchronous on `stream`) ----
 
+// blk_z (nullable): per-block sums of logsumexp(logits)^2 for the z-loss.
 cudaError_t launch_router(moe_dtype dtype, const void* x, const void* w_router, const float* b_router, int T,
-                          int d, int E, int k, int renorm, int32_t* topk_idx, float* topk_gate, int32_t* lrank,
-                          int32_t* blk_cnt, float* blk_psum, int32_t* status, cudaStream_t stream);
+                          int d, int E, int k, int renorm, const RouterNorm& norm, int32_t* topk_idx,
+                          float* topk_gate, int32_t* lrank, int32_t* blk_cnt, float* blk_psum, float* blk_z,
+                          int32_t* status, cudaStream_t stream);
 
 cudaError_t launch_router_tc(const void* x, const void* w_router, const float* b_router, int T, int d, int E, int k,
-                             int renorm, int32_t* topk_idx, float* topk_gate, int32_t* lrank, int32_t* blk_cnt,
-                             float* blk_psum, int32_t* status, cudaStream_t stream);
+                             int renorm, const RouterNorm& norm, int32_t* topk_idx, float* topk_gate, int32_t* lrank,
+                             int32_t* blk_cnt, float* blk_psum, float* blk_z, int32_t* status, cudaStream_t stream);
 
-cudaError_t launch_route_scan(int nb, int T, int E, int k, int32_t* blk_cnt, const float* blk_psum, int32_t* counts,
-                              int32_t* offsets, int32_t* mtile, float* aux, cudaStream_t stream);
+// hi[e,c] + lo[e,c] = w[c] * W_r[e,c] (bf16 + bf16; the fp32 product is exact).
+cudaError_t launch_split_router_weight(const void* w_router, const void* norm_w, int E, int d, void* hi, void* lo,
+                                       cudaStream_t stream);
+
+// cap < 0: no capacity. Writes counts (before dropping), offsets and the GEMM
+// tile prefix over the kept rows and the shared groups, aux, and optionally
+// the z-loss (from blk_z) and the dropped count.
+cudaError_t launch_route_scan(int nb, int T, int E, int k, int cap, int n_shared, int32_t* blk_cnt,
+                              const float* blk_psum, const float* blk_z, int32_t* counts, int32_t* offsets,
+                              int32_t* mtile, float* aux, float* zloss, int32_t* dropped, cudaStream_t stream);
 
 // Also records the gate of every dispatched row (rgate) and, when zero_out is
 // given, clears out[T, d] for a combine done by the down GEMM's epilogue.
+// rnorm != NULL: rows are x * rnorm[t] * norm_w (norm_w NULL: ones), rounded
+// to the dtype. shared_row0 >= 0: the (normalised) row of token t is also
+// written at row shared_row0 + t. has_cap: a row past its expert's kept count
+// is a dropped slot (inv = -1), not an error.
 cudaError_t launch_permute(moe_dtype dtype, const void* x, int T, int d, int E, int k, int rb, const int32_t* topk_idx,
-                           const int32_t* lrank, const int32_t* blk_base, int32_t* perm_tok, int32_t* inv,
-                           void* xp, const float* topk_gate, float* rgate, float* zero_out, int32_t* status,
+                           const int32_t* lrank, const int32_t* blk_base, const int32_t* offsets, int has_cap,
+                           int32_t* perm_tok, int32_t* inv, void* xp, const float* topk_gate, float* rgate,
+                           float* zero_out, const float* rnorm, const void* norm_w, int shared_row0, int32_t* status,
                            cudaStream_t stream);
 
+// out[t] = sum_j gate[t,j] * Y[inv[t,j]] (dropped slots skipped when has_cap)
+//        + sum_s Y[shared_row0 + s*T + t].
 cudaError_t launch_combine(int T, int d, int k, const float* y, const int32_t* inv, const float* topk_gate,
-                           float* out, int32_t* status, cudaStream_t stream);
+                           int has_cap, int n_shared, int shared_row0, float* out, int32_t* status,
+                           cudaStream_t stream);
 
 // tcgen05 grouped GEMMs (bf16) on CTA pairs: 256 weight rows x up to 256
 // dispatched tokens per tile. mode 0: H = SiLU(Xp Wg^T) * (Xp Wu^T) per
-// expert; mode 1: Y = H Wd^T per expert.
-cudaError_t launch_gemm_gateup_tc2(const CUtensorMap& tm_wg, const CUtensorMap& tm_wu, const CUtensorMap& tm_xp,
-                                   const CUtensorMap& tm_xp_small, const int32_t* offsets, const int32_t* mtile,
-                                   int R, int E, int I, int d, void* h, int32_t* status, cudaStream_t stream);
+// expert; mode 1: Y = H Wd^T per expert. Groups 0..E-1 are the routed experts
+// (rows from `offsets`), groups E.. the shared experts (`sh`, weights from the
+// tm_s* maps). R_rows: rows of the output scratch.
+cudaError_t launch_gemm_gateup_tc2(const CUtensorMap& tm_wg, const CUtensorMap& tm_wu, const CUtensorMap& tm_sg,
+                                   const CUtensorMap& tm_su, const CUtensorMap& tm_xp, const CUtensorMap& tm_xp_small,
+                                   const int32_t* offsets, const int32_t* mtile, int R_rows, int E,
+                                   const SharedGroups& sh, int I, int d, void* h, int32_t* status,
+                                   cudaStream_t stream);
 // comb_out != nullptr: instead of storing Y, add gate * y of every dispatched
-// row into comb_out[token] (used when k = 2, where the two adds commute).
-cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_wd, const CUtensorMap& tm_h, const CUtensorMap& tm_h_small,
-                                 const int32_t* offsets, const int32_t* mtile, int R, int E, int I, int d, float* y,
+// row into comb_out[token] (used when k = 2 without shared experts, where the
+// two adds commute).
+cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_wd, const CUtensorMap& tm_sd, const CUtensorMap& tm_h,
+                                 const CUtensorMap& tm_h_small, const int32_t* offsets, const int32_t* mtile,
+                                 int R_rows, int E, const SharedGroups& sh, int I, int d, float* y,
                                  const int32_t* perm_tok, const float* rgate, float* comb_out, int32_t* status,
                                  cudaStream_t stream);
 
-// fp32 SIMT grouped GEMMs.
-cudaError_t launch_gemm_gateup_simt(const float* xp, const float* wg, const float* wu, const int32_t* offsets,
-                                    int R, int E, int I, int d, float* h, cudaStream_t stream);
-cudaError_t launch_gemm_down_simt(const float* h, const float* wd, const int32_t* offsets, int R, int E, int I,
-                                  int d, float* y, cudaStream_t stream);
+// fp32 SIMT grouped GEMMs (same groups as above; sw*: the shared weights).
+cudaError_t launch_gemm_gateup_simt(const float* xp, const float* wg, const float* wu, const float* swg,
+                                    const float* swu, const int32_t* offsets, int R_rows, int E,
+                                    const SharedGroups& sh, int I, int d, float* h, cudaStream_t stream);
+cudaError_t launch_gemm_down_simt(const float* h, const float* wd, const float* swd, const int32_t* offsets,
+                                  int R_rows, int E, const SharedGroups& sh, int I, int d, float* y,
+                                  cudaStream_t stream);
 
 }  // namespace moe

@@ -4,6 +4,10 @@
 // expert"), and the token's row of x is copied to each of its k rows; and
 // kernel (d), the combine: out[t] = sum_j gate[t,j] * Y[row(t,j)] (same page,
 // "Scatter weighted outputs back", each expert weighted by its own gate).
+// Options: the pre-MoE RMSNorm is applied on the copy; with a capacity
+// ("moe_capacity_factor", KempnerForge ModelConfig) a slot whose rank in its
+// expert reaches the capacity is dropped; shared experts ("moe_shared_experts")
+// get every token's row and add their outputs with weight 1.
 #include "common.cuh"
 
 namespace moe {
@@ -11,18 +15,43 @@ namespace {
 
 constexpr int kCopyThreads = 256;  // 16-byte vectors per block (4 KB of a row)
 
+// x_hat = x * r * w for one 16-byte vector (8 bf16 or 4 fp32), rounded to
+// the dtype (the pre-MoE RMSNorm applied on the copy).
+__device__ __forceinline__ uint4 scale_vec(uint4 v, uint4 w, float r, bool bf16, bool has_w) {
+  uint32_t u[4] = {v.x, v.y, v.z, v.w};
+  const uint32_t uw[4] = {w.x, w.y, w.z, w.w};
+  if (bf16) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float a = __uint_as_float(u[i] << 16) * r, b = __uint_as_float(u[i] & 0xffff0000u) * r;
+      if (has_w) {
+        a *= __uint_as_float(uw[i] << 16);
+        b *= __uint_as_float(uw[i] & 0xffff0000u);
+      }
+      u[i] = pack_bf16x2(a, b);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float a = __uint_as_float(u[i]) * r;
+      if (has_w) a *= __uint_as_float(uw[i]);
+      u[i] = __float_as_uint(a);
+    }
+  }
+  return make_uint4(u[0], u[1], u[2], u[3]);
+}
+
 // Block (token t, chunk c): threads j < k compute the row of slot j from the
 // per-block base row of its expert plus its rank inside the router block
 // (chunk 0 also records perm_tok / inv); then every thread copies one 16-byte
-// vector of x[t] to each of the token's k rows.
-__global__ void __launch_bounds__(kCopyThreads) permute_kernel(const uint4* __restrict__ x, int nvec, int E, int k,
-                                                              int rb, int R, const int32_t* __restrict__ topk_idx,
-                                                              const int32_t* __restrict__ lrank,
-                                                              const int32_t* __restrict__ blk_base,
-                                                              int32_t* __restrict__ perm_tok, int32_t* __restrict__ inv,
-                                                              uint4* __restrict__ xp, const float* __restrict__ gate,
-                                                              float* __restrict__ rgate, float4* __restrict__ zero_out,
-                                                              int nout4, int32_t* status) {
+// vector of x[t] (normalised when rnorm is given) to each of the token's kept
+// rows and, with shared experts, to row shared_row0 + t.
+__global__ void __launch_bounds__(kCopyThreads) permute_kernel(
+    const uint4* __restrict__ x, int nvec, int E, int k, int rb, int R, const int32_t* __restrict__ topk_idx,
+    const int32_t* __restrict__ lrank, const int32_t* __restrict__ blk_base, const int32_t* __restrict__ offsets,
+    int has_cap, int32_t* __restrict__ perm_tok, int32_t* __restrict__ inv, uint4* __restrict__ xp,
+    const float* __restrict__ gate, float* __restrict__ rgate, float4* __restrict__ zero_out, int nout4,
+    const float* __restrict__ rnorm, const uint4* __restrict__ norm_w, int bf16, int shared_row0, int32_t* status) {
   const int t = blockIdx.x;
   __shared__ int s_rows[kMaxTopK];
   pdl_wait();
@@ -30,11 +59,20 @@ __global__ void __launch_bounds__(kCopyThreads) permute_kernel(const uint4* __re
     const int j = threadIdx.x;
     const int e = topk_idx[(size_t)t * k + j];
     int row = -1;
-    if (e >= 0 && e < E) row = blk_base[(size_t)(t / rb) * E + e] + lrank[(size_t)t * k + j];
-    if (row < 0 || row >= R) {
+    bool bad = e < 0 || e >= E;
+    if (!bad) {
+      row = blk_base[(size_t)(t / rb) * E + e] + lrank[(size_t)t * k + j];
+      if (has_cap && row >= offsets[e + 1]) {
+        row = -1;  // past the expert's capacity: this slot is dropped
+        if (blockIdx.y == 0) inv[(size_t)t * k + j] = -1;
+      } else if (row < 0 || row >= R) {
+        bad = true;
+      }
+    }
+    if (bad) {
       atomicOr(status, MOE_DEV_INTERNAL);
       row = -1;
-    } else if (blockIdx.y == 0) {
+    } else if (row >= 0 && blockIdx.y == 0) {
       perm_tok[row] = t;
       inv[(size_t)t * k + j] = row;
       rgate[row] = gate[(size_t)t * k + j];
@@ -49,17 +87,22 @@ __global__ void __launch_bounds__(kCopyThreads) permute_kernel(const uint4* __re
   }
   const int i = blockIdx.y * kCopyThreads + threadIdx.x;
   if (i >= nvec) return;
-  const uint4 v = __ldg(x + (size_t)t * nvec + i);
+  uint4 v = __ldg(x + (size_t)t * nvec + i);
+  if (rnorm) v = scale_vec(v, norm_w ? __ldg(norm_w + i) : make_uint4(0u, 0u, 0u, 0u), rnorm[t], bf16 != 0,
+                           norm_w != nullptr);
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j)
     if (j < k && s_rows[j] >= 0) xp[(size_t)s_rows[j] * nvec + i] = v;
+  if (shared_row0 >= 0) xp[(size_t)(shared_row0 + t) * nvec + i] = v;
 }
 
 // Block (token t, chunk c): every thread sums one float4 of its token's k
-// expert rows, weighted by the gates, in slot order (fp32).
+// expert rows, weighted by the gates, in slot order (fp32), skipping dropped
+// slots, then adds the token's rows of the shared experts in order.
 __global__ void __launch_bounds__(kCopyThreads) combine_kernel(const float4* __restrict__ y, int nvec4, int k, int R,
-                                                              const int32_t* __restrict__ inv,
-                                                              const float* __restrict__ gate,
+                                                              int T, const int32_t* __restrict__ inv,
+                                                              const float* __restrict__ gate, int has_cap,
+                                                              int n_shared, int shared_row0,
                                                               float4* __restrict__ out, int32_t* status) {
   const int t = blockIdx.x;
   __shared__ int s_rows[kMaxTopK];
@@ -69,10 +112,11 @@ __global__ void __launch_bounds__(kCopyThreads) combine_kernel(const float4* __r
     const int j = threadIdx.x;
     int row = inv[(size_t)t * k + j];
     float g = gate[(size_t)t * k + j];
-    if (row < 0 || row >= R) {
+    if (row < 0 && has_cap) {
+      row = -1;  // dropped slot
+    } else if (row < 0 || row >= R) {
       atomicOr(status, MOE_DEV_INTERNAL);
-      row = 0;
-      g = 0.f;
+      row = -1;
     }
     s_rows[j] = row;
     s_g[j] = g;
@@ -83,11 +127,11 @@ __global__ void __launch_bounds__(kCopyThreads) combine_kernel(const float4* __r
   float4 v[kMaxTopK];
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j)
-    if (j < k) v[j] = __ldg(y + (size_t)s_rows[j] * nvec4 + i);
+    if (j < k && s_rows[j] >= 0) v[j] = __ldg(y + (size_t)s_rows[j] * nvec4 + i);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j) {
-    if (j < k) {
+    if (j < k && s_rows[j] >= 0) {
       const float g = s_g[j];
       acc.x = fmaf(g, v[j].x, acc.x);
       acc.y = fmaf(g, v[j].y, acc.y);
@@ -95,29 +139,39 @@ __global__ void __launch_bounds__(kCopyThreads) combine_kernel(const float4* __r
       acc.w = fmaf(g, v[j].w, acc.w);
     }
   }
+  for (int s2 = 0; s2 < n_shared; ++s2) {
+    const float4 u = __ldg(y + (size_t)(shared_row0 + s2 * T + t) * nvec4 + i);
+    acc.x += u.x;
+    acc.y += u.y;
+    acc.z += u.z;
+    acc.w += u.w;
+  }
   out[(size_t)t * nvec4 + i] = acc;
 }
 
 }  // namespace
 
 cudaError_t launch_permute(moe_dtype dtype, const void* x, int T, int d, int E, int k, int rb, const int32_t* topk_idx,
-                           const int32_t* lrank, const int32_t* blk_base, int32_t* perm_tok, int32_t* inv, void* xp,
-                           const float* topk_gate, float* rgate, float* zero_out, int32_t* status,
+                           const int32_t* lrank, const int32_t* blk_base, const int32_t* offsets, int has_cap,
+                           int32_t* perm_tok, int32_t* inv, void* xp, const float* topk_gate, float* rgate,
+                           float* zero_out, const float* rnorm, const void* norm_w, int shared_row0, int32_t* status,
                            cudaStream_t stream) {
   const int elem = dtype == MOE_BF16 ? 2 : 4;
   const int nvec = d * elem / 16;
   const dim3 grid(T, (nvec + kCopyThreads - 1) / kCopyThreads);
   return launch_pdl(permute_kernel, grid, dim3(kCopyThreads), 0, stream, static_cast<const uint4*>(x), nvec, E, k, rb,
-                    T * k, topk_idx, lrank, blk_base, perm_tok, inv, static_cast<uint4*>(xp), topk_gate, rgate,
-                    reinterpret_cast<float4*>(zero_out), d / 4, status);
+                    T * k, topk_idx, lrank, blk_base, offsets, has_cap, perm_tok, inv, static_cast<uint4*>(xp),
+                    topk_gate, rgate, reinterpret_cast<float4*>(zero_out), d / 4, rnorm,
+                    static_cast<const uint4*>(norm_w), dtype == MOE_BF16 ? 1 : 0, shared_row0, status);
 }
 
-cudaError_t launch_combine(int T, int d, int k, const float* y, const int32_t* inv, const float* topk_gate, float* out,
-                           int32_t* status, cudaStream_t stream) {
+cudaError_t launch_combine(int T, int d, int k, const float* y, const int32_t* inv, const float* topk_gate,
+                           int has_cap, int n_shared, int shared_row0, float* out, int32_t* status,
+                           cudaStream_t stream) {
   const int nvec4 = d / 4;
   const dim3 grid(T, (nvec4 + kCopyThreads - 1) / kCopyThreads);
   return launch_pdl(combine_kernel, grid, dim3(kCopyThreads), 0, stream, reinterpret_cast<const float4*>(y), nvec4, k,
-                    T * k, inv, topk_gate, reinterpret_cast<float4*>(out), status);
+                    T * k, T, inv, topk_gate, has_cap, n_shared, shared_row0, reinterpret_cast<float4*>(out), status);
 }
 
 }  // namespace moe

@@ -19,8 +19,10 @@ namespace moe {
 namespace {
 
 // fp32 logits with plain FFMA (the fp32 workload is small; TF32 tensor cores
-// would not meet its 1e-4 tolerance).
-__device__ void router_logits_f32(const float* __restrict__ x, const float* __restrict__ wr, int T, int d, int E,
+// would not meet its 1e-4 tolerance). With the RMSNorm, s_r[row] holds the
+// token's scale and the logit is r * sum_c x[c] * (w[c] * W_r[e,c]).
+__device__ void router_logits_f32(const float* __restrict__ x, const float* __restrict__ wr,
+                                  const float* __restrict__ nw, bool norm, const float* s_r, int T, int d, int E,
                                   int tok0, float* s_logit, int ld) {
   for (int i = threadIdx.x; i < kRouterTokensSimt * E; i += blockDim.x) {
     const int e = i / kRouterTokensSimt, row = i - e * kRouterTokensSimt;
@@ -29,7 +31,11 @@ __device__ void router_logits_f32(const float* __restrict__ x, const float* __re
     if (t < T) {
       const float* xr = x + (size_t)t * d;
       const float* wrow = wr + (size_t)e * d;
-      for (int c = 0; c < d; ++c) s = fmaf(xr[c], wrow[c], s);
+      if (nw)
+        for (int c = 0; c < d; ++c) s = fmaf(xr[c], nw[c] * wrow[c], s);
+      else
+        for (int c = 0; c < d; ++c) s = fmaf(xr[c], wrow[c], s);
+      if (norm) s *= s_r[row];
     }
     s_logit[row * ld + e] = s;
   }
@@ -38,25 +44,50 @@ __device__ void router_logits_f32(const float* __restrict__ x, const float* __re
 
 __global__ void __launch_bounds__(kRouterThreads) router_kernel(
     const float* __restrict__ x, const float* __restrict__ wr, const float* __restrict__ br, int T, int d, int E, int k,
-    int renorm, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate, int32_t* __restrict__ lrank,
-    int32_t* __restrict__ blk_cnt, float* __restrict__ blk_psum, int32_t* status) {
+    int renorm, int norm_form, float norm_eps, const float* __restrict__ nw, float* __restrict__ rnorm,
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate, int32_t* __restrict__ lrank,
+    int32_t* __restrict__ blk_cnt, float* __restrict__ blk_psum, float* __restrict__ blk_z, int32_t* status) {
   extern __shared__ float smem[];
   const int ld = E + 1;
   float* s_p = smem;  // [32][E+1] logits, then probabilities
   __shared__ int32_t s_idx[kRouterTokensSimt][kMaxTopK];
+  __shared__ float s_r[kRouterTokensSimt];  // RMSNorm scale per token
+  __shared__ float s_z[kRouterTokensSimt];  // logsumexp^2 per token
 
   const int tok0 = blockIdx.x * kRouterTokensSimt;
   const int ntok = min(kRouterTokensSimt, T - tok0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   pdl_wait();
-  router_logits_f32(x, wr, T, d, E, tok0, s_p, ld);
+  if (norm_form) {
+    // one thread per token: the sum of x^2 in 32-element pieces
+    if (threadIdx.x < kRouterTokensSimt) {
+      const int t = tok0 + threadIdx.x;
+      float r = 1.0f;
+      if (t < T) {
+        const float* xr = x + (size_t)t * d;
+        float ss = 0.f;
+        for (int c0 = 0; c0 < d; c0 += 32) {
+          float part = 0.f;
+          for (int c = c0; c < min(d, c0 + 32); ++c) part = fmaf(xr[c], xr[c], part);
+          ss += part;
+        }
+        const float ms = ss / (float)d;
+        r = norm_form == MOE_NORM_RMS ? 1.0f / sqrtf(ms + norm_eps) : 1.0f / (sqrtf(ms) + norm_eps);
+        rnorm[t] = r;
+      }
+      s_r[threadIdx.x] = r;
+    }
+    __syncthreads();
+  }
+  router_logits_f32(x, wr, nw, norm_form != 0, s_r, T, d, E, tok0, s_p, ld);
 
   // ---- softmax, top-k and gates: one warp per token --------------------
   const int NE = (E + 31) >> 5;  // values per lane (<= 8)
   for (int row = warp; row < kRouterTokensSimt; row += kRouterThreads / 32) {
     if (row >= ntok) {
       if (lane < kMaxTopK) s_idx[row][lane] = -1;
+      if (lane == 0) s_z[row] = 0.f;
       for (int e = lane; e < E; e += 32) s_p[row * ld + e] = 0.f;
       continue;
     }
@@ -88,6 +119,10 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(
     }
 #pragma unroll
     for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) {
+      const float lse = m + logf(s);
+      s_z[row] = lse * lse;
+    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int e = lane + 32 * i;
@@ -175,15 +210,28 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(
     for (int row = 0; row < ntok; ++row) s += s_p[row * ld + e];
     blk_psum[(size_t)blockIdx.x * E + e] = s;
   }
+  if (blk_z && threadIdx.x == 0) {
+    float z = 0.f;
+    for (int row = 0; row < ntok; ++row) z += s_z[row];
+    blk_z[blockIdx.x] = z;
+  }
 }
 
 // One CTA of 1024 threads. Thread (e, slice) reduces a contiguous range of
 // router blocks for expert e; slices are then scanned in order, so every
-// result is deterministic.
-__global__ void __launch_bounds__(1024) route_scan_kernel(int nb, int T, int E, int k, int32_t* __restrict__ blk_cnt,
+// result is deterministic. With a capacity (cap >= 0) an expert keeps
+// min(count, cap) rows: offsets and the GEMM tile prefix cover the kept rows
+// only, and a row computed past its expert's kept count is a dropped slot.
+// The shared experts follow the routed experts in the tile prefix, T rows
+// each. Warp 1 sums the per-block z-loss partials in fp64 while thread 0
+// walks the experts.
+__global__ void __launch_bounds__(1024) route_scan_kernel(int nb, int T, int E, int k, int cap, int n_shared,
+                                                          int32_t* __restrict__ blk_cnt,
                                                           const float* __restrict__ blk_psum,
+                                                          const float* __restrict__ blk_z,
                                                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                                                          int32_t* __restrict__ mtile, float* __restrict__ aux) {
+                                                          int32_t* __restrict__ mtile, float* __restrict__ aux,
+                                                          float* __restrict__ zloss, int32_t* __restrict__ dropped) {
   __shared__ int s_cnt[1024];
   __shared__ double s_ps[1024];
   __shared__ int s_tot[kMaxExperts];
@@ -222,21 +270,37 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int nb, int T, int E, 
   }
   __syncthreads();
   if (tid == 0) {
-    int off = 0, mt = 0;
+    int off = 0, mt = 0, drop = 0;
     double a = 0.0;
     for (int ee = 0; ee < E; ++ee) {
+      const int tot = s_tot[ee];
+      const int kept = cap >= 0 ? min(tot, cap) : tot;
       s_off[ee] = off;
       offsets[ee] = off;
       mtile[ee] = mt;
-      if (counts) counts[ee] = s_tot[ee];
-      a += ((double)s_tot[ee] / ((double)T * (double)k)) * (s_ptot[ee] / (double)T);
-      off += s_tot[ee];
-      mt += (s_tot[ee] + kTileM - 1) / kTileM;
+      if (counts) counts[ee] = tot;
+      a += ((double)tot / ((double)T * (double)k)) * (s_ptot[ee] / (double)T);
+      off += kept;
+      drop += tot - kept;
+      mt += (kept + kTileM - 1) / kTileM;
     }
     offsets[E] = off;
-    mtile[E] = mt;
     s_off[E] = off;
+    mtile[E] = mt;
+    for (int s2 = 0; s2 < n_shared; ++s2) {
+      mt += (T + kTileM - 1) / kTileM;
+      mtile[E + 1 + s2] = mt;
+    }
     if (aux) *aux = (float)((double)E * a);
+    if (dropped) *dropped = drop;
+  }
+  if (zloss && tid >= 32 && tid < 64) {
+    const int ln = tid - 32;
+    double z = 0.0;
+    for (int b = ln; b < nb; b += 32) z += (double)blk_z[b];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (ln == 0) *zloss = (float)(z / (double)T);
   }
   __syncthreads();
   if (active) {
@@ -252,24 +316,27 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int nb, int T, int E, 
 }  // namespace
 
 cudaError_t launch_router(moe_dtype dtype, const void* x, const void* w_router, const float* b_router, int T, int d,
-                          int E, int k, int renorm, int32_t* topk_idx, float* topk_gate, int32_t* lrank,
-                          int32_t* blk_cnt, float* blk_psum, int32_t* status, cudaStream_t stream) {
+                          int E, int k, int renorm, const RouterNorm& norm, int32_t* topk_idx, float* topk_gate,
+                          int32_t* lrank, int32_t* blk_cnt, float* blk_psum, float* blk_z, int32_t* status,
+                          cudaStream_t stream) {
   if (dtype == MOE_BF16)
-    return launch_router_tc(x, w_router, b_router, T, d, E, k, renorm, topk_idx, topk_gate, lrank, blk_cnt, blk_psum,
-                            status, stream);
+    return launch_router_tc(x, w_router, b_router, T, d, E, k, renorm, norm, topk_idx, topk_gate, lrank, blk_cnt,
+                            blk_psum, blk_z, status, stream);
   const int nb = router_blocks(T, MOE_F32);
   const size_t smem = (size_t)kRouterTokensSimt * (E + 1) * sizeof(float);
   cudaError_t err = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   return launch_pdl(router_kernel, dim3(nb), dim3(kRouterThreads), smem, stream, static_cast<const float*>(x),
-                    static_cast<const float*>(w_router), b_router, T, d, E, k, renorm, topk_idx, topk_gate, lrank,
-                    blk_cnt, blk_psum, status);
+                    static_cast<const float*>(w_router), b_router, T, d, E, k, renorm, norm.form, norm.eps,
+                    static_cast<const float*>(norm.w), norm.rnorm, topk_idx, topk_gate, lrank, blk_cnt, blk_psum,
+                    blk_z, status);
 }
 
-cudaError_t launch_route_scan(int nb, int T, int E, int k, int32_t* blk_cnt, const float* blk_psum, int32_t* counts,
-                              int32_t* offsets, int32_t* mtile, float* aux, cudaStream_t stream) {
-  return launch_pdl(route_scan_kernel, dim3(1), dim3(1024), 0, stream, nb, T, E, k, blk_cnt, blk_psum, counts, offsets,
-                    mtile, aux);
+cudaError_t launch_route_scan(int nb, int T, int E, int k, int cap, int n_shared, int32_t* blk_cnt,
+                              const float* blk_psum, const float* blk_z, int32_t* counts, int32_t* offsets,
+                              int32_t* mtile, float* aux, float* zloss, int32_t* dropped, cudaStream_t stream) {
+  return launch_pdl(route_scan_kernel, dim3(1), dim3(1024), 0, stream, nb, T, E, k, cap, n_shared, blk_cnt, blk_psum,
+                    blk_z, counts, offsets, mtile, aux, zloss, dropped);
 }
 
 }  // namespace moe

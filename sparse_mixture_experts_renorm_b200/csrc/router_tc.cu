@@ -18,7 +18,16 @@
 // the leading CTA's shared memory, which finishes the block: one thread per
 // token does the softmax, top-k and gates without cross-thread reductions
 // (logits in registers for E <= 64), then the block's histogram, ranks and
-// probability sums.
+// probability sums, and the block's sum of logsumexp^2 for the z-loss.
+//
+// With the pre-MoE RMSNorm (Mixtral MoE Block, nn.RMSNorm before the MoE;
+// Model Architecture Patterns, "RMSNorm") the logits are
+//   l[t,e] = r_t * sum_c x[t,c] * (w[c] * W_r[e,c]) + b[e],
+// r_t = 1/sqrt(mean x^2 + eps) or 1/(sqrt(mean x^2) + eps): the epilogue
+// warps square-sum their token's row of every x tile while the UMMAs run
+// (they are extra consumers of the ring), and w * W_r enters as two bf16
+// operands hi + lo whose products go to two accumulators, so x is used as
+// stored and the weight's product is carried to about 16 bits.
 #include <math.h>
 
 #include "common.cuh"
@@ -31,30 +40,33 @@ constexpr int kRegE = 64;             // up to this many experts a token's logit
 
 struct RouterCfg {
   int npad;         // UMMA N
+  int lo_col;       // TMEM column of the second (w * W_r low part) accumulator
   int S;            // CTAs per token block (split of the K loop)
   int stages;       // ring depth
-  int stage_bytes;  // x tile + W_r tile
-  int part_bytes;   // partial-logit buffer of the leading CTA
+  int stage_bytes;  // x tile + W_r tile(s)
+  int part_bytes;   // partial-logit (and partial square-sum) buffer of the leading CTA
   int tmem_cols;    // power of two >= max(32, columns read)
   int smem_bytes;   // dynamic shared memory
 };
 
-RouterCfg router_cfg(int T, int d, int E, int num_sms) {
+RouterCfg router_cfg(int T, int d, int E, bool norm, bool split, int num_sms) {
   RouterCfg c;
   c.npad = ((E + 15) / 16) * 16;
-  c.stage_bytes = kRB * kBK * 2 + c.npad * kBK * 2;
+  c.lo_col = 32 * ((E + 31) / 32);
+  c.stage_bytes = kRB * kBK * 2 + (split ? 2 : 1) * c.npad * kBK * 2;
   const int nb = (T + kRB - 1) / kRB;
   const int KB = d / kBK;
+  const int per_cta = kRB * (E + (norm ? 1 : 0)) * 4;
   // split K only while the grid leaves SMs idle, the partial logits stay
   // small, and each CTA keeps at least two k-blocks
   c.S = 1;
   if (E <= kRegE)
-    while (c.S < 8 && nb * c.S * 2 <= num_sms && (c.S * 2 - 1) * kRB * E * 4 <= 64 * 1024 && KB / (c.S * 2) >= 2)
+    while (c.S < 8 && nb * c.S * 2 <= num_sms && (c.S * 2 - 1) * per_cta <= 64 * 1024 && KB / (c.S * 2) >= 2)
       c.S *= 2;
-  c.part_bytes = (c.S - 1) * kRB * E * 4;
+  c.part_bytes = (c.S - 1) * per_cta;
   c.stages = (192 * 1024 - c.part_bytes) / c.stage_bytes;
   if (c.stages > 8) c.stages = 8;
-  const int cols = 32 * ((E + 31) / 32);
+  const int cols = split ? 2 * c.lo_col : c.lo_col;
   c.tmem_cols = 32;
   while (c.tmem_cols < cols) c.tmem_cols <<= 1;
   c.smem_bytes = c.stages * c.stage_bytes + c.part_bytes + 1024 + 12288;
@@ -102,15 +114,18 @@ __device__ __forceinline__ void topk_insert(float (&bv)[kMaxTopK], int (&be)[kMa
 template <int kE>  // E <= kE: logits in registers; kE == 0: E > kRegE, logits in shared memory
 __global__ void __launch_bounds__(kGemmThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                     const float* __restrict__ br, int T, int d, int E, int k, int renorm, int npad, int S,
-                     int stages, int stage_bytes, int tmem_cols, int32_t* __restrict__ topk_idx,
-                     float* __restrict__ topk_gate, int32_t* __restrict__ lrank, int32_t* __restrict__ blk_cnt,
-                     float* __restrict__ blk_psum, int32_t* status, uint64_t limit_ns) {
+                     const __grid_constant__ CUtensorMap tmW2, const float* __restrict__ br, int T, int d, int E,
+                     int k, int renorm, int npad, int lo_col, int split, int S, int stages, int stage_bytes,
+                     int part_bytes, int tmem_cols, int norm_form, float norm_eps, float* __restrict__ rnorm,
+                     int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate, int32_t* __restrict__ lrank,
+                     int32_t* __restrict__ blk_cnt, float* __restrict__ blk_psum, float* __restrict__ blk_z,
+                     int32_t* status, uint64_t limit_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
   float* part = reinterpret_cast<float*>(smem + stages * stage_bytes);  // [S-1][128][E] (leading CTA)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes + (S - 1) * kRB * E * 4);
+  float* part_ss = part + (size_t)(S - 1) * kRB * E;                   // [S-1][128] square sums (norm)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes + part_bytes);
   uint64_t* full = bars;           // [stages]
   uint64_t* empty = bars + 8;      // [stages]
   uint64_t* tfull = bars + 16;
@@ -119,6 +134,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_idx = reinterpret_cast<int*>(s_tmem + 4);  // [128][kMaxTopK]
   int* s_wcnt = s_idx + kRB * kMaxTopK;              // [4][E] per-warp counts, then exclusive prefix
+  float* s_z = reinterpret_cast<float*>(s_wcnt + 4 * E);  // [4] per-warp sums of logsumexp^2
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = S > 1 ? cta_rank_in_cluster() : 0u;
@@ -127,11 +143,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int KB = d / kBK;
   const int kb0 = (int)rank * KB / S, kb1 = ((int)rank + 1) * KB / S;
   const int a_bytes = kRB * kBK * 2;
+  const int w_bytes = npad * kBK * 2;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      // the UMMA commit, plus the 4 epilogue warps when they read x for the norm
+      mbar_init(&empty[s], norm_form ? 5 : 1);
     }
     mbar_init(tfull, 1);
     mbar_init(done, 1);
@@ -141,6 +159,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmW);
+    if (split) tma_prefetch_desc(&tmW2);
   }
   if (warp == 1) {
     tmem_alloc(s_tmem, tmem_cols);
@@ -153,7 +172,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   pdl_wait();
 
   constexpr int kL = kE > 0 ? kE : 1;
-  float lg[kL];  // this token's logits (register path)
+  float lg[kL];    // this token's logits (register path)
+  float ss = 0.f;  // this token's sum of x^2 (RMSNorm)
   if (warp == 0) {
     if (lane == 0) {
       int stage = 0;
@@ -165,6 +185,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint8_t* st = ring + stage * stage_bytes;
         tma_load_2d(st, &tmX, &full[stage], kb * kBK, tok0);
         tma_load_2d(st + a_bytes, &tmW, &full[stage], kb * kBK, 0);
+        if (split) tma_load_2d(st + a_bytes + w_bytes, &tmW2, &full[stage], kb * kBK, 0);
         ++issued;
         if (++stage == stages) {
           stage = 0;
@@ -197,10 +218,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint8_t* st = ring + stage * stage_bytes;
         const uint64_t adesc = sw128_kmajor_desc(smem_u32(st));
         const uint64_t bdesc = sw128_kmajor_desc(smem_u32(st + a_bytes));
+        const uint64_t bdesc2 = sw128_kmajor_desc(smem_u32(st + a_bytes + w_bytes));
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk)
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint32_t accum = (kb > kb0 || kk > 0) ? 1u : 0u;
           tc_mma_bf16(tmem_base, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2), idesc,
-                      (kb > kb0 || kk > 0) ? 1u : 0u);
+                      accum);
+          if (split)
+            tc_mma_bf16(tmem_base + static_cast<uint32_t>(lo_col), adesc + static_cast<uint64_t>(kk * 2),
+                        bdesc2 + static_cast<uint64_t>(kk * 2), idesc, accum);
+        }
         tc_commit(&empty[stage]);
         if (++stage == stages) {
           stage = 0;
@@ -213,9 +240,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     __syncwarp();
   } else {
-    // -------------------------- read this CTA's partial logits from TMEM --
     const int q = warp & 3;
     const int r = q * 32 + lane;
+    // ------------- RMSNorm: this token's sum of x^2 over this CTA's K slice --
+    // Row r of a 128B-swizzled x tile holds its 16-byte chunk c at position
+    // c ^ (r & 7); each stage is summed on its own, then added to the total.
+    if (norm_form) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[stage], phase, s_abort, status, limit_ns))) break;
+        const uint8_t* row = ring + stage * stage_bytes + r * 128;
+        float part_s = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(row + ((c ^ (r & 7)) << 4));
+          const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float lo = __uint_as_float(u[i] << 16), hi = __uint_as_float(u[i] & 0xffff0000u);
+            part_s = fmaf(lo, lo, part_s);
+            part_s = fmaf(hi, hi, part_s);
+          }
+        }
+        ss += part_s;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[stage]);
+        if (++stage == stages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    // -------------------------- read this CTA's partial logits from TMEM --
     const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull, 0, s_abort, status, limit_ns));
     tc_fence_after();
     const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
@@ -227,6 +284,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (ok) {
         tmem_ld_x32(trow + c * 32, v);
         tmem_ld_wait();
+        if (split) {
+          uint32_t v2[32];
+          __syncwarp();
+          tmem_ld_x32(trow + static_cast<uint32_t>(lo_col) + c * 32, v2);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) + __uint_as_float(v2[i]));
+        }
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = 0u;
@@ -248,6 +313,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
       for (int e = 0; e < kL; ++e)
         if (e < E) st_cluster_f32(dst + e, 0, lg[e]);
+      if (norm_form) st_cluster_f32(part_ss + (size_t)(rank - 1) * kRB + r, 0, ss);
     }
   }
 
@@ -269,8 +335,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       be[j] = 0x7fffffff;
     }
     bool finite = true;
+    // RMSNorm scale of this token (1 without the norm)
+    float rn = 1.0f;
+    if (norm_form) {
+      for (int s2 = 0; s2 < S - 1; ++s2) ss += part_ss[(size_t)s2 * kRB + r];
+      const float ms = ss / (float)d;
+      rn = norm_form == MOE_NORM_RMS ? 1.0f / sqrtf(ms + norm_eps) : 1.0f / (sqrtf(ms) + norm_eps);
+      if (valid) rnorm[t] = rn;
+    }
+    float lse;  // log sum_e exp(logit)
     if (kE > 0) {
-      // the other CTAs' partial logits in rank order, the bias, the maximum
+      // the other CTAs' partial logits in rank order, the norm scale, the
+      // bias, the maximum
       for (int s2 = 0; s2 < S - 1; ++s2) {
         const float* src = part + ((size_t)s2 * kRB + r) * E;
 #pragma unroll
@@ -281,6 +357,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
       for (int e = 0; e < kL; ++e)
         if (e < E) {
+          if (norm_form) lg[e] *= rn;
           if (br) lg[e] += br[e];
           finite = finite && isfinite(lg[e]);
           m = fmaxf(m, lg[e]);
@@ -292,6 +369,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           lg[e] = __expf(lg[e] - m);
           s += lg[e];
         }
+      lse = m + logf(s);
       const float inv_s = 1.0f / s;
 #pragma unroll
       for (int e = 0; e < kL; ++e)
@@ -304,6 +382,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       float m = -INFINITY;
       for (int e = 0; e < E; ++e) {
         float l = s_p[r * ld + e];
+        if (norm_form) l *= rn;
         if (br) l += br[e];
         finite = finite && isfinite(l);
         m = fmaxf(m, l);
@@ -315,6 +394,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         s_p[r * ld + e] = ex;
         s += ex;
       }
+      lse = m + logf(s);
       const float inv_s = 1.0f / s;
       for (int e = 0; e < E; ++e) {
         const float p = s_p[r * ld + e] * inv_s;
@@ -323,6 +403,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
     if (valid && !finite) atomicOr(status, MOE_DEV_NONFINITE);
+    if (blk_z) {  // this warp's sum of logsumexp^2 (a fixed shuffle tree)
+      float z = valid ? lse * lse : 0.f;
+#pragma unroll
+      for (int off = 16; off; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+      if (lane == 0) s_z[q] = z;
+    }
     float psel = 0.f;
 #pragma unroll
     for (int j = 0; j < kMaxTopK; ++j)
@@ -381,6 +467,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int rr = 0; rr < kRB; ++rr) ps += s_p[rr * ld + e];
       blk_psum[(size_t)blk * E + e] = ps;
     }
+    if (blk_z && r == 0) blk_z[blk] = ((s_z[0] + s_z[1]) + s_z[2]) + s_z[3];
     epi_bar();
     if (valid) {
 #pragma unroll
@@ -414,12 +501,14 @@ int sm_count() {
 }  // namespace
 
 cudaError_t launch_router_tc(const void* x, const void* w_router, const float* b_router, int T, int d, int E, int k,
-                             int renorm, int32_t* topk_idx, float* topk_gate, int32_t* lrank, int32_t* blk_cnt,
-                             float* blk_psum, int32_t* status, cudaStream_t stream) {
-  const RouterCfg c = router_cfg(T, d, E, sm_count());
-  CUtensorMap tmX, tmW;
+                             int renorm, const RouterNorm& norm, int32_t* topk_idx, float* topk_gate, int32_t* lrank,
+                             int32_t* blk_cnt, float* blk_psum, float* blk_z, int32_t* status, cudaStream_t stream) {
+  const bool split = norm.form != 0 && norm.w_hi != nullptr;
+  const RouterCfg c = router_cfg(T, d, E, norm.form != 0, split, sm_count());
+  CUtensorMap tmX, tmW, tmW2;
   if (!make_tmap_bf16_2d(&tmX, x, (uint64_t)T, (uint64_t)d, kRB) ||
-      !make_tmap_bf16_2d(&tmW, w_router, (uint64_t)E, (uint64_t)d, (uint32_t)c.npad))
+      !make_tmap_bf16_2d(&tmW, split ? norm.w_hi : w_router, (uint64_t)E, (uint64_t)d, (uint32_t)c.npad) ||
+      !make_tmap_bf16_2d(&tmW2, split ? norm.w_lo : w_router, (uint64_t)E, (uint64_t)d, (uint32_t)c.npad))
     return cudaErrorInvalidValue;
   auto kern = E <= 16 ? router_tc_kernel<16> : E <= 32 ? router_tc_kernel<32> : E <= kRegE ? router_tc_kernel<kRegE>
                                                                                            : router_tc_kernel<0>;
@@ -440,9 +529,52 @@ cudaError_t launch_router_tc(const void* x, const void* w_router, const float* b
   attrs[1].val.clusterDim.z = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = c.S > 1 ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, kern, tmX, tmW, b_router, T, d, E, k, renorm, c.npad, c.S, c.stages,
-                            c.stage_bytes, c.tmem_cols, topk_idx, topk_gate, lrank, blk_cnt, blk_psum, status,
-                            kWaitLimitNs);
+  return cudaLaunchKernelEx(&cfg, kern, tmX, tmW, tmW2, b_router, T, d, E, k, renorm, c.npad, c.lo_col, split ? 1 : 0,
+                            c.S, c.stages, c.stage_bytes, c.part_bytes, c.tmem_cols, norm.form, norm.eps, norm.rnorm,
+                            topk_idx, topk_gate, lrank, blk_cnt, blk_psum, blk_z, status, kWaitLimitNs);
+}
+
+namespace {
+
+// hi = bf16(w * W_r) (round to nearest even), lo = bf16(w * W_r - hi): the
+// product of two bf16 values is exact in fp32, and hi + lo keeps about 16 of
+// its bits.
+__global__ void __launch_bounds__(256) split_router_weight_kernel(const uint4* __restrict__ wr,
+                                                                 const uint4* __restrict__ w, int E, int dv,
+                                                                 uint4* __restrict__ hi, uint4* __restrict__ lo) {
+  pdl_wait();
+  const int n = E * dv;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const uint4 a = wr[i], b = w[i % dv];
+    const uint32_t ua[4] = {a.x, a.y, a.z, a.w}, ub[4] = {b.x, b.y, b.z, b.w};
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float p0 = __uint_as_float(ua[j] << 16) * __uint_as_float(ub[j] << 16);
+      const float p1 = __uint_as_float(ua[j] & 0xffff0000u) * __uint_as_float(ub[j] & 0xffff0000u);
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(p0), h1 = __float2bfloat16_rn(p1);
+      const __nv_bfloat16 l0 = __float2bfloat16_rn(p0 - __bfloat162float(h0));
+      const __nv_bfloat16 l1 = __float2bfloat16_rn(p1 - __bfloat162float(h1));
+      h[j] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+      l[j] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+    }
+    hi[i] = make_uint4(h[0], h[1], h[2], h[3]);
+    lo[i] = make_uint4(l[0], l[1], l[2], l[3]);
+  }
+  pdl_trigger();
+}
+
+}  // namespace
+
+cudaError_t launch_split_router_weight(const void* w_router, const void* norm_w, int E, int d, void* hi, void* lo,
+                                       cudaStream_t stream) {
+  const int dv = d / 8;
+  const int n = E * dv;
+  int blocks = (n + 255) / 256;
+  if (blocks > 4 * sm_count()) blocks = 4 * sm_count();
+  return launch_pdl(split_router_weight_kernel, dim3(blocks), dim3(256), 0, stream,
+                    static_cast<const uint4*>(w_router), static_cast<const uint4*>(norm_w), E, dv,
+                    static_cast<uint4*>(hi), static_cast<uint4*>(lo));
 }
 
 }  // namespace moe

@@ -107,6 +107,35 @@ def make_inputs(wl: Workload, device="cpu", seed: int = 0) -> Inputs:
     return Inputs(wl, x, w_router, b, w_gate, w_up, w_down)
 
 
+@dataclass
+class OptionInputs:
+    """Tensors of the layer's options: the RMSNorm weight and the shared
+    experts' weights (None where unused)."""
+    norm_weight: torch.Tensor | None  # [d]
+    shared_gate: torch.Tensor | None  # [S, I, d]
+    shared_up: torch.Tensor | None  # [S, I, d]
+    shared_down: torch.Tensor | None  # [S, d, I]
+
+
+def make_option_inputs(wl: Workload, device="cpu", seed: int = 0, n_shared: int = 0,
+                       norm_weight: bool = False) -> OptionInputs:
+    """Draws, from a generator seeded with ``seed + 7919``, in this order: the
+    RMSNorm weight ``1 + 0.1 * N(0, 1)`` (when asked for), then the shared
+    experts' gate, up and down weights with the workload's weight std."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed + 7919)
+    dt = wl.torch_dtype
+    nw = None
+    if norm_weight:
+        nw = (1.0 + _randn((wl.d,), 0.1, gen, device, torch.float32)).to(dt)
+    sg = su = sd = None
+    if n_shared:
+        sg = _randn((n_shared, wl.I, wl.d), wl.w_std, gen, device, dt)
+        su = _randn((n_shared, wl.I, wl.d), wl.w_std, gen, device, dt)
+        sd = _randn((n_shared, wl.d, wl.I), wl.w_std, gen, device, dt)
+    return OptionInputs(nw, sg, su, sd)
+
+
 def make_tokens(wl: Workload, T: int, device="cpu", seed: int = 1) -> torch.Tensor:
     """A fresh batch of activations with the workload's distribution."""
     gen = torch.Generator(device=device)

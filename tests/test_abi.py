@@ -126,3 +126,66 @@ def test_selftest_argument_checks(lib):
     assert lib.moe_selftest_wait_timeout(None, 50_000_000, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_selftest_wait_timeout(ctypes.c_void_p(4096), 10, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_selftest_wait_timeout(ctypes.c_void_p(4096), 10**10, None) == B.MOE_ERR_INVALID_ARG
+
+
+def _opts(**kw):
+    o = B.moe_options()
+    o.struct_bytes = ctypes.sizeof(B.moe_options)
+    for k, v in kw.items():
+        setattr(o, k, v)
+    return o
+
+
+def test_options_struct_size_matches_the_library(lib):
+    o = _opts()
+    assert lib.moe_workspace_size_ex(64, 128, 4, 2, 128, B.MOE_BF16, ctypes.byref(o)) == \
+        lib.moe_workspace_size(64, 128, 4, 2, 128, B.MOE_BF16)
+    assert lib.moe_workspace_size_ex(64, 128, 4, 2, 128, B.MOE_BF16, None) == \
+        lib.moe_workspace_size(64, 128, 4, 2, 128, B.MOE_BF16)
+
+
+def test_options_grow_the_workspace(lib):
+    base = lib.moe_workspace_size(4096, 4096, 8, 2, 14336, B.MOE_BF16)
+    sh = _opts(n_shared=1, shared_gate=4096, shared_up=4096, shared_down=4096)
+    # one more copy of x (T*d bf16), T more hidden rows (bf16) and T more fp32 output rows
+    grow = lib.moe_workspace_size_ex(4096, 4096, 8, 2, 14336, B.MOE_BF16, ctypes.byref(sh)) - base
+    assert 4096 * (4096 * 2 + 14336 * 2 + 4096 * 4) <= grow < 4096 * (4096 * 2 + 14336 * 2 + 4096 * 4) + 4096
+    nm = _opts(norm_form=B.MOE_NORM_RMS, norm_eps=1e-5)
+    assert lib.moe_workspace_size_ex(4096, 4096, 8, 2, 14336, B.MOE_BF16, ctypes.byref(nm)) > base
+
+
+@pytest.mark.parametrize("field,value,msg", [
+    ("struct_bytes", 8, "struct_bytes"),
+    ("norm_form", 3, "norm_form"),
+    ("n_shared", 9, "n_shared"),
+    ("n_shared", -1, "n_shared"),
+    ("capacity_factor", -0.5, "capacity_factor"),
+    ("capacity_factor", float("nan"), "capacity_factor"),
+    ("capacity_factor", float("inf"), "capacity_factor"),
+])
+def test_invalid_options_are_rejected(lib, field, value, msg):
+    o = _opts(**{field: value})
+    assert lib.moe_workspace_size_ex(64, 128, 4, 2, 128, B.MOE_BF16, ctypes.byref(o)) == 0
+    assert msg in B.last_error_detail(lib)
+    fake = ctypes.c_void_p(4096)
+    st = lib.moe_forward_ex(fake, fake, None, fake, fake, fake, 64, 128, 4, 2, 128, 1, B.MOE_BF16, ctypes.byref(o),
+                            fake, fake, fake, None, None, fake, 1 << 30, None, None, None, 0)
+    assert st == B.MOE_ERR_INVALID_ARG
+
+
+def test_invalid_norm_eps_and_missing_shared_weights(lib):
+    fake = ctypes.c_void_p(4096)
+    for o in (_opts(norm_form=1, norm_eps=-1.0), _opts(norm_form=1, norm_eps=float("nan")),
+              _opts(n_shared=1), _opts(n_shared=1, shared_gate=4096, shared_up=4104, shared_down=4096),
+              _opts(norm_form=1, norm_weight=4100)):
+        st = lib.moe_forward_ex(fake, fake, None, fake, fake, fake, 64, 128, 4, 2, 128, 1, B.MOE_BF16,
+                                ctypes.byref(o), fake, fake, fake, None, None, fake, 1 << 30, None, None, None, 0)
+        assert st == B.MOE_ERR_INVALID_ARG, B.last_error_detail(lib)
+
+
+def test_forward_ex_event_count_is_checked(lib):
+    fake = ctypes.c_void_p(4096)
+    evs = (ctypes.c_void_p * 3)(4096, 4096, 4096)
+    st = lib.moe_forward_ex(fake, fake, None, fake, fake, fake, 64, 128, 4, 2, 128, 1, B.MOE_BF16, None,
+                            fake, fake, fake, None, None, fake, 1 << 30, None, None, evs, 3)
+    assert st == B.MOE_ERR_INVALID_ARG
