@@ -93,22 +93,47 @@ __device__ __forceinline__ void st_cluster_f32(const void* local_in_leader_layou
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
-// Insert (v, e) into the list of the kMaxTopK best, kept sorted best first.
+// Insert (v, e) into the list of the kMaxTopK best, kept sorted best first
+// (an element that ranks behind all of them leaves the list unchanged).
+// Branch-free: its position is the number of entries ranked ahead of it, and
+// every slot then selects its old value, the new one or its predecessor.
 __device__ __forceinline__ void topk_insert(float (&bv)[kMaxTopK], int (&be)[kMaxTopK], float v, int e) {
-  if (!ahead(v, e, bv[kMaxTopK - 1], be[kMaxTopK - 1])) return;
-  bv[kMaxTopK - 1] = v;
-  be[kMaxTopK - 1] = e;
+  int pos = 0;
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) pos += ahead(bv[j], be[j], v, e) ? 1 : 0;
 #pragma unroll
   for (int j = kMaxTopK - 1; j > 0; --j) {
-    if (ahead(bv[j], be[j], bv[j - 1], be[j - 1])) {
-      const float tv = bv[j];
-      bv[j] = bv[j - 1];
-      bv[j - 1] = tv;
-      const int te = be[j];
-      be[j] = be[j - 1];
-      be[j - 1] = te;
+    const bool shift = j > pos, here = j == pos;
+    bv[j] = shift ? bv[j - 1] : (here ? v : bv[j]);
+    be[j] = shift ? be[j - 1] : (here ? e : be[j]);
+  }
+  if (pos == 0) {
+    bv[0] = v;
+    be[0] = e;
+  }
+}
+
+// The top kMaxTopK of p[0..E) (row of shared memory) in two independent
+// insertion chains (even and odd experts), merged at the end.
+__device__ __forceinline__ void topk_of_row(const float* p, int E, float (&bv)[kMaxTopK], int (&be)[kMaxTopK]) {
+  float bv1[kMaxTopK];
+  int be1[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) {
+    bv1[j] = -INFINITY;
+    be1[j] = 0x7fffffff;
+  }
+#pragma unroll 1
+  for (int e = 0; e < E; e += 2) {
+    const float p0 = p[e];
+    topk_insert(bv, be, (p0 != p0) ? -INFINITY : p0, e);
+    if (e + 1 < E) {
+      const float p1 = p[e + 1];
+      topk_insert(bv1, be1, (p1 != p1) ? -INFINITY : p1, e + 1);
     }
   }
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) topk_insert(bv, be, bv1[j], be1[j]);
 }
 
 template <int kE>  // E <= kE: logits in registers; kE == 0: E > kRegE, logits in shared memory
@@ -135,6 +160,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   int* s_idx = reinterpret_cast<int*>(s_tmem + 4);  // [128][kMaxTopK]
   int* s_wcnt = s_idx + kRB * kMaxTopK;              // [4][E] per-warp counts, then exclusive prefix
   float* s_z = reinterpret_cast<float*>(s_wcnt + 4 * E);  // [4] per-warp sums of logsumexp^2
+  float* s_bias = s_z + 4;                                 // [E] router bias (leading CTA)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = S > 1 ? cta_rank_in_cluster() : 0u;
@@ -335,6 +361,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       be[j] = 0x7fffffff;
     }
     bool finite = true;
+    if (br) {  // the bias once per block, then read from shared memory
+      for (int e = r; e < E; e += kRB) s_bias[e] = br[e];
+      epi_bar();
+    }
     // RMSNorm scale of this token (1 without the norm)
     float rn = 1.0f;
     if (norm_form) {
@@ -358,7 +388,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int e = 0; e < kL; ++e)
         if (e < E) {
           if (norm_form) lg[e] *= rn;
-          if (br) lg[e] += br[e];
+          if (br) lg[e] += s_bias[e];
           finite = finite && isfinite(lg[e]);
           m = fmaxf(m, lg[e]);
         }
@@ -376,14 +406,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (e < E) {
           const float p = lg[e] * inv_s;
           s_p[r * ld + e] = valid ? p : 0.f;
-          topk_insert(bv, be, (p != p) ? -INFINITY : p, e);
+          if (kE <= 16) topk_insert(bv, be, (p != p) ? -INFINITY : p, e);
         }
+      // more than 16 experts: a rolled loop over the stored probabilities
+      // (E unrolled copies of the insertion would overflow the instruction
+      // cache)
+      if (kE > 16) topk_of_row(s_p + r * ld, E, bv, be);
     } else {
       float m = -INFINITY;
       for (int e = 0; e < E; ++e) {
         float l = s_p[r * ld + e];
         if (norm_form) l *= rn;
-        if (br) l += br[e];
+        if (br) l += s_bias[e];
         finite = finite && isfinite(l);
         m = fmaxf(m, l);
         s_p[r * ld + e] = l;
@@ -399,8 +433,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int e = 0; e < E; ++e) {
         const float p = s_p[r * ld + e] * inv_s;
         s_p[r * ld + e] = valid ? p : 0.f;
-        topk_insert(bv, be, (p != p) ? -INFINITY : p, e);
       }
+      topk_of_row(s_p + r * ld, E, bv, be);
     }
     if (valid && !finite) atomicOr(status, MOE_DEV_NONFINITE);
     if (blk_z) {  // this warp's sum of logsumexp^2 (a fixed shuffle tree)
