@@ -217,14 +217,18 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(
   }
 }
 
-// One CTA of 1024 threads. Thread (e, slice) reduces a contiguous range of
-// router blocks for expert e; slices are then scanned in order, so every
-// result is deterministic. With a capacity (cap >= 0) an expert keeps
-// min(count, cap) rows: offsets and the GEMM tile prefix cover the kept rows
-// only, and a row computed past its expert's kept count is a dropped slot.
-// The shared experts follow the routed experts in the tile prefix, T rows
-// each. Warp 1 sums the per-block z-loss partials in fp64 while thread 0
-// walks the experts.
+// One CTA of 1024 threads. Thread (slice, e) sums the counts and
+// probability sums of a contiguous range of router blocks for expert e (the
+// loads of neighbouring threads are neighbouring experts of one block, so they
+// coalesce). One warp per expert then scans its slice sums with shuffles;
+// warp 0 scans the expert totals (kept counts under a capacity: an expert
+// keeps min(count, cap) rows, and a row computed past that is a dropped slot)
+// into the offsets and the tile schedule, the shared experts following the
+// routed ones with T rows each, and the balance statistic; warp 1 sums the
+// per-block z-loss partials. Finally every thread walks its slice once more,
+// writing each block's base row. Every sum runs in a fixed order (fp64 for
+// the probabilities, the statistic and the z-loss), so the results are
+// deterministic.
 __global__ void __launch_bounds__(1024) route_scan_kernel(int nb, int T, int E, int k, int cap, int n_shared,
                                                           int32_t* __restrict__ blk_cnt,
                                                           const float* __restrict__ blk_psum,
@@ -232,13 +236,14 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int nb, int T, int E, 
                                                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                                           int32_t* __restrict__ mtile, float* __restrict__ aux,
                                                           float* __restrict__ zloss, int32_t* __restrict__ dropped) {
-  __shared__ int s_cnt[1024];
-  __shared__ double s_ps[1024];
+  __shared__ int s_cnt[1024];      // [slice][E] slice sums, then exclusive slice prefixes
+  __shared__ double s_ps[1024];    // [slice][E] probability slice sums
   __shared__ int s_tot[kMaxExperts];
   __shared__ double s_ptot[kMaxExperts];
   __shared__ int s_off[kMaxExperts + 1];
-  const int S = max(1, (int)blockDim.x / E);
-  const int tid = threadIdx.x;
+  const unsigned full = 0xffffffffu;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+  const int S = max(1, min((int)blockDim.x / E, nb));  // slices
   const int e = tid % E, sl = tid / E;
   const bool active = sl < S;
   const int chunk = (nb + S - 1) / S;
@@ -247,7 +252,6 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int nb, int T, int E, 
   if (active) {
     int c = 0;
     double ps = 0.0;
-#pragma unroll 8
     for (int b = b0; b < b1; ++b) {
       c += blk_cnt[(size_t)b * E + e];
       ps += (double)blk_psum[(size_t)b * E + e];
@@ -256,54 +260,88 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int nb, int T, int E, 
     s_ps[sl * E + e] = ps;
   }
   __syncthreads();
-  if (tid < E) {
-    int run = 0;
-    double p = 0.0;
-    for (int s2 = 0; s2 < S; ++s2) {
-      const int v = s_cnt[s2 * E + tid];
-      s_cnt[s2 * E + tid] = run;
-      run += v;
-      p += s_ps[s2 * E + tid];
-    }
-    s_tot[tid] = run;
-    s_ptot[tid] = p;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int off = 0, mt = 0, drop = 0;
-    double a = 0.0;
-    for (int ee = 0; ee < E; ++ee) {
-      const int tot = s_tot[ee];
-      const int kept = cap >= 0 ? min(tot, cap) : tot;
-      s_off[ee] = off;
-      offsets[ee] = off;
-      mtile[ee] = mt;
-      if (counts) counts[ee] = tot;
-      a += ((double)tot / ((double)T * (double)k)) * (s_ptot[ee] / (double)T);
-      off += kept;
-      drop += tot - kept;
-      mt += (kept + kTileM - 1) / kTileM;
-    }
-    offsets[E] = off;
-    s_off[E] = off;
-    mtile[E] = mt;
-    for (int s2 = 0; s2 < n_shared; ++s2) {
-      mt += (T + kTileM - 1) / kTileM;
-      mtile[E + 1 + s2] = mt;
-    }
-    if (aux) *aux = (float)((double)E * a);
-    if (dropped) *dropped = drop;
-  }
-  if (zloss && tid >= 32 && tid < 64) {
-    const int ln = tid - 32;
-    double z = 0.0;
-    for (int b = ln; b < nb; b += 32) z += (double)blk_z[b];
+  for (int ee = warp; ee < E; ee += nw) {  // one warp per expert: scan over the slices
+    int carry = 0;
+    double ps = 0.0;
+    for (int s0 = 0; s0 < S; s0 += 32) {
+      const int s1 = s0 + lane;
+      const int c = s1 < S ? s_cnt[s1 * E + ee] : 0;
+      double p = s1 < S ? s_ps[s1 * E + ee] : 0.0;
+      int incl = c;
 #pragma unroll
-    for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    if (ln == 0) *zloss = (float)(z / (double)T);
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(full, incl, o);
+        if (lane >= o) incl += n;
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) p += __shfl_xor_sync(full, p, o);
+      if (s1 < S) s_cnt[s1 * E + ee] = carry + incl - c;
+      carry += __shfl_sync(full, incl, 31);
+      ps += p;
+    }
+    if (lane == 0) {
+      s_tot[ee] = carry;
+      s_ptot[ee] = ps;
+    }
   }
   __syncthreads();
-  if (active) {
+  if (warp == 0) {
+    int run = 0, mt = 0, drop = 0;
+    double a = 0.0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int ee = e0 + lane;
+      const int tot = ee < E ? s_tot[ee] : 0;
+      const int kept = cap >= 0 ? min(tot, cap) : tot;
+      const int tiles = (kept + kTileM - 1) / kTileM;
+      int ik = kept, it = tiles;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n1 = __shfl_up_sync(full, ik, o), n2 = __shfl_up_sync(full, it, o);
+        if (lane >= o) {
+          ik += n1;
+          it += n2;
+        }
+      }
+      double ae = ee < E ? ((double)tot / ((double)T * (double)k)) * (s_ptot[ee] / (double)T) : 0.0;
+      int dr = tot - kept;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        ae += __shfl_xor_sync(full, ae, o);
+        dr += __shfl_xor_sync(full, dr, o);
+      }
+      if (ee < E) {
+        const int off = run + ik - kept;
+        offsets[ee] = off;
+        s_off[ee] = off;
+        mtile[ee] = mt + it - tiles;
+        if (counts) counts[ee] = tot;
+      }
+      run += __shfl_sync(full, ik, 31);
+      mt += __shfl_sync(full, it, 31);
+      a += ae;
+      drop += dr;
+    }
+    if (lane == 0) {
+      offsets[E] = run;
+      s_off[E] = run;
+      mtile[E] = mt;
+      for (int s2 = 0; s2 < n_shared; ++s2) {
+        mt += (T + kTileM - 1) / kTileM;
+        mtile[E + 1 + s2] = mt;
+      }
+      if (aux) *aux = (float)((double)E * a);
+      if (dropped) *dropped = drop;
+    }
+  }
+  if (zloss && warp == 1) {
+    double z = 0.0;
+    for (int b = lane; b < nb; b += 32) z += (double)blk_z[b];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(full, z, o);
+    if (lane == 0) *zloss = (float)(z / (double)T);
+  }
+  __syncthreads();
+  if (active) {  // base row of every block: expert offset + slice prefix + blocks before it in the slice
     int run = s_off[e] + s_cnt[sl * E + e];
     for (int b = b0; b < b1; ++b) {
       const int v = blk_cnt[(size_t)b * E + e];

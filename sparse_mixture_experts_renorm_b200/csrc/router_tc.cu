@@ -36,7 +36,8 @@ namespace moe {
 namespace {
 
 constexpr int kRB = kRouterTokensTc;  // 128 tokens per block
-constexpr int kRegE = 64;             // up to this many experts a token's logits stay in registers
+constexpr int kRegE = 16;             // up to this many experts a token's logits stay in registers
+constexpr int kSplitE = 64;           // up to this many experts the K loop may be split over a cluster
 
 struct RouterCfg {
   int npad;         // UMMA N
@@ -60,7 +61,7 @@ RouterCfg router_cfg(int T, int d, int E, bool norm, bool split, int num_sms) {
   // split K only while the grid leaves SMs idle, the partial logits stay
   // small, and each CTA keeps at least two k-blocks
   c.S = 1;
-  if (E <= kRegE)
+  if (E <= kSplitE)
     while (c.S < 8 && nb * c.S * 2 <= num_sms && (c.S * 2 - 1) * per_cta <= 64 * 1024 && KB / (c.S * 2) >= 2)
       c.S *= 2;
   c.part_bytes = (c.S - 1) * per_cta;
@@ -113,30 +114,44 @@ __device__ __forceinline__ void topk_insert(float (&bv)[kMaxTopK], int (&be)[kMa
   }
 }
 
-// The top kMaxTopK of p[0..E) (row of shared memory) in two independent
-// insertion chains (even and odd experts), merged at the end.
+// The top kMaxTopK of p[0..E) (a row in shared memory): four independent
+// insertion chains over the experts e mod 4, merged at the end.
 __device__ __forceinline__ void topk_of_row(const float* p, int E, float (&bv)[kMaxTopK], int (&be)[kMaxTopK]) {
-  float bv1[kMaxTopK];
-  int be1[kMaxTopK];
+  float cv[3][kMaxTopK];
+  int ce[3][kMaxTopK];
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) {
-    bv1[j] = -INFINITY;
-    be1[j] = 0x7fffffff;
+  for (int c = 0; c < 3; ++c)
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      cv[c][j] = -INFINITY;
+      ce[c][j] = 0x7fffffff;
+    }
+  auto val = [&](int e) {
+    const float x = p[e];
+    return (x != x) ? -INFINITY : x;
+  };
+  int e = 0;
+#pragma unroll 1
+  for (; e + 4 <= E; e += 4) {
+    const float p0 = val(e), p1 = val(e + 1), p2 = val(e + 2), p3 = val(e + 3);
+    topk_insert(bv, be, p0, e);
+    topk_insert(cv[0], ce[0], p1, e + 1);
+    topk_insert(cv[1], ce[1], p2, e + 2);
+    topk_insert(cv[2], ce[2], p3, e + 3);
   }
 #pragma unroll 1
-  for (int e = 0; e < E; e += 2) {
-    const float p0 = p[e];
-    topk_insert(bv, be, (p0 != p0) ? -INFINITY : p0, e);
-    if (e + 1 < E) {
-      const float p1 = p[e + 1];
-      topk_insert(bv1, be1, (p1 != p1) ? -INFINITY : p1, e + 1);
-    }
-  }
+  for (; e < E; ++e) topk_insert(bv, be, val(e), e);
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) topk_insert(bv, be, bv1[j], be1[j]);
+  for (int c = 0; c < 3; ++c)
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) topk_insert(bv, be, cv[c][j], ce[c][j]);
 }
 
-template <int kE>  // E <= kE: logits in registers; kE == 0: E > kRegE, logits in shared memory
+// E <= kE: logits in registers (fully unrolled code); kE == 0: E > kRegE,
+// logits in shared memory and rolled loops (code executed once per block must
+// stay small: unrolled per-expert code for large E thrashes the instruction
+// cache)
+template <int kE>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const __grid_constant__ CUtensorMap tmW2, const float* __restrict__ br, int T, int d, int E,
@@ -336,9 +351,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     if (S > 1 && rank > 0) {  // this CTA's share of the K loop goes to the leader
       float* dst = part + ((size_t)(rank - 1) * kRB + r) * E;
+      if (kE > 0) {
 #pragma unroll
-      for (int e = 0; e < kL; ++e)
-        if (e < E) st_cluster_f32(dst + e, 0, lg[e]);
+        for (int e = 0; e < kL; ++e)
+          if (e < E) st_cluster_f32(dst + e, 0, lg[e]);
+      } else {
+        for (int e = 0; e < E; ++e) st_cluster_f32(dst + e, 0, s_p[r * (E + 1) + e]);
+      }
       if (norm_form) st_cluster_f32(part_ss + (size_t)(rank - 1) * kRB + r, 0, ss);
     }
   }
@@ -383,22 +402,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int e = 0; e < kL; ++e)
           if (e < E) lg[e] += src[e];
       }
-      float m = -INFINITY;
+      // four independent chains (experts e mod 4) for the maximum and the sum
+      float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int e = 0; e < kL; ++e)
         if (e < E) {
           if (norm_form) lg[e] *= rn;
           if (br) lg[e] += s_bias[e];
           finite = finite && isfinite(lg[e]);
-          m = fmaxf(m, lg[e]);
+          mc[e & 3] = fmaxf(mc[e & 3], lg[e]);
         }
-      float s = 0.f;
+      const float m = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
+      float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int e = 0; e < kL; ++e)
         if (e < E) {
           lg[e] = __expf(lg[e] - m);
-          s += lg[e];
+          sc[e & 3] += lg[e];
         }
+      const float s = (sc[0] + sc[1]) + (sc[2] + sc[3]);
       lse = m + logf(s);
       const float inv_s = 1.0f / s;
 #pragma unroll
@@ -406,35 +428,54 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (e < E) {
           const float p = lg[e] * inv_s;
           s_p[r * ld + e] = valid ? p : 0.f;
-          if (kE <= 16) topk_insert(bv, be, (p != p) ? -INFINITY : p, e);
+          topk_insert(bv, be, (p != p) ? -INFINITY : p, e);
         }
-      // more than 16 experts: a rolled loop over the stored probabilities
-      // (E unrolled copies of the insertion would overflow the instruction
-      // cache)
-      if (kE > 16) topk_of_row(s_p + r * ld, E, bv, be);
     } else {
-      float m = -INFINITY;
-      for (int e = 0; e < E; ++e) {
-        float l = s_p[r * ld + e];
+      // rolled loops over this token's row of s_p, four experts per trip
+      // (independent chains for the maximum and the sum)
+      float* pr = s_p + r * ld;
+      auto logit = [&](int e) {
+        float l = pr[e];
+        for (int s2 = 0; s2 < S - 1; ++s2) l += part[((size_t)s2 * kRB + r) * E + e];
         if (norm_form) l *= rn;
         if (br) l += s_bias[e];
         finite = finite && isfinite(l);
-        m = fmaxf(m, l);
-        s_p[r * ld + e] = l;
+        pr[e] = l;
+        return l;
+      };
+      float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+      int e4 = 0;
+#pragma unroll 1
+      for (; e4 + 4 <= E; e4 += 4) {
+        m0 = fmaxf(m0, logit(e4));
+        m1 = fmaxf(m1, logit(e4 + 1));
+        m2 = fmaxf(m2, logit(e4 + 2));
+        m3 = fmaxf(m3, logit(e4 + 3));
       }
-      float s = 0.f;
-      for (int e = 0; e < E; ++e) {
-        const float ex = __expf(s_p[r * ld + e] - m);
-        s_p[r * ld + e] = ex;
-        s += ex;
+#pragma unroll 1
+      for (int e = e4; e < E; ++e) m0 = fmaxf(m0, logit(e));
+      const float m = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+      auto expo = [&](int e) {
+        const float ex = __expf(pr[e] - m);
+        pr[e] = ex;
+        return ex;
+      };
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll 1
+      for (int e = 0; e + 4 <= E; e += 4) {
+        s0 += expo(e);
+        s1 += expo(e + 1);
+        s2 += expo(e + 2);
+        s3 += expo(e + 3);
       }
+#pragma unroll 1
+      for (int e = e4; e < E; ++e) s0 += expo(e);
+      const float s = (s0 + s1) + (s2 + s3);
       lse = m + logf(s);
       const float inv_s = 1.0f / s;
-      for (int e = 0; e < E; ++e) {
-        const float p = s_p[r * ld + e] * inv_s;
-        s_p[r * ld + e] = valid ? p : 0.f;
-      }
-      topk_of_row(s_p + r * ld, E, bv, be);
+#pragma unroll 4
+      for (int e = 0; e < E; ++e) pr[e] = valid ? pr[e] * inv_s : 0.f;
+      topk_of_row(pr, E, bv, be);
     }
     if (valid && !finite) atomicOr(status, MOE_DEV_NONFINITE);
     if (blk_z) {  // this warp's sum of logsumexp^2 (a fixed shuffle tree)
@@ -497,9 +538,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         run += c;
       }
       blk_cnt[(size_t)blk * E + e] = run;
-      float ps = 0.f;
-      for (int rr = 0; rr < kRB; ++rr) ps += s_p[rr * ld + e];
-      blk_psum[(size_t)blk * E + e] = ps;
+      float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;  // four chains over the block's tokens
+#pragma unroll 4
+      for (int rr = 0; rr < kRB; rr += 4) {
+        ps0 += s_p[rr * ld + e];
+        ps1 += s_p[(rr + 1) * ld + e];
+        ps2 += s_p[(rr + 2) * ld + e];
+        ps3 += s_p[(rr + 3) * ld + e];
+      }
+      blk_psum[(size_t)blk * E + e] = (ps0 + ps1) + (ps2 + ps3);
     }
     if (blk_z && r == 0) blk_z[blk] = ((s_z[0] + s_z[1]) + s_z[2]) + s_z[3];
     epi_bar();
@@ -544,8 +591,7 @@ cudaError_t launch_router_tc(const void* x, const void* w_router, const float* b
       !make_tmap_bf16_2d(&tmW, split ? norm.w_hi : w_router, (uint64_t)E, (uint64_t)d, (uint32_t)c.npad) ||
       !make_tmap_bf16_2d(&tmW2, split ? norm.w_lo : w_router, (uint64_t)E, (uint64_t)d, (uint32_t)c.npad))
     return cudaErrorInvalidValue;
-  auto kern = E <= 16 ? router_tc_kernel<16> : E <= 32 ? router_tc_kernel<32> : E <= kRegE ? router_tc_kernel<kRegE>
-                                                                                           : router_tc_kernel<0>;
+  auto kern = E <= kRegE ? router_tc_kernel<kRegE> : router_tc_kernel<0>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, c.smem_bytes);
   if (err != cudaSuccess) return err;
   const int nb = (T + kRB - 1) / kRB;
