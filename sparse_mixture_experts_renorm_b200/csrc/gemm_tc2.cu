@@ -11,16 +11,17 @@
 // compute on neighbouring rows (or TMA zero fill) and are masked at the store.
 //
 // A cluster of two CTAs on two SMs owns one tile at a time. Each CTA stages
-// its own 128 rows of A and one half of the 256 B rows (mode 0: CTA 0 the 128
-// gate rows, CTA 1 the 128 up rows of the same hidden units; mode 1: 128
-// W_down rows each) through a 6-stage TMA ring, both signalling the leading
-// CTA's barrier. One thread of the leading CTA issues 256x256x16 UMMAs that
-// read A and B from both CTAs' shared memory and write each CTA's 128 rows of
-// the fp32 accumulator into that CTA's TMEM (double-buffered, 2 x 256
-// columns); commits are multicast to both CTAs. Each CTA's 4 epilogue warps
-// drain their own TMEM lanes (SwiGLU + bf16 in mode 0, fp32 in mode 1) and
-// release the accumulator to the leader. Per UMMA FLOP this moves a third
-// fewer bytes from L2 to shared memory than one CTA per 128 x 256 tile.
+// its own 128 rows of A and one half of the 256 B rows (mode 0: the 64 gate
+// rows and the 64 up rows of its 64 hidden units; mode 1: 128 W_down rows)
+// through a 5-stage TMA ring, both signalling the leading CTA's barrier. One
+// thread of the leading CTA issues 256xNx16 UMMAs that read A and B from both
+// CTAs' shared memory and write each CTA's 128 rows of the fp32 accumulator
+// into that CTA's TMEM (double-buffered, 2 x 256 columns); commits are
+// multicast to both CTAs. Each CTA's 8 epilogue warps, two per TMEM lane
+// quarter taking alternate 32-token chunks, drain their TMEM lanes (SwiGLU +
+// bf16 in mode 0, fp32 in mode 1) and release the accumulator to the leader.
+// Per UMMA FLOP this moves a third fewer bytes from L2 to shared memory than
+// one CTA per 128 x 256 tile.
 //
 // Persistent: clusters walk a device-side tile list built from the routing
 // counts (experts in order; n-tile outer, m-tile inner inside an expert, so
@@ -33,16 +34,34 @@
 namespace moe {
 namespace {
 
-constexpr int kStages2 = 6;
 constexpr int kHalfBytes = 128 * kBK * 2;          // 16 KB: 128 rows x 64 bf16
 constexpr int kStage2Bytes = 2 * kHalfBytes;       // A half + B half per CTA
 constexpr int kSmallRows = 16;                     // B box for tiles of <= 32 tokens
-// epilogue staging: gate and up halves of a 32-token chunk (mode 0, 2 x 64 x 33
-// fp32) or one 32 x 32 fp32 transpose tile per epilogue warp (mode 1, 4 x 32 x 36)
-constexpr int kEpiBytes = 4 * 32 * 36 * 4 > 2 * 64 * 33 * 4 ? 4 * 32 * 36 * 4 : 2 * 64 * 33 * 4;
-constexpr int kGemm2SmemBytes = kStages2 * kStage2Bytes + kEpiBytes + 1024 + 4096;
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Two configurations of the kernel. "Wide" tiles (many tokens per expert):
+// the epilogue is the long pole, so warps 2-9 drain the accumulator, two per
+// TMEM lane quarter taking alternate 32-token chunks, with a 5-stage ring.
+// "Narrow" tiles (decode-sized batches that stream the weights from HBM): a
+// deeper 6-stage ring keeps more bytes in flight and warps 2-5 drain it.
+// Epilogue staging: per group of four epilogue warps the gate and up rows of
+// a 32-token chunk (mode 0, 2 x 64 x 33 fp32), or one 32 x 32 fp32 transpose
+// tile per epilogue warp (mode 1, 32 x 36).
+template <int kSt, int kEw>
+struct Gemm2Cfg {
+  static constexpr int kStages = kSt;
+  static constexpr int kEpiWarps = kEw;
+  static constexpr int kThreads = 64 + 32 * kEw;
+  static constexpr int kEpiBytesM0 = (kEw / 4) * (2 * 64 * 33 * 4);
+  static constexpr int kEpiBytesM1 = kEw * 32 * 36 * 4;
+  static constexpr int kEpiBytes = kEpiBytesM1 > kEpiBytesM0 ? kEpiBytesM1 : kEpiBytesM0;
+  static constexpr int kSmemBytes = kSt * kStage2Bytes + kEpiBytes + 1024 + 4096;
+};
+using Gemm2Wide = Gemm2Cfg<5, 8>;
+using Gemm2Narrow = Gemm2Cfg<6, 4>;
+static_assert(Gemm2Wide::kSmemBytes <= 227 * 1024 && Gemm2Narrow::kSmemBytes <= 227 * 1024, "shared memory");
+
+// named barrier of one group of four epilogue warps (ids 1 and 2, 128 threads)
+__device__ __forceinline__ void epi_bar(int half) { asm volatile("bar.sync %0, 128;" ::"r"(1 + half) : "memory"); }
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -186,8 +205,8 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, int n_tiles, const in
 
 __device__ __forceinline__ float silu_f32(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
-template <int kMode>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+template <int kMode, int kSt, int kEw>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
     grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                             const __grid_constant__ CUtensorMap tmS0, const __grid_constant__ CUtensorMap tmS1,
                             const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBs,
@@ -196,17 +215,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                             const int32_t* __restrict__ perm_tok,
                             const float* __restrict__ rgate, float* __restrict__ comb_out, int32_t* status,
                             uint64_t limit_ns) {
+  using Cfg = Gemm2Cfg<kSt, kEw>;
+  constexpr int kGroups = kEw / 4;  // groups of four epilogue warps (one per TMEM lane quarter each)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;                           // [stages][128 weight rows x 64]
-  uint8_t* sB = smem + kStages2 * kHalfBytes;   // [stages][<=128 token rows x 64]
-  float* sG = reinterpret_cast<float*>(smem + kStages2 * kStage2Bytes);  // [64][33] gate chunk (mode 0)
-  float* sU = sG + 64 * 33;                                              // [64][33] up chunk (mode 0)
-  float* sY = sG;                                                        // [4][32][36] (mode 1)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages2 * kStage2Bytes + kEpiBytes);
+  uint8_t* sB = smem + kSt * kHalfBytes;   // [stages][<=128 token rows x 64]
+  float* sEpi = reinterpret_cast<float*>(smem + kSt * kStage2Bytes);
+  float* sY = sEpi;  // [8][32][36] (mode 1)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSt * kStage2Bytes + Cfg::kEpiBytes);
   uint64_t* full = bars;                 // leader: A+B bytes of both CTAs
-  uint64_t* empty = bars + kStages2;     // both: stage consumed by the pair's UMMAs
-  uint64_t* tfull = bars + 2 * kStages2; // both: accumulator ready
+  uint64_t* empty = bars + kSt;     // both: stage consumed by the pair's UMMAs
+  uint64_t* tfull = bars + 2 * kSt; // both: accumulator ready
   uint64_t* tempty = tfull + 2;          // leader: 256 epilogue arrivals
   uint64_t* done = tempty + 2;           // leader: every UMMA completed
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(done + 1);
@@ -225,13 +245,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const int KB = K / kBK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages2; ++s) {
+    for (int s = 0; s < kSt; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 256);
+      mbar_init(&tempty[b], 2 * 32 * kEw);
     }
     mbar_init(done, 1);
     *s_abort = 0;
@@ -298,7 +318,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           }
           tma_load_2d_pair(sB + stage * kHalfBytes, small ? &tmBs : &tmB, fbar, kb * kBK, brow);
           ++issued;
-          if (++stage == kStages2) {
+          if (++stage == kSt) {
             stage = 0;
             phase ^= 1u;
           }
@@ -307,10 +327,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       // Loads land on the leader's barriers: the leader waits for the last
       // phase of each stage it armed (these cover both CTAs' bytes).
       if (leader) {
-        const int n = issued < kStages2 ? issued : kStages2;
+        const int n = issued < kSt ? issued : kSt;
         for (int i = 0; i < n; ++i) {
           if (stage == 0) {
-            stage = kStages2;
+            stage = kSt;
             phase ^= 1u;
           }
           --stage;
@@ -353,7 +373,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                              bdesc + static_cast<uint64_t>(kk * 2), idesc, (kb > 0 || kk >= nacc) ? 1u : 0u);
           }
           tc_commit_pair_both(&empty[stage]);
-          if (++stage == kStages2) {
+          if (++stage == kSt) {
             stage = 0;
             phase ^= 1u;
           }
@@ -394,19 +414,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         // CTA's 64 hidden units. Per 32-token chunk both halves go to shared
         // memory; then every thread finishes 16 (token, unit) pairs and
         // writes them as two 16-byte vectors of H.
+        const int half = (warp - 2) >> 2;  // which group of epilogue warps
+        float* sG = sEpi + half * (2 * 64 * 33);  // [64][33] gate chunk
+        float* sU = sG + 64 * 33;                 // [64][33] up chunk
         const int j = (q & 1) * 32 + lane;
         float* sdst = (q < 2 ? sG : sU) + j * 33;
-        const int et = threadIdx.x - 64;  // 0..127
+        const int et = ((warp - 2) & 3) * 32 + lane;  // 0..127 within the group
         const int tt = et >> 2;           // token of the chunk
         const int ug = (et & 3) * 16;     // first of its 16 units
         const int hid0 = tc.n * 128 + (int)rank * 64;
 #pragma unroll 1
-        for (int c = 0; c < nchunks; ++c) {
+        for (int c = half; c < nchunks; c += kGroups) {
           uint32_t v[32];
           ld_chunk_sum(tbase + c * 32, nacc, acc_stride, v);
 #pragma unroll
           for (int t = 0; t < 32; ++t) sdst[t] = __uint_as_float(v[t]);
-          epi_bar();
+          epi_bar(half);
           uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -415,7 +438,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             const float h1 = silu_f32(sG[(u0 + 1) * 33 + tt]) * sU[(u0 + 1) * 33 + tt];
             pk[i] = pack_bf16x2(h0, h1);
           }
-          epi_bar();
+          epi_bar(half);
           const int tok = c * 32 + tt;
           if (tok < ntok && hid0 < N) {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + (row0 + tok) * N + hid0 + ug);
@@ -431,7 +454,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         float* tw = sY + (warp - 2) * (32 * 36);
         const int vr = lane >> 3, vc = (lane & 7) * 4;
 #pragma unroll 1
-        for (int c = 0; c < nchunks; ++c) {
+        for (int c = (warp - 2) >> 2; c < nchunks; c += kGroups) {
           uint32_t v[32];
           ld_chunk_sum(tbase + c * 32, nacc, acc_stride, v);
 #pragma unroll
@@ -480,15 +503,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-int max_active_pairs(const void* kern, int smem) {
+template <class Cfg>
+int max_active_pairs(const void* kern) {
   static int cache[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   if (cache[dev] == 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
-    cfg.blockDim = dim3(kGemmThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
+    cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeClusterDimension;
     attr.val.clusterDim.x = 2;
@@ -503,23 +527,41 @@ int max_active_pairs(const void* kern, int smem) {
   return cache[dev];
 }
 
+template <int kMode, class Cfg>
+cudaError_t launch_tc2_cfg(const CUtensorMap& tmA0, const CUtensorMap& tmA1, const CUtensorMap& tmS0,
+                           const CUtensorMap& tmS1, const CUtensorMap& tmB, const CUtensorMap& tmBs,
+                           const int32_t* offsets, const int32_t* mtile256, int R_rows, int E, const SharedGroups& sh,
+                           int N, int K, void* out, const int32_t* perm_tok, const float* rgate, float* comb_out,
+                           int32_t* status, cudaStream_t stream) {
+  auto kern = grouped_gemm_tc2_kernel<kMode, Cfg::kStages, Cfg::kEpiWarps>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+  if (err != cudaSuccess) return err;
+  const int pairs = max_active_pairs<Cfg>(reinterpret_cast<const void*>(kern));
+  if (pairs <= 0) return cudaErrorInvalidConfiguration;
+  const int n_wb = kMode == 0 ? (N + 127) / 128 : (N + 255) / 256;
+  const long long max_tiles = (long long)(R_rows / 256 + E + sh.n) * n_wb;
+  const int clusters = (int)(max_tiles < pairs ? max_tiles : pairs);
+  if (clusters <= 0) return cudaSuccess;
+  return launch_pdl(kern, dim3(2 * clusters), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, tmA0, tmA1, tmS0, tmS1,
+                    tmB, tmBs, offsets, mtile256, E, sh, N, K, out, perm_tok, rgate, comb_out, status, kWaitLimitNs);
+}
+
+// Decode-sized batches (fewer than 64 rows per group on average) take the
+// narrow configuration, everything else the wide one; the down projection
+// only with the combine folded in (its fp32 Y stores run better with fewer
+// epilogue warps and the deeper ring).
 template <int kMode>
 cudaError_t launch_tc2(const CUtensorMap& tmA0, const CUtensorMap& tmA1, const CUtensorMap& tmS0,
                        const CUtensorMap& tmS1, const CUtensorMap& tmB, const CUtensorMap& tmBs, const int32_t* offsets,
                        const int32_t* mtile256, int R_rows, int E, const SharedGroups& sh, int N, int K, void* out,
                        const int32_t* perm_tok, const float* rgate, float* comb_out, int32_t* status,
                        cudaStream_t stream) {
-  auto kern = grouped_gemm_tc2_kernel<kMode>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemm2SmemBytes);
-  if (err != cudaSuccess) return err;
-  const int pairs = max_active_pairs(reinterpret_cast<const void*>(kern), kGemm2SmemBytes);
-  if (pairs <= 0) return cudaErrorInvalidConfiguration;
-  const int n_wb = kMode == 0 ? (N + 127) / 128 : (N + 255) / 256;
-  const long long max_tiles = (long long)(R_rows / 256 + E + sh.n) * n_wb;
-  const int clusters = (int)(max_tiles < pairs ? max_tiles : pairs);
-  if (clusters <= 0) return cudaSuccess;
-  return launch_pdl(kern, dim3(2 * clusters), dim3(kGemmThreads), kGemm2SmemBytes, stream, tmA0, tmA1, tmS0, tmS1,
-                    tmB, tmBs, offsets, mtile256, E, sh, N, K, out, perm_tok, rgate, comb_out, status, kWaitLimitNs);
+  const bool wide = (long long)R_rows >= 64ll * (E + sh.n) && (kMode == 0 || comb_out != nullptr);
+  if (wide)
+    return launch_tc2_cfg<kMode, Gemm2Wide>(tmA0, tmA1, tmS0, tmS1, tmB, tmBs, offsets, mtile256, R_rows, E, sh, N, K,
+                                            out, perm_tok, rgate, comb_out, status, stream);
+  return launch_tc2_cfg<kMode, Gemm2Narrow>(tmA0, tmA1, tmS0, tmS1, tmB, tmBs, offsets, mtile256, R_rows, E, sh, N, K,
+                                            out, perm_tok, rgate, comb_out, status, stream);
 }
 
 }  // namespace
