@@ -428,8 +428,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (e < E) {
           const float p = lg[e] * inv_s;
           s_p[r * ld + e] = valid ? p : 0.f;
-          topk_insert(bv, be, (p != p) ? -INFINITY : p, e);
+          lg[e] = (p != p) ? -INFINITY : p;
         }
+      // k passes of an arg-max over the (at most kE) probabilities: a strict
+      // comparison in ascending expert order keeps the lower index on ties,
+      // and the first candidate is always taken, so every token gets k
+      // distinct experts even when some probabilities are -inf
+      uint32_t taken = 0;
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j) {
+        if (j < k) {
+          float best = -INFINITY;
+          int bi = -1;
+#pragma unroll
+          for (int e = 0; e < kL; ++e)
+            if (e < E && !((taken >> e) & 1u) && (bi < 0 || lg[e] > best)) {
+              best = lg[e];
+              bi = e;
+            }
+          taken |= 1u << bi;
+          bv[j] = best;
+          be[j] = bi;
+        }
+      }
     } else {
       // rolled loops over this token's row of s_p, four experts per trip
       // (independent chains for the maximum and the sum)
