@@ -35,30 +35,37 @@ namespace moe {
 namespace {
 
 constexpr int kHalfBytes = 128 * kBK * 2;          // 16 KB: 128 rows x 64 bf16
-constexpr int kStage2Bytes = 2 * kHalfBytes;       // A half + B half per CTA
 constexpr int kSmallRows = 16;                     // B box for tiles of <= 32 tokens
 
-// Two configurations of the kernel. "Wide" tiles (many tokens per expert):
+// Three configurations of the kernel. "Wide" tiles (many tokens per expert):
 // the epilogue is the long pole, so warps 2-9 drain the accumulator, two per
 // TMEM lane quarter taking alternate 32-token chunks, with a 5-stage ring.
 // "Narrow" tiles (decode-sized batches that stream the weights from HBM): a
 // deeper 6-stage ring keeps more bytes in flight and warps 2-5 drain it.
+// "Stream" (at most 32 tokens in the whole batch, so every tile's token rows
+// fit the 16-row box): the B slot shrinks to 2 KB and the ring to 11 stages
+// of 18 KB, nearly twice the weight bytes in flight of the narrow ring.
 // Epilogue staging: per group of four epilogue warps the gate and up rows of
 // a 32-token chunk (mode 0, 2 x 64 x 33 fp32), or one 32 x 32 fp32 transpose
 // tile per epilogue warp (mode 1, 32 x 36).
-template <int kSt, int kEw>
+template <int kSt, int kEw, int kBRows>
 struct Gemm2Cfg {
   static constexpr int kStages = kSt;
   static constexpr int kEpiWarps = kEw;
+  static constexpr int kBSlotRows = kBRows;            // token rows a stage holds per CTA
+  static constexpr int kBSlotBytes = kBRows * kBK * 2;
   static constexpr int kThreads = 64 + 32 * kEw;
   static constexpr int kEpiBytesM0 = (kEw / 4) * (2 * 64 * 33 * 4);
   static constexpr int kEpiBytesM1 = kEw * 32 * 36 * 4;
   static constexpr int kEpiBytes = kEpiBytesM1 > kEpiBytesM0 ? kEpiBytesM1 : kEpiBytesM0;
-  static constexpr int kSmemBytes = kSt * kStage2Bytes + kEpiBytes + 1024 + 4096;
+  static constexpr int kSmemBytes = kSt * (kHalfBytes + kBSlotBytes) + kEpiBytes + 1024 + 4096;
 };
-using Gemm2Wide = Gemm2Cfg<5, 8>;
-using Gemm2Narrow = Gemm2Cfg<6, 4>;
-static_assert(Gemm2Wide::kSmemBytes <= 227 * 1024 && Gemm2Narrow::kSmemBytes <= 227 * 1024, "shared memory");
+using Gemm2Wide = Gemm2Cfg<5, 8, 128>;
+using Gemm2Narrow = Gemm2Cfg<6, 4, 128>;
+using Gemm2Stream = Gemm2Cfg<11, 4, kSmallRows>;
+static_assert(Gemm2Wide::kSmemBytes <= 227 * 1024 && Gemm2Narrow::kSmemBytes <= 227 * 1024 &&
+                  Gemm2Stream::kSmemBytes <= 227 * 1024,
+              "shared memory");
 
 // named barrier of one group of four epilogue warps (ids 1 and 2, 128 threads)
 __device__ __forceinline__ void epi_bar(int half) { asm volatile("bar.sync %0, 128;" ::"r"(1 + half) : "memory"); }
@@ -205,7 +212,7 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, int n_tiles, const in
 
 __device__ __forceinline__ float silu_f32(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
-template <int kMode, int kSt, int kEw>
+template <int kMode, int kSt, int kEw, int kBRows>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
     grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                             const __grid_constant__ CUtensorMap tmS0, const __grid_constant__ CUtensorMap tmS1,
@@ -215,15 +222,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
                             const int32_t* __restrict__ perm_tok,
                             const float* __restrict__ rgate, float* __restrict__ comb_out, int32_t* status,
                             uint64_t limit_ns) {
-  using Cfg = Gemm2Cfg<kSt, kEw>;
+  using Cfg = Gemm2Cfg<kSt, kEw, kBRows>;
+  constexpr int kBSlot = Cfg::kBSlotBytes;
   constexpr int kGroups = kEw / 4;  // groups of four epilogue warps (one per TMEM lane quarter each)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;                           // [stages][128 weight rows x 64]
-  uint8_t* sB = smem + kSt * kHalfBytes;   // [stages][<=128 token rows x 64]
-  float* sEpi = reinterpret_cast<float*>(smem + kSt * kStage2Bytes);
+  uint8_t* sB = smem + kSt * kHalfBytes;   // [stages][<= kBRows token rows x 64]
+  float* sEpi = reinterpret_cast<float*>(smem + kSt * (kHalfBytes + kBSlot));
   float* sY = sEpi;  // [8][32][36] (mode 1)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSt * kStage2Bytes + Cfg::kEpiBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSt * (kHalfBytes + kBSlot) + Cfg::kEpiBytes);
   uint64_t* full = bars;                 // leader: A+B bytes of both CTAs
   uint64_t* empty = bars + kSt;     // both: stage consumed by the pair's UMMAs
   uint64_t* tfull = bars + 2 * kSt; // both: accumulator ready
@@ -296,6 +304,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
         const int ntok = min(256, gr.cnt - tc.m * 256);
         const int half = ((ntok + 15) & ~15) >> 1;  // token rows of B held by each CTA
         const bool small = half <= kSmallRows;
+        if (!small && kBRows < 128) {  // the launcher guarantees this cannot happen
+          atomicOr(status, MOE_DEV_INTERNAL);
+          *s_abort = 1;
+          ok = false;
+          break;
+        }
         const int brow = gr.in0 + tc.m * 256 + (int)rank * half;
         const int arow =
             kMode == 0 ? gr.widx * N + tc.n * 128 + (int)rank * 64 : gr.widx * N + tc.n * 256 + (int)rank * 128;
@@ -316,7 +330,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
           } else {
             tma_load_2d_pair(sA + stage * kHalfBytes, mA0, fbar, kb * kBK, arow);
           }
-          tma_load_2d_pair(sB + stage * kHalfBytes, small ? &tmBs : &tmB, fbar, kb * kBK, brow);
+          tma_load_2d_pair(sB + stage * kBSlot, small ? &tmBs : &tmB, fbar, kb * kBK, brow);
           ++issued;
           if (++stage == kSt) {
             stage = 0;
@@ -365,7 +379,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
           }
           tc_fence_after();
           const uint64_t adesc = sw128_kmajor_desc(smem_u32(sA + stage * kHalfBytes));
-          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sB + stage * kHalfBytes));
+          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sB + stage * kBSlot));
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const int a = kk % nacc;
@@ -533,7 +547,7 @@ cudaError_t launch_tc2_cfg(const CUtensorMap& tmA0, const CUtensorMap& tmA1, con
                            const int32_t* offsets, const int32_t* mtile256, int R_rows, int E, const SharedGroups& sh,
                            int N, int K, void* out, const int32_t* perm_tok, const float* rgate, float* comb_out,
                            int32_t* status, cudaStream_t stream) {
-  auto kern = grouped_gemm_tc2_kernel<kMode, Cfg::kStages, Cfg::kEpiWarps>;
+  auto kern = grouped_gemm_tc2_kernel<kMode, Cfg::kStages, Cfg::kEpiWarps, Cfg::kBSlotRows>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (err != cudaSuccess) return err;
   const int pairs = max_active_pairs<Cfg>(reinterpret_cast<const void*>(kern));
@@ -546,17 +560,22 @@ cudaError_t launch_tc2_cfg(const CUtensorMap& tmA0, const CUtensorMap& tmA1, con
                     tmB, tmBs, offsets, mtile256, E, sh, N, K, out, perm_tok, rgate, comb_out, status, kWaitLimitNs);
 }
 
-// Decode-sized batches (fewer than 64 rows per group on average) take the
-// narrow configuration, everything else the wide one; the down projection
+// Batches whose every group has at most 32 rows (max_rows_per_group: T, the
+// most a routed expert or a shared expert can receive) take the stream
+// configuration; other decode-sized batches (fewer than 64 rows per group on
+// average) the narrow one, everything else the wide one; the down projection
 // only with the combine folded in (its fp32 Y stores run better with fewer
 // epilogue warps and the deeper ring).
 template <int kMode>
 cudaError_t launch_tc2(const CUtensorMap& tmA0, const CUtensorMap& tmA1, const CUtensorMap& tmS0,
                        const CUtensorMap& tmS1, const CUtensorMap& tmB, const CUtensorMap& tmBs, const int32_t* offsets,
-                       const int32_t* mtile256, int R_rows, int E, const SharedGroups& sh, int N, int K, void* out,
-                       const int32_t* perm_tok, const float* rgate, float* comb_out, int32_t* status,
-                       cudaStream_t stream) {
+                       const int32_t* mtile256, int R_rows, int max_rows_per_group, int E, const SharedGroups& sh,
+                       int N, int K, void* out, const int32_t* perm_tok, const float* rgate, float* comb_out,
+                       int32_t* status, cudaStream_t stream) {
   const bool wide = (long long)R_rows >= 64ll * (E + sh.n) && (kMode == 0 || comb_out != nullptr);
+  if (max_rows_per_group <= 2 * kSmallRows)
+    return launch_tc2_cfg<kMode, Gemm2Stream>(tmA0, tmA1, tmS0, tmS1, tmB, tmBs, offsets, mtile256, R_rows, E, sh, N,
+                                              K, out, perm_tok, rgate, comb_out, status, stream);
   if (wide)
     return launch_tc2_cfg<kMode, Gemm2Wide>(tmA0, tmA1, tmS0, tmS1, tmB, tmBs, offsets, mtile256, R_rows, E, sh, N, K,
                                             out, perm_tok, rgate, comb_out, status, stream);
@@ -571,8 +590,8 @@ cudaError_t launch_gemm_gateup_tc2(const CUtensorMap& tm_wg, const CUtensorMap& 
                                    const int32_t* offsets, const int32_t* mtile, int R_rows, int E,
                                    const SharedGroups& sh, int I, int d, void* h, int32_t* status,
                                    cudaStream_t stream) {
-  return launch_tc2<0>(tm_wg, tm_wu, tm_sg, tm_su, tm_xp, tm_xp_small, offsets, mtile, R_rows, E, sh, I, d, h, nullptr,
-                       nullptr, nullptr, status, stream);
+  return launch_tc2<0>(tm_wg, tm_wu, tm_sg, tm_su, tm_xp, tm_xp_small, offsets, mtile, R_rows, sh.rows, E, sh, I, d, h,
+                       nullptr, nullptr, nullptr, status, stream);
 }
 
 cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_wd, const CUtensorMap& tm_sd, const CUtensorMap& tm_h,
@@ -580,8 +599,8 @@ cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_wd, const CUtensorMap& tm
                                  int R_rows, int E, const SharedGroups& sh, int I, int d, float* y,
                                  const int32_t* perm_tok, const float* rgate, float* comb_out, int32_t* status,
                                  cudaStream_t stream) {
-  return launch_tc2<1>(tm_wd, tm_wd, tm_sd, tm_sd, tm_h, tm_h_small, offsets, mtile, R_rows, E, sh, d, I, y, perm_tok,
-                       rgate, comb_out, status, stream);
+  return launch_tc2<1>(tm_wd, tm_wd, tm_sd, tm_sd, tm_h, tm_h_small, offsets, mtile, R_rows, sh.rows, E, sh, d, I, y,
+                       perm_tok, rgate, comb_out, status, stream);
 }
 
 }  // namespace moe
