@@ -242,8 +242,9 @@ def run_reference(args, wl):
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = inputs_to_cpu(make_inputs(wl, dev, seed=0))
     threads = len(os.sched_getaffinity(0))
-    # each step: the whole layer on a bounded contiguous sample of the batch
-    per_step_budget = float(os.environ.get("MOE_REF_STEP_S", "3.0"))
+    # each step: the whole layer on a bounded contiguous sample of the batch,
+    # sized so that warm-up plus timed steps take about two minutes in all
+    per_step_budget = min(3.0, 120.0 / max(1, args.steps + args.warmup))
     _, n, _, _ = cpu_oracle_rate(inp, wl, per_step_budget)
     import oracle
 
