@@ -327,7 +327,7 @@ int64_t oracle_dispatch(const int32_t* topk_idx, int64_t T, int k, int E, int64_
 /* y[r, :] = down_e(SiLU(gate_e(x_t)) * up_e(x_t)) for each requested row
  * (t = tok[r], e = expert[r]); x is read as x_dtype, the weights as dtype.
  * h_round = 1 rounds the hidden activation to
- * bf16 (a diagnostic mode; parity is judged with h_round = 0). */
+ * bf16 (a diagnostic mode; the parity bars use h_round = 0). */
 void oracle_expert_rows(const void* x, int x_dtype, const void* w_gate, const void* w_up, const void* w_down,
                         int dtype, int64_t d, int64_t I, int64_t n, const int32_t* tok,
                         const int32_t* expert, int h_round, double* y) {

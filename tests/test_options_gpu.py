@@ -42,6 +42,8 @@ CASES = [
               router_std=0.1, zipf_bias=True), 1, True, 2, 1.25, True),
     (Workload("f32_all_options", T=100, d=64, E=6, k=2, I=64, renorm=False, dtype="f32", x_std=2.0, router_std=0.5,
               zipf_bias=True), 2, True, 1, 1.0, True),
+    (Workload("bf16_decode_all_options", T=32, d=512, E=8, k=2, I=512, renorm=True, dtype="bf16", x_std=2.0,
+              router_std=0.1, zipf_bias=True), 1, True, 1, 1.0, True),
 ]
 
 

@@ -43,6 +43,11 @@ EDGE = [
     Workload("bf16_k_eq_E", T=150, d=128, E=4, k=4, I=192, renorm=True, dtype="bf16"),
     Workload("bf16_max_E256_k8", T=96, d=64, E=256, k=8, I=64, renorm=True, dtype="bf16", router_std=0.5),
     Workload("bf16_many_tiles", T=1000, d=256, E=3, k=2, I=384, renorm=True, dtype="bf16", router_std=0.1),
+    # the GEMMs' configurations: at most 32 tokens (every tile in the 16-row
+    # token box), one more token, and an expert that receives all 32 tokens
+    Workload("bf16_T32_all_experts_full", T=32, d=256, E=8, k=8, I=256, renorm=True, dtype="bf16", router_std=0.3),
+    Workload("bf16_T33", T=33, d=256, E=4, k=2, I=192, renorm=False, dtype="bf16", router_std=0.3),
+    Workload("bf16_T32_one_expert", T=32, d=128, E=1, k=1, I=320, renorm=True, dtype="bf16"),
 ]
 
 
