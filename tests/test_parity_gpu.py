@@ -191,3 +191,43 @@ def test_bounded_wait_gives_up_and_reports():
     wl = Workload("after_timeout", T=40, d=128, E=4, k=2, I=128, renorm=True, dtype="bf16", router_std=0.3)
     inp, res, perm = run(wl, seed=11)
     check(wl, inp, res, perm)
+
+
+# ------------------------------------------------------------- CUDA graphs --
+
+@pytest.mark.parametrize("name", ["mixtral_decode", "small_bf16"])
+def test_layer_replays_from_a_cuda_graph(name):
+    """The whole call (its kernels chained by programmatic dependent launch)
+    can be captured once and replayed: the replay gives bit-identical outputs
+    to the eager call, also on a second batch copied into the captured input
+    buffer. The layer's status word is OR-ed by every call and never cleared
+    here, so the final check covers the warm-up, the capture and both
+    replays."""
+    from sparse_mixture_experts_renorm_b200 import MoELayer
+    from sparse_mixture_experts_renorm_b200.workloads import make_tokens
+
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl, "cuda", 0)
+    layer = MoELayer(inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k, wl.renorm, wl.T)
+    x = inp.x.clone()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())  # x and the weights were written on the current stream
+    with torch.cuda.stream(s):
+        for _ in range(2):  # warm-up outside the capture (attributes, occupancy queries)
+            layer(x, stream=s.cuda_stream)
+    torch.cuda.synchronize()
+    eager = layer.out.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        layer(x, stream=s.cuda_stream)
+    layer.out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(layer.out, eager)
+    x2 = make_tokens(wl, wl.T, "cuda", seed=7)
+    ref2 = moe_forward(x2, inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k, wl.renorm)
+    x.copy_(x2)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(layer.out, ref2.out) and torch.equal(layer.topk_idx, ref2.topk_idx)
+    assert int(layer.status.item()) == 0
