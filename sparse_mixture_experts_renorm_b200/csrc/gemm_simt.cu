@@ -12,7 +12,8 @@
 namespace moe {
 namespace {
 
-constexpr int kSK = 16;
+constexpr int kSK = 32;  // K columns per staged slice
+static_assert(kSimtBM == kSimtBN, "the staging loop fills the A and B slices with one index");
 
 template <int kMode>
 __global__ void __launch_bounds__(256) grouped_gemm_simt_kernel(const float* __restrict__ A,
@@ -71,7 +72,9 @@ __global__ void __launch_bounds__(256) grouped_gemm_simt_kernel(const float* __r
   const float* Bexp1 = kMode == 0 ? (shared ? S1 : B1) + widx * N * K : nullptr;
 
   for (int k0 = 0; k0 < K; k0 += kSK) {
-    for (int i = tid; i < kSimtBM * kSK; i += 256) {
+#pragma unroll 4  // the loads of half a slice in flight at once
+    for (int i0 = 0; i0 < kSimtBM * kSK; i0 += 256) {
+      const int i = i0 + tid;
       const int r = i / kSK, c = i % kSK;
       sA[c][r] = (r < rows && k0 + c < K) ? A[(size_t)(in0 + r) * K + k0 + c] : 0.f;
       const bool nok = n0 + r < N && k0 + c < K;

@@ -18,7 +18,7 @@ namespace moe {
 // (the UMMA M) for the bf16 tensor-core router, 32 for the fp32 SIMT router.
 constexpr int kRouterTokensTc = 128;
 constexpr int kRouterTokensSimt = 32;
-constexpr int kRouterThreads = 128;
+constexpr int kRouterThreads = 256;
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 8;
 

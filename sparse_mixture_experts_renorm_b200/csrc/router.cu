@@ -21,27 +21,74 @@ namespace {
 // fp32 logits with plain FFMA (the fp32 workload is small; TF32 tensor cores
 // would not meet its 1e-4 tolerance). With the RMSNorm, s_r[row] holds the
 // token's scale and the logit is r * sum_c x[c] * (w[c] * W_r[e,c]).
+// Thread pair (row, e) keeps its sum in a register while 32-column slices of
+// the block's x rows and of up to 32 router rows pass through shared memory
+// (coalesced loads, all of a slice in flight at once); each sum still runs
+// over c in index order. Experts beyond 32 take further passes.
+constexpr int kRC = 32;  // columns per staged slice
+constexpr int kRP = 8;   // (token, expert) pairs per thread and pass: 32 experts per pass
+
 __device__ void router_logits_f32(const float* __restrict__ x, const float* __restrict__ wr,
                                   const float* __restrict__ nw, bool norm, const float* s_r, int T, int d, int E,
                                   int tok0, float* s_logit, int ld) {
-  for (int i = threadIdx.x; i < kRouterTokensSimt * E; i += blockDim.x) {
-    const int e = i / kRouterTokensSimt, row = i - e * kRouterTokensSimt;
-    const int t = tok0 + row;
-    float s = 0.f;
-    if (t < T) {
-      const float* xr = x + (size_t)t * d;
-      const float* wrow = wr + (size_t)e * d;
-      if (nw)
-        for (int c = 0; c < d; ++c) s = fmaf(xr[c], nw[c] * wrow[c], s);
-      else
-        for (int c = 0; c < d; ++c) s = fmaf(xr[c], wrow[c], s);
-      if (norm) s *= s_r[row];
+  __shared__ float s_x[kRouterTokensSimt][kRC + 1];
+  __shared__ float s_w[kRouterThreads * kRP / kRouterTokensSimt][kRC + 1];
+  constexpr int kPassE = kRouterThreads * kRP / kRouterTokensSimt;
+  for (int e0 = 0; e0 < E; e0 += kPassE) {
+    const int ne = min(kPassE, E - e0);
+    float acc[kRP];
+#pragma unroll
+    for (int j = 0; j < kRP; ++j) acc[j] = 0.f;
+    for (int c0 = 0; c0 < d; c0 += kRC) {
+      const int w = min(kRC, d - c0);
+      __syncthreads();  // the previous slice has been consumed
+#pragma unroll
+      for (int i0 = 0; i0 < kRouterTokensSimt * kRC; i0 += kRouterThreads) {
+        const int i = i0 + threadIdx.x;
+        const int row = i / kRC, c = i % kRC;
+        const int t = tok0 + row;
+        s_x[row][c] = (t < T && c < w) ? x[(size_t)t * d + c0 + c] : 0.f;
+      }
+#pragma unroll
+      for (int i0 = 0; i0 < kPassE * kRC; i0 += kRouterThreads) {
+        const int i = i0 + threadIdx.x;
+        const int el = i / kRC, c = i % kRC;
+        float v = 0.f;
+        if (el < ne && c < w) {
+          v = wr[(size_t)(e0 + el) * d + c0 + c];
+          if (nw) v = nw[c0 + c] * v;
+        }
+        s_w[el][c] = v;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int j = 0; j < kRP; ++j) {
+        const int il = threadIdx.x + j * kRouterThreads;  // a warp shares el, lanes are rows
+        const int el = il / kRouterTokensSimt, row = il % kRouterTokensSimt;
+        if (el < ne) {
+          float s = acc[j];
+          for (int c = 0; c < w; ++c) s = fmaf(s_x[row][c], s_w[el][c], s);
+          acc[j] = s;
+        }
+      }
     }
-    s_logit[row * ld + e] = s;
+#pragma unroll
+    for (int j = 0; j < kRP; ++j) {
+      const int il = threadIdx.x + j * kRouterThreads;
+      const int el = il / kRouterTokensSimt, row = il % kRouterTokensSimt;
+      if (el < ne) {
+        float s = 0.f;
+        if (tok0 + row < T) s = norm ? acc[j] * s_r[row] : acc[j];
+        s_logit[row * ld + e0 + el] = s;
+      }
+    }
   }
   __syncthreads();
 }
 
+// kNE: probabilities per lane (E <= 32 * kNE), so that the per-token loops
+// hold no predicated-off copies for small E.
+template <int kNE>
 __global__ void __launch_bounds__(kRouterThreads) router_kernel(
     const float* __restrict__ x, const float* __restrict__ wr, const float* __restrict__ br, int T, int d, int E, int k,
     int renorm, int norm_form, float norm_eps, const float* __restrict__ nw, float* __restrict__ rnorm,
@@ -83,7 +130,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(
   router_logits_f32(x, wr, nw, norm_form != 0, s_r, T, d, E, tok0, s_p, ld);
 
   // ---- softmax, top-k and gates: one warp per token --------------------
-  const int NE = (E + 31) >> 5;  // values per lane (<= 8)
+  constexpr int NE = kNE;
   for (int row = warp; row < kRouterTokensSimt; row += kRouterThreads / 32) {
     if (row >= ntok) {
       if (lane < kMaxTopK) s_idx[row][lane] = -1;
@@ -92,11 +139,11 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(
       continue;
     }
     const int t = tok0 + row;
-    float v[8];
+    float v[kNE];
     float m = -INFINITY;
     bool finite = true;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < kNE; ++i) {
       const int e = lane + 32 * i;
       v[i] = -INFINITY;
       if (i < NE && e < E) {
@@ -111,7 +158,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(
     for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     float s = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < kNE; ++i) {
       const int e = lane + 32 * i;
       const float ex = (i < NE && e < E) ? expf(v[i] - m) : 0.f;
       v[i] = ex;
@@ -124,7 +171,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(
       s_z[row] = lse * lse;
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < kNE; ++i) {
       const int e = lane + 32 * i;
       v[i] = v[i] / s;
       if (i < NE && e < E) s_p[row * ld + e] = v[i];
@@ -145,7 +192,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(
         float bv = -INFINITY;
         int be = 0x7fffffff;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < kNE; ++i) {
           const int e = lane + 32 * i;
           if (i < NE && e < E && !((taken >> i) & 1u)) {
             float pv = v[i];
@@ -362,9 +409,10 @@ cudaError_t launch_router(moe_dtype dtype, const void* x, const void* w_router, 
                             blk_psum, blk_z, status, stream);
   const int nb = router_blocks(T, MOE_F32);
   const size_t smem = (size_t)kRouterTokensSimt * (E + 1) * sizeof(float);
-  cudaError_t err = cudaFuncSetAttribute(router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = E <= 32 ? router_kernel<1> : E <= 64 ? router_kernel<2> : E <= 128 ? router_kernel<4> : router_kernel<8>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
-  return launch_pdl(router_kernel, dim3(nb), dim3(kRouterThreads), smem, stream, static_cast<const float*>(x),
+  return launch_pdl(kern, dim3(nb), dim3(kRouterThreads), smem, stream, static_cast<const float*>(x),
                     static_cast<const float*>(w_router), b_router, T, d, E, k, renorm, norm.form, norm.eps,
                     static_cast<const float*>(norm.w), norm.rnorm, topk_idx, topk_gate, lrank, blk_cnt, blk_psum,
                     blk_z, status);
