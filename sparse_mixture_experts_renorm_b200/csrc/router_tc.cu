@@ -15,10 +15,14 @@
 // TMA, warp 1 issues 128 x N x 16 UMMAs (N = E rounded up to 16; TMA zero-fills
 // the missing router rows), and warps 2-5 read each token's logits from their
 // own TMEM lane. The other CTAs of the cluster add their partial logits into
-// the leading CTA's shared memory, which finishes the block: one thread per
-// token does the softmax, top-k and gates without cross-thread reductions
-// (logits in registers for E <= 64), then the block's histogram, ranks and
-// probability sums, and the block's sum of logsumexp^2 for the z-loss.
+// the leading CTA's shared memory, which finishes the block. For E <= 16 one
+// thread per token does the softmax, top-k and gates with its logits in
+// registers, then per-warp ballots give the histogram and ranks; for E > 16
+// the logits go to shared memory and all six warps take four lanes per token
+// (the softmax reduced by two shuffles, per-lane sorted top-k lists merged by
+// a four-lane arg-max), the histogram being a bit mask per (expert, 32-token
+// chunk). Both end with the block's probability sums and its sum of
+// logsumexp^2 for the z-loss.
 //
 // With the pre-MoE RMSNorm (Mixtral MoE Block, nn.RMSNorm before the MoE;
 // Model Architecture Patterns, "RMSNorm") the logits are
@@ -70,7 +74,7 @@ RouterCfg router_cfg(int T, int d, int E, bool norm, bool split, int num_sms) {
   const int cols = split ? 2 * c.lo_col : c.lo_col;
   c.tmem_cols = 32;
   while (c.tmem_cols < cols) c.tmem_cols <<= 1;
-  c.smem_bytes = c.stages * c.stage_bytes + c.part_bytes + 1024 + 12288;
+  c.smem_bytes = c.stages * c.stage_bytes + c.part_bytes + 1024 + 13312;
   return c;
 }
 
@@ -114,39 +118,6 @@ __device__ __forceinline__ void topk_insert(float (&bv)[kMaxTopK], int (&be)[kMa
   }
 }
 
-// The top kMaxTopK of p[0..E) (a row in shared memory): four independent
-// insertion chains over the experts e mod 4, merged at the end.
-__device__ __forceinline__ void topk_of_row(const float* p, int E, float (&bv)[kMaxTopK], int (&be)[kMaxTopK]) {
-  float cv[3][kMaxTopK];
-  int ce[3][kMaxTopK];
-#pragma unroll
-  for (int c = 0; c < 3; ++c)
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      cv[c][j] = -INFINITY;
-      ce[c][j] = 0x7fffffff;
-    }
-  auto val = [&](int e) {
-    const float x = p[e];
-    return (x != x) ? -INFINITY : x;
-  };
-  int e = 0;
-#pragma unroll 1
-  for (; e + 4 <= E; e += 4) {
-    const float p0 = val(e), p1 = val(e + 1), p2 = val(e + 2), p3 = val(e + 3);
-    topk_insert(bv, be, p0, e);
-    topk_insert(cv[0], ce[0], p1, e + 1);
-    topk_insert(cv[1], ce[1], p2, e + 2);
-    topk_insert(cv[2], ce[2], p3, e + 3);
-  }
-#pragma unroll 1
-  for (; e < E; ++e) topk_insert(bv, be, val(e), e);
-#pragma unroll
-  for (int c = 0; c < 3; ++c)
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) topk_insert(bv, be, cv[c][j], ce[c][j]);
-}
-
 // E <= kE: logits in registers (fully unrolled code); kE == 0: E > kRegE,
 // logits in shared memory and rolled loops (code executed once per block must
 // stay small: unrolled per-expert code for large E thrashes the instruction
@@ -176,9 +147,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   int* s_wcnt = s_idx + kRB * kMaxTopK;              // [4][E] per-warp counts, then exclusive prefix
   float* s_z = reinterpret_cast<float*>(s_wcnt + 4 * E);  // [4] per-warp sums of logsumexp^2
   float* s_bias = s_z + 4;                                 // [E] router bias (leading CTA)
+  float* s_rn = s_bias + E;                                // [128] RMSNorm scale per token (E > kRegE)
+  float* s_lse2 = s_rn + kRB;                              // [128] logsumexp^2 per token (E > kRegE)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = S > 1 ? cta_rank_in_cluster() : 0u;
+  // row stride of the logits in shared memory (E > kRegE): odd, so a warp's
+  // 32 token rows fall in 32 banks
+  const int ldp = (E + 1) | 1;
   const int blk = blockIdx.x / S;
   const int tok0 = blk * kRB;
   const int KB = d / kBK;
@@ -318,7 +294,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
     const uint32_t trow = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     const int nchunks = (E + 31) >> 5;
-    float* s_p = reinterpret_cast<float*>(ring);  // [128][E+1] when E > kRegE (ring free after the MMAs)
+    float* s_p = reinterpret_cast<float*>(ring);  // [128][ldp] when E > kRegE (ring free after the MMAs)
     for (int c = 0; c < nchunks; ++c) {
       uint32_t v[32];
       __syncwarp();
@@ -346,7 +322,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       } else {
 #pragma unroll
         for (int i = 0; i < 32; ++i)
-          if (c * 32 + i < E) s_p[r * (E + 1) + c * 32 + i] = __uint_as_float(v[i]);
+          if (c * 32 + i < E) s_p[r * ldp + c * 32 + i] = __uint_as_float(v[i]);
       }
     }
     if (S > 1 && rank > 0) {  // this CTA's share of the K loop goes to the leader
@@ -356,7 +332,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int e = 0; e < kL; ++e)
           if (e < E) st_cluster_f32(dst + e, 0, lg[e]);
       } else {
-        for (int e = 0; e < E; ++e) st_cluster_f32(dst + e, 0, s_p[r * (E + 1) + e]);
+        for (int e = 0; e < E; ++e) st_cluster_f32(dst + e, 0, s_p[r * ldp + e]);
       }
       if (norm_form) st_cluster_f32(part_ss + (size_t)(rank - 1) * kRB + r, 0, ss);
     }
@@ -364,8 +340,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (S > 1) cluster_sync_all();  // every partial has landed in the leading CTA
 
-  if (rank == 0 && warp >= 2) {
-    // ------------------------------------------------ one thread per token --
+  if (kE > 0 && rank == 0 && warp >= 2) {
+    // ------------------------- E <= kRegE: one thread per token, in registers --
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const int t = tok0 + r;
@@ -451,52 +427,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           be[j] = bi;
         }
       }
-    } else {
-      // rolled loops over this token's row of s_p, four experts per trip
-      // (independent chains for the maximum and the sum)
-      float* pr = s_p + r * ld;
-      auto logit = [&](int e) {
-        float l = pr[e];
-        for (int s2 = 0; s2 < S - 1; ++s2) l += part[((size_t)s2 * kRB + r) * E + e];
-        if (norm_form) l *= rn;
-        if (br) l += s_bias[e];
-        finite = finite && isfinite(l);
-        pr[e] = l;
-        return l;
-      };
-      float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-      int e4 = 0;
-#pragma unroll 1
-      for (; e4 + 4 <= E; e4 += 4) {
-        m0 = fmaxf(m0, logit(e4));
-        m1 = fmaxf(m1, logit(e4 + 1));
-        m2 = fmaxf(m2, logit(e4 + 2));
-        m3 = fmaxf(m3, logit(e4 + 3));
-      }
-#pragma unroll 1
-      for (int e = e4; e < E; ++e) m0 = fmaxf(m0, logit(e));
-      const float m = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
-      auto expo = [&](int e) {
-        const float ex = __expf(pr[e] - m);
-        pr[e] = ex;
-        return ex;
-      };
-      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll 1
-      for (int e = 0; e + 4 <= E; e += 4) {
-        s0 += expo(e);
-        s1 += expo(e + 1);
-        s2 += expo(e + 2);
-        s3 += expo(e + 3);
-      }
-#pragma unroll 1
-      for (int e = e4; e < E; ++e) s0 += expo(e);
-      const float s = (s0 + s1) + (s2 + s3);
-      lse = m + logf(s);
-      const float inv_s = 1.0f / s;
-#pragma unroll 4
-      for (int e = 0; e < E; ++e) pr[e] = valid ? pr[e] * inv_s : 0.f;
-      topk_of_row(pr, E, bv, be);
     }
     if (valid && !finite) atomicOr(status, MOE_DEV_NONFINITE);
     if (blk_z) {  // this warp's sum of logsumexp^2 (a fixed shuffle tree)
@@ -575,6 +505,177 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
       for (int j = 0; j < kMaxTopK; ++j)
         if (j < k) lrank[(size_t)t * k + j] = (int)myrank[j] + s_wcnt[q * E + be[j]];
+    }
+  }
+
+  if (kE == 0 && rank == 0) {
+    // ------------- E > kRegE: all six warps finish the block, four lanes a token --
+    // Expert e of a token belongs to lane e mod 4 of its four: the softmax
+    // reduces over the four lanes with two shuffles, each lane keeps a sorted
+    // top-k list of its experts, and k rounds of a four-lane arg-max merge
+    // them (ties to the lower index, as every list is). A warp takes eight
+    // tokens four rows apart, so its 32 lanes read 32 different banks of the
+    // odd-strided rows. The histogram is a bit mask per (expert, 32-token
+    // chunk), from which the in-block ranks and the counts follow; one warp
+    // per expert sums its probabilities in a fixed order.
+    float* s_p = reinterpret_cast<float*>(ring);             // [128][ldp] logits, then probabilities
+    uint32_t* s_mask = reinterpret_cast<uint32_t*>(s_wcnt);  // [E][4] tokens of a chunk choosing e
+    if (warp >= 2) {
+      const int r = (warp & 3) * 32 + lane;
+      float rn = 1.0f;  // RMSNorm scale of this token (1 without the norm)
+      if (norm_form) {
+        for (int s2 = 0; s2 < S - 1; ++s2) ss += part_ss[(size_t)s2 * kRB + r];
+        const float ms = ss / (float)d;
+        rn = norm_form == MOE_NORM_RMS ? 1.0f / sqrtf(ms + norm_eps) : 1.0f / (sqrtf(ms) + norm_eps);
+        if (tok0 + r < T) rnorm[tok0 + r] = rn;
+      }
+      s_rn[r] = rn;
+    }
+    if (br)
+      for (int e = threadIdx.x; e < E; e += kGemmThreads) s_bias[e] = br[e];
+    for (int i = threadIdx.x; i < 4 * E; i += kGemmThreads) s_mask[i] = 0u;
+    __syncthreads();
+
+    const int sub = lane & 3;
+    for (int set = warp; set < kRB / 8; set += kGemmThreads / 32) {  // 16 sets of 8 tokens
+      const int r = (set >> 2) * 32 + (set & 3) + 4 * (lane >> 2);
+      const int t = tok0 + r;
+      const bool valid = t < T;
+      float* pr = s_p + r * ldp;
+      const float rn = s_rn[r];
+      float m = -INFINITY;
+      bool finite = true;
+      for (int e = sub; e < E; e += 4) {
+        float l = pr[e];
+        for (int s2 = 0; s2 < S - 1; ++s2) l += part[((size_t)s2 * kRB + r) * E + e];
+        if (norm_form) l *= rn;
+        if (br) l += s_bias[e];
+        finite = finite && isfinite(l);
+        pr[e] = l;
+        m = fmaxf(m, l);
+      }
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      float sum = 0.f;
+      for (int e = sub; e < E; e += 4) {
+        const float ex = __expf(pr[e] - m);
+        pr[e] = ex;
+        sum += ex;
+      }
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+      const float lse = m + logf(sum);
+      const float inv_s = 1.0f / sum;
+      float bv[kMaxTopK];
+      int be[kMaxTopK];
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j) {
+        bv[j] = -INFINITY;
+        be[j] = 0x7fffffff;
+      }
+      for (int e = sub; e < E; e += 4) {
+        const float p = pr[e] * inv_s;
+        pr[e] = valid ? p : 0.f;
+        topk_insert(bv, be, (p != p) ? -INFINITY : p, e);  // a NaN ranks last
+      }
+      // k rounds: the best head of the four lists wins and leaves its list
+      float gv[kMaxTopK];
+      int ge[kMaxTopK];
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j) {
+        gv[j] = 0.f;
+        ge[j] = 0;
+        if (j < k) {
+          float cv = bv[0];
+          int ce = be[0];
+#pragma unroll
+          for (int off = 1; off <= 2; off <<= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, cv, off);
+            const int oe = __shfl_xor_sync(0xffffffffu, ce, off);
+            if (ahead(ov, oe, cv, ce)) {
+              cv = ov;
+              ce = oe;
+            }
+          }
+          gv[j] = cv;
+          ge[j] = ce;
+          const bool won = be[0] == ce;
+#pragma unroll
+          for (int i = 0; i + 1 < kMaxTopK; ++i) {
+            bv[i] = won ? bv[i + 1] : bv[i];
+            be[i] = won ? be[i + 1] : be[i];
+          }
+          if (won) {
+            bv[kMaxTopK - 1] = -INFINITY;
+            be[kMaxTopK - 1] = 0x7fffffff;
+          }
+        }
+      }
+      int fin = finite ? 1 : 0;
+      fin &= __shfl_xor_sync(0xffffffffu, fin, 1);
+      fin &= __shfl_xor_sync(0xffffffffu, fin, 2);
+      float psel = 0.f;
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j)
+        if (j < k) psel += gv[j];
+      if (sub == 0) {
+        if (valid && !fin) atomicOr(status, MOE_DEV_NONFINITE);
+        s_lse2[r] = valid ? lse * lse : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < kMaxTopK; ++j) {
+        if (j < k && (j & 3) == sub) {  // slot j is written by lane j mod 4
+          float g;
+          if (!renorm)
+            g = gv[j];
+          else if (psel > 0.f)
+            g = gv[j] / psel;
+          else
+            g = 1.0f / (float)k;
+          if (valid) {
+            topk_idx[(size_t)t * k + j] = ge[j];
+            topk_gate[(size_t)t * k + j] = g;
+            atomicOr(&s_mask[ge[j] * 4 + (r >> 5)], 1u << (r & 31));
+          }
+          s_idx[r * kMaxTopK + j] = valid ? ge[j] : -1;
+        }
+      }
+    }
+    __syncthreads();
+
+    // rank of each assignment among the block's tokens choosing its expert
+    for (int i = threadIdx.x; i < kRB * k; i += kGemmThreads) {
+      const int r = i / k, j = i - r * k;
+      const int e = s_idx[r * kMaxTopK + j];
+      if (e >= 0) {
+        const int c = r >> 5;
+        int rk = __popc(s_mask[e * 4 + c] & ((1u << (r & 31)) - 1u));
+        for (int cc = 0; cc < c; ++cc) rk += __popc(s_mask[e * 4 + cc]);
+        lrank[(size_t)(tok0 + r) * k + j] = rk;
+      }
+    }
+    // per expert: the block's count and its probability sum (a fixed tree)
+    for (int e = warp; e < E; e += kGemmThreads / 32) {
+      float ps = ((s_p[lane * ldp + e] + s_p[(lane + 32) * ldp + e]) + s_p[(lane + 64) * ldp + e]) +
+                 s_p[(lane + 96) * ldp + e];
+#pragma unroll
+      for (int off = 16; off; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+      if (lane == 0) {
+        blk_psum[(size_t)blk * E + e] = ps;
+        blk_cnt[(size_t)blk * E + e] =
+            __popc(s_mask[e * 4]) + __popc(s_mask[e * 4 + 1]) + __popc(s_mask[e * 4 + 2]) + __popc(s_mask[e * 4 + 3]);
+      }
+    }
+    if (blk_z && warp == 0) {  // per 32-token quarter a shuffle tree, then the quarters in order
+      float z = 0.f;
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {
+        float zq = s_lse2[qq * 32 + lane];
+#pragma unroll
+        for (int off = 16; off; off >>= 1) zq += __shfl_xor_sync(0xffffffffu, zq, off);
+        z = qq == 0 ? zq : z + zq;
+      }
+      if (lane == 0) blk_z[blk] = z;
     }
   }
 
