@@ -231,3 +231,35 @@ def test_layer_replays_from_a_cuda_graph(name):
     torch.cuda.synchronize()
     assert torch.equal(layer.out, ref2.out) and torch.equal(layer.topk_idx, ref2.topk_idx)
     assert int(layer.status.item()) == 0
+
+
+# ------------------------------------------------------- host-memory path --
+
+@pytest.mark.parametrize("name", ["small_bf16", "tiny_f32"])
+def test_host_pipeline_matches_device_calls(name):
+    """The end-to-end path (pinned host batches in, copies on their own
+    streams overlapped with the compute of neighbouring batches, fp32 output
+    and statistic back to pinned host memory) returns, for every batch, the
+    bit-identical output and statistic of a plain device call on the same
+    batch, also when batches reuse the two device buffers in turn."""
+    from sparse_mixture_experts_renorm_b200 import HostPipeline, MoELayer
+    from sparse_mixture_experts_renorm_b200.workloads import make_tokens
+
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl, "cuda", 0)
+    layer = MoELayer(inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k, wl.renorm, wl.T)
+    pipe = HostPipeline(layer)
+    n = 5
+    xs = [make_tokens(wl, wl.T, "cpu", seed=100 + i).pin_memory() for i in range(n)]
+    outs = [torch.empty((wl.T, wl.d), dtype=torch.float32).pin_memory() for _ in range(n)]
+    auxs = [torch.empty((1,), dtype=torch.float32).pin_memory() for _ in range(n)]
+    for i in range(n):
+        pipe.submit(xs[i], outs[i], auxs[i])
+    pipe.synchronize()
+    assert int(layer.status.item()) == 0
+    for i in range(n):
+        ref = moe_forward(xs[i].cuda(), inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k,
+                          wl.renorm)
+        torch.cuda.synchronize()
+        assert torch.equal(outs[i], ref.out.cpu()), f"batch {i}"
+        assert torch.equal(auxs[i], ref.aux.cpu()), f"batch {i}"
