@@ -1,7 +1,7 @@
 """Host logic of bench.py (CPU): the algorithmic work behind the roofline
 fractions, the L2 policy, the fused-combine rule and the lookup of committed
-ncu traffic. The expected values are the survey's per-workload totals,
-recomputed here from the shapes."""
+ncu traffic. The expected values are the per-workload totals (active-expert
+FLOPs, expert weight bytes) recomputed here from the shapes."""
 import os
 import sys
 
