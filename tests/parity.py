@@ -28,7 +28,7 @@ Rules:
     oracle, and max-abs <= 2e-2 against the fp64 oracle that rounds the two
     stored bf16 operands (x_hat and H) as the kernels store them. The
     max-abs bar is an absolute bound set for the plain layer at the
-    spec shapes; x_hat is one more bf16 rounding and each shared
+    benchmark workloads' shapes; x_hat is one more bf16 rounding and each shared
     expert one more full expert output of weight 1, which at the Mixtral
     prefill shape takes the pure-oracle max-abs to about 4e-2 while the
     relative error stays below 3e-3. z-loss: relative error <= 1e-4 (each token's
