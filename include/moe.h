@@ -20,8 +20,8 @@
  *
  * Conventions for every entry point:
  *   - All tensors are row-major and contiguous. Weights use the nn.Linear
- *     [out, in] layout, stacked per expert ("packed experts", KempnerForge
- *     ModelConfig.moe_packed_experts): W_router [E, d], W_gate [E, I, d],
+ *     [out, in] layout, stacked per expert (the layout that KempnerForge
+ *     ModelConfig.moe_packed_experts selects): W_router [E, d], W_gate [E, I, d],
  *     W_up [E, I, d], W_down [E, d, I].
  *   - Pointers documented as "device" must be CUDA device (or managed)
  *     memory on the current device; the caller owns every buffer. The
@@ -165,13 +165,13 @@ moe_status moe_get_permutation(const void* workspace, size_t workspace_bytes, in
  * the per-token scale into its logits (exact x, w * W_r split into two bf16
  * terms), and the experts read x_hat rounded once to the layer dtype.
  *
- * Shared experts ("moe_shared_experts: shared experts that process all
- * tokens", KempnerForge ModelConfig): n_shared SwiGLU MLPs of the routed
+ * Shared experts (KempnerForge ModelConfig, moe_shared_experts: experts
+ * that every token passes through): n_shared SwiGLU MLPs of the routed
  * experts' shape, applied to every token and added with weight 1:
  *   out[t] += sum_s W_sdown[s] (SiLU(W_sgate[s] x_t) * (W_sup[s] x_t))
  *
- * Capacity ("moe_capacity_factor: 0 = no drop, > 0 = cap tokens per
- * expert"): every expert keeps at most C = ceil(cf * T * k / E) assignments,
+ * Capacity (KempnerForge ModelConfig, moe_capacity_factor: zero keeps
+ * every assignment, a positive factor limits the tokens an expert takes): every expert keeps at most C = ceil(cf * T * k / E) assignments,
  * its first C in dispatch order (tokens ascending); a dropped slot adds
  * nothing to out. topk_idx, topk_gate, counts and aux are those before
  * dropping; moe_get_permutation reports the kept rows and inv = -1 for a
@@ -241,9 +241,12 @@ moe_status moe_forward_ex(const void* x, const void* w_router, const float* b_ro
  *     16 MiB covers, for example, a 32-token decode batch of the Mixtral
  *     shape (d=4096, E=8, k=2, I=14336), which needs about 3.3 MB.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture. The call allocates nothing: no cudaMalloc,
- *     no cudaFree.
+ *     (cudaGetSymbolAddress, with that device current) and caches it with
+ *     the id of the current CUDA context; a call in another context (after
+ *     cudaDeviceReset, or in a context the caller made current) looks it up
+ *     again. Make the first call on a device, and the first in a new
+ *     context, before any stream capture. The call allocates nothing: no
+ *     cudaMalloc, no cudaFree.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind; the library rewrites everything it reads on each call, and
  *     clears its own status word when status_dev is NULL. Calls that overlap

@@ -8,6 +8,8 @@
 // fixed. They still own the inputs and outputs; only the scratch moves into
 // the static array below. Every GPU that loads the library keeps the array
 // for as long as the process lives.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "moe_internal.h"
@@ -17,11 +19,54 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
 
-// Device address of the array on each device. In host code the array's name
-// is only a host-side stand-in, so the address is looked up once per device
-// (with that device current) and passed to the kernels as a plain pointer.
+// Device address of the array, per device, together with the unique id of
+// the CUDA context it was looked up in. In host code the array's name is only
+// a host-side stand-in, so the address is looked up (with that device and
+// context current) and passed to the kernels as a plain pointer. A context
+// that is destroyed and created again (cudaDeviceReset, or a caller that
+// switches to its own context) loads the module again, possibly at another
+// address, and gets a new id, so the lookup is then repeated.
+struct ScratchAddr {
+  unsigned long long ctx_id;
+  void* addr;
+};
 std::mutex g_mu;
-void* g_scratch_addr[64] = {};
+ScratchAddr g_scratch_addr[64] = {};
+
+// The driver's cuCtxGetCurrent and cuCtxGetId through the runtime's entry
+// point query (the library links only the runtime).
+struct CtxFns {
+  PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  PFN_cuCtxGetId_v12000 get_id = nullptr;
+};
+const CtxFns& ctx_fns() {
+  static CtxFns f;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  return f;
+}
+
+// Unique id of the calling thread's current context, or 0 when there is none
+// yet (or the driver cannot say).
+unsigned long long current_ctx_id() {
+  const CtxFns& f = ctx_fns();
+  if (!f.get_current || !f.get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (f.get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  unsigned long long id = 0;
+  if (f.get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 }  // namespace
 }  // namespace moe
@@ -56,17 +101,20 @@ extern "C" moe_status moe_forward_noalloc(const void* x, const void* w_router, c
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_addr[dev]) {
+    const unsigned long long id = current_ctx_id();
+    ScratchAddr& slot = g_scratch_addr[dev];
+    if (!slot.addr || id == 0 || slot.ctx_id != id) {
       void* p = nullptr;
-      err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      err = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // also makes the device's primary context current
       if (err != cudaSuccess || !p) {
         set_error_detail("moe_forward_noalloc: cudaGetSymbolAddress of the static scratch failed: %s",
                          cudaGetErrorString(err));
         return MOE_ERR_CUDA;
       }
-      g_scratch_addr[dev] = p;
+      slot.addr = p;
+      slot.ctx_id = current_ctx_id();
     }
-    scratch = g_scratch_addr[dev];
+    scratch = slot.addr;
   }
   return moe_forward(x, w_router, b_router, w_gate, w_up, w_down, T, d, E, k, I, renorm, dtype, out, topk_idx,
                      topk_gate, counts, aux, scratch, (size_t)MOE_NOALLOC_SCRATCH_BYTES, status_dev, stream);
