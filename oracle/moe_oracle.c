@@ -12,21 +12,22 @@
  *   router        logits[t,e] = sum_c x[t,c] * Wr[e,c] (+ b[e])
  *                 axonml-nn layers/moe.rs, MoERouter::route (gate Linear,
  *                 no bias); the optional per-expert bias is the skewed-load
- *                 workload's "router logit bias", added before the softmax.
+ *                 workload's per-expert bias on the router logits, added before
+ *                 the softmax.
  *   softmax       p = exp(l - max l) / sum exp(l - max l)
  *                 axonml-nn moe.rs, MoERouter::route (softmax(-1));
- *                 Mixtral MoE Block, "The PyTorch it exports" (_moe_forward).
+ *                 Mixtral MoE Block, the exported PyTorch (_moe_forward).
  *   top-k         the k largest p, ordered by (p descending, index ascending):
  *                 axonml-nn moe.rs, MoERouter::route sorts (index, prob) pairs
  *                 with a stable descending sort, so equal probabilities keep
  *                 the lower expert index first.
  *   gates         renorm: g_j = p_j / sum_j p_j (1/k each if that sum is <= 0),
- *                 axonml-nn moe.rs, MoERouter::route ("Normalize top-k
- *                 weights"); Mixtral MoE Block, _moe_forward (top_w / sum).
+ *                 axonml-nn moe.rs, MoERouter::route (its renormalisation of
+ *                 the k weights); Mixtral MoE Block, _moe_forward (top_w / sum).
  *                 no renorm: g_j = p_j, Model Architecture Patterns,
  *                 "Top-K Router" (TopKRouter returns the raw top-k softmax).
  *   statistics    counts[e] = #{(t,j) : idx[t,j] = e}, axonml-nn moe.rs,
- *                 MoELayer::forward ("Track expert utilization") and
+ *                 MoELayer::forward (its utilization counts) and
  *                 expert_utilization(); P[e] = mean_t p[t,e] and
  *                 aux = E * sum_e f_e * P_e, load_balancing_loss().
  *                 f_e is read as counts_e / (T*k), the fraction of the T*k
@@ -35,7 +36,7 @@
  *                 by T only, which is k times this value.
  *   dispatch      for e ascending, for t ascending, every (t,j) with
  *                 idx[t,j] = e takes the next row: axonml-nn moe.rs,
- *                 MoELayer::forward ("Process each expert: gather tokens").
+ *                 MoELayer::forward (its loop over experts collecting their tokens).
  *   expert        y = down(SiLU(gate(x)) * up(x)), SiLU(z) = z / (1 + e^-z),
  *                 axonml-nn moe.rs, Expert::forward; Model Architecture
  *                 Patterns, "SwiGLU FFN". Weights are nn.Linear layout
@@ -43,7 +44,7 @@
  *                 down [E, d, I].
  *   combine       out[t] = sum_j g[t,j] * y_{idx[t,j]}(x[t]), each expert's
  *                 output weighted by its own gate: axonml-nn moe.rs,
- *                 MoELayer::forward ("Scatter weighted outputs back");
+ *                 MoELayer::forward (its weighted scatter back to token order);
  *                 Mixtral MoE Block markdown, _moe_forward.
  *
  * Options of the layer that the pages name as configuration knobs:
@@ -58,14 +59,16 @@
  *                 config enables ("moe_router_z_loss_weight"; the Mixtral
  *                 page's note on the router z-loss): mean over tokens of
  *                 (logsumexp_e logits[t,e])^2, on the logits with their bias.
- *   capacity      "moe_capacity_factor: 0 = no drop, > 0 = cap tokens per
- *                 expert": capacity C = ceil(cf * T * k / E) assignments per
+ *   capacity      KempnerForge ModelConfig, moe_capacity_factor (zero keeps
+ *                 every assignment, a positive factor limits the tokens an
+ *                 expert takes): capacity C = ceil(cf * T * k / E) assignments per
  *                 expert; an expert keeps its first C assignments in dispatch
  *                 order (tokens ascending) and drops the rest, whose slots
  *                 then contribute nothing to the output. Routing, gates,
  *                 counts and the balance statistic are those before dropping.
- *   shared        "moe_shared_experts: shared experts that process all
- *                 tokens", each the same SwiGLU MLP as a routed expert
+ *   shared        KempnerForge ModelConfig, moe_shared_experts (experts that
+ *                 every token passes through), each the same SwiGLU MLP as a
+ *                 routed expert
  *                 (the parameter count adds n_shared * expert_mlp); their
  *                 outputs are added to every token with weight 1.
  *

@@ -29,6 +29,8 @@
 // ("moe_shared_experts", KempnerForge ModelConfig) are extra groups after the
 // routed experts, each over all T tokens, with their own weight tensor maps.
 // Every wait is bounded.
+#include <atomic>
+
 #include "common.cuh"
 
 namespace moe {
@@ -517,12 +519,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
   }
 }
 
+// Resident CTA pairs per GPU for one configuration, queried once per device.
+// Host threads may race on the first query of a device; each computes the
+// same value and the atomic store publishes it.
 template <class Cfg>
 int max_active_pairs(const void* kern) {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (cache[dev] == 0) {
+  const int have = cache[dev].load(std::memory_order_acquire);
+  if (have > 0) return have;
+  {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
@@ -536,9 +543,9 @@ int max_active_pairs(const void* kern) {
     cfg.numAttrs = 1;
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return 0;
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_release);
+    return n;
   }
-  return cache[dev];
 }
 
 template <int kMode, class Cfg>

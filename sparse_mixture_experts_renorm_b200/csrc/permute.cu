@@ -1,9 +1,10 @@
 // permute.cu — kernel (b), the dispatch: every (token, slot) gets its row in
 // the expert-contiguous order (experts ascending, tokens ascending within an
-// expert, axonml-nn layers/moe.rs, MoELayer::forward "gather tokens for this
-// expert"), and the token's row of x is copied to each of its k rows; and
-// kernel (d), the combine: out[t] = sum_j gate[t,j] * Y[row(t,j)] (same page,
-// "Scatter weighted outputs back", each expert weighted by its own gate).
+// expert: the order in which axonml-nn layers/moe.rs, MoELayer::forward,
+// collects each expert's tokens), and the token's row of x is copied to each
+// of its k rows; and kernel (d), the combine: out[t] = sum_j gate[t,j] *
+// Y[row(t,j)] (the same function's scatter of the expert outputs back to
+// token order, each expert weighted by its own gate).
 // Options: the pre-MoE RMSNorm is applied on the copy; with a capacity
 // ("moe_capacity_factor", KempnerForge ModelConfig) a slot whose rank in its
 // expert reaches the capacity is dropped; shared experts ("moe_shared_experts")

@@ -8,7 +8,7 @@
 //
 // Method: axonml-nn layers/moe.rs, MoERouter::route (Linear -> softmax ->
 // stable descending sort -> first k -> renormalise, 1/k if the sum is not
-// positive), MoELayer::forward ("Track expert utilization") and
+// positive), MoELayer::forward (its per-expert utilization counts) and
 // load_balancing_loss (E * sum_i f_i * P_i); Model Architecture Patterns,
 // "Top-K Router" (raw top-k softmax gates when not renormalised).
 #include <math.h>

@@ -5,7 +5,7 @@
 //
 // Method: axonml-nn layers/moe.rs, MoERouter::route (Linear -> softmax ->
 // stable descending sort -> first k -> renormalise, 1/k if the sum is not
-// positive), MoELayer::forward ("Track expert utilization"),
+// positive), MoELayer::forward (its per-expert utilization counts),
 // load_balancing_loss (E * sum_i f_i * P_i); Model Architecture Patterns,
 // "Top-K Router" (raw top-k softmax gates when not renormalised).
 //
@@ -33,6 +33,8 @@
 // operands hi + lo whose products go to two accumulators, so x is used as
 // stored and the weight's product is carried to about 16 bits.
 #include <math.h>
+
+#include <atomic>
 
 #include "common.cuh"
 
@@ -689,16 +691,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// SMs of the current device, queried once per device (host threads that race
+// on the first query store the same value).
 int sm_count() {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cache[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
-    cache[dev] = n;
-  }
-  return cache[dev];
+  const int have = cache[dev].load(std::memory_order_acquire);
+  if (have > 0) return have;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  cache[dev].store(n, std::memory_order_release);
+  return n;
 }
 
 }  // namespace
