@@ -4,6 +4,7 @@
 // on the caller's stream. Nothing here synchronises the host or allocates.
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -194,6 +195,17 @@ int capacity_of(double cf, int T, int k, int E) {
   return c >= (double)T ? T : (int)c;
 }
 
+// NVTX range on the host thread for one call and one range per kernel
+// launch, so a timeline tool (Nsight Systems) can tie each kernel to the call
+// and step that issued it. Without an attached tool the push and pop return
+// at once.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 struct EventMarks {
   void* const* events;
   int n;
@@ -209,6 +221,7 @@ moe_status forward_impl(const void* x, const void* w_router, const float* b_rout
                         moe_dtype dtype, const Opts& o, float* out, int32_t* topk_idx, float* topk_gate,
                         int32_t* counts, float* aux, void* workspace, size_t workspace_bytes, int32_t* status_dev,
                         void* stream_ptr, EventMarks marks) {
+  NvtxRange call_range("moe_forward");
   moe_status st = check_shape(T, d, E, k, I, dtype);
   if (st != MOE_OK) return st;
   if (renorm != 0 && renorm != 1) return fail(MOE_ERR_INVALID_ARG, "renorm must be 0 or 1 (got %d)", renorm);
@@ -276,16 +289,23 @@ moe_status forward_impl(const void* x, const void* w_router, const float* b_rout
   if (norm && dtype == MOE_BF16 && o.norm_w) {
     rn.w_hi = ws + w.wr_hi;
     rn.w_lo = ws + w.wr_lo;
+    NvtxRange r("split_router_weight");
     err = launch_split_router_weight(w_router, o.norm_w, E, d, ws + w.wr_hi, ws + w.wr_lo, stream);
     if (err != cudaSuccess) return fail_cuda(err, "router weight split kernel");
   }
   float* blk_z = o.zloss ? reinterpret_cast<float*>(ws + w.blk_z) : nullptr;
-  err = launch_router(dtype, x, w_router, b_router, T, d, E, k, renorm, rn, topk_idx, topk_gate, lrank, blk_cnt,
-                      blk_psum, blk_z, status, stream);
+  {
+    NvtxRange r("router_topk");
+    err = launch_router(dtype, x, w_router, b_router, T, d, E, k, renorm, rn, topk_idx, topk_gate, lrank, blk_cnt,
+                        blk_psum, blk_z, status, stream);
+  }
   if (err != cudaSuccess) return fail_cuda(err, "router kernel");
   marks.mark(stream);
-  err = launch_route_scan(router_blocks(T, dtype), T, E, k, cap, o.n_shared, blk_cnt, blk_psum, blk_z, cnt, offsets,
-                          mtile, aux_p, o.zloss, o.dropped, stream);
+  {
+    NvtxRange r("route_scan");
+    err = launch_route_scan(router_blocks(T, dtype), T, E, k, cap, o.n_shared, blk_cnt, blk_psum, blk_z, cnt,
+                            offsets, mtile, aux_p, o.zloss, o.dropped, stream);
+  }
   if (err != cudaSuccess) return fail_cuda(err, "routing scan kernel");
   marks.mark(stream);
   // With k = 2 (and no shared experts) the bf16 path folds the combine into
@@ -293,9 +313,12 @@ moe_status forward_impl(const void* x, const void* w_router, const float* b_rout
   // result stays deterministic); otherwise a separate combine kernel sums the
   // rows in a fixed order.
   const bool fused_combine = dtype == MOE_BF16 && k == 2 && o.n_shared == 0;
-  err = launch_permute(dtype, x, T, d, E, k, router_block_tokens(dtype), topk_idx, lrank, blk_cnt, offsets,
-                       cap >= 0 ? 1 : 0, perm_tok, inv, xp, topk_gate, rgate, fused_combine ? out : nullptr, rnorm,
-                       o.norm_w, o.n_shared > 0 ? R : -1, status, stream);
+  {
+    NvtxRange r("permute");
+    err = launch_permute(dtype, x, T, d, E, k, router_block_tokens(dtype), topk_idx, lrank, blk_cnt, offsets,
+                         cap >= 0 ? 1 : 0, perm_tok, inv, xp, topk_gate, rgate, fused_combine ? out : nullptr, rnorm,
+                         o.norm_w, o.n_shared > 0 ? R : -1, status, stream);
+  }
   if (err != cudaSuccess) return fail_cuda(err, "permute kernel");
 
   // shared experts: gate/up read the one copy of x at rows R..R+T-1 and write
@@ -321,27 +344,40 @@ moe_status forward_impl(const void* x, const void* w_router, const float* b_rout
         !make_tmap_bf16_2d(&tm_h_s, h, (uint64_t)Rh, (uint64_t)I, 16))
       return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point unavailable or bad pointer)");
     marks.mark(stream);
-    err = launch_gemm_gateup_tc2(tm_wg, tm_wu, tm_sg, tm_su, tm_xp, tm_xp_s, offsets, mtile, Rh, E, sh_up, I, d, h,
-                                 status, stream);
+    {
+      NvtxRange r("grouped_gemm_gateup_swiglu");
+      err = launch_gemm_gateup_tc2(tm_wg, tm_wu, tm_sg, tm_su, tm_xp, tm_xp_s, offsets, mtile, Rh, E, sh_up, I, d, h,
+                                   status, stream);
+    }
     if (err != cudaSuccess) return fail_cuda(err, "gate/up grouped GEMM");
     marks.mark(stream);
-    err = launch_gemm_down_tc2(tm_wd, tm_sd, tm_h, tm_h_s, offsets, mtile, Rh, E, sh_down, I, d, y, perm_tok, rgate,
-                               fused_combine ? out : nullptr, status, stream);
+    {
+      NvtxRange r("grouped_gemm_down");
+      err = launch_gemm_down_tc2(tm_wd, tm_sd, tm_h, tm_h_s, offsets, mtile, Rh, E, sh_down, I, d, y, perm_tok,
+                                 rgate, fused_combine ? out : nullptr, status, stream);
+    }
     if (err != cudaSuccess) return fail_cuda(err, "down grouped GEMM");
   } else {
     marks.mark(stream);
-    err = launch_gemm_gateup_simt(static_cast<const float*>(xp), static_cast<const float*>(w_gate),
-                                  static_cast<const float*>(w_up), static_cast<const float*>(o.sg),
-                                  static_cast<const float*>(o.su), offsets, Rh, E, sh_up, I, d,
-                                  static_cast<float*>(h), stream);
+    {
+      NvtxRange r("grouped_gemm_gateup_swiglu");
+      err = launch_gemm_gateup_simt(static_cast<const float*>(xp), static_cast<const float*>(w_gate),
+                                    static_cast<const float*>(w_up), static_cast<const float*>(o.sg),
+                                    static_cast<const float*>(o.su), offsets, Rh, E, sh_up, I, d,
+                                    static_cast<float*>(h), stream);
+    }
     if (err != cudaSuccess) return fail_cuda(err, "gate/up grouped GEMM (fp32)");
     marks.mark(stream);
-    err = launch_gemm_down_simt(static_cast<const float*>(h), static_cast<const float*>(w_down),
-                                static_cast<const float*>(o.sd), offsets, Rh, E, sh_down, I, d, y, stream);
+    {
+      NvtxRange r("grouped_gemm_down");
+      err = launch_gemm_down_simt(static_cast<const float*>(h), static_cast<const float*>(w_down),
+                                  static_cast<const float*>(o.sd), offsets, Rh, E, sh_down, I, d, y, stream);
+    }
     if (err != cudaSuccess) return fail_cuda(err, "down grouped GEMM (fp32)");
   }
   marks.mark(stream);
   if (!fused_combine) {
+    NvtxRange r("combine");
     err = launch_combine(T, d, k, y, inv, topk_gate, cap >= 0 ? 1 : 0, o.n_shared, R, out, status, stream);
     if (err != cudaSuccess) return fail_cuda(err, "combine kernel");
   }
