@@ -60,8 +60,8 @@ def _bind(lib):
     lib.oracle_capacity.restype = I64
     lib.oracle_dispatch.argtypes = [P, I64, I32, I32, I64, P, P, P]
     lib.oracle_dispatch.restype = I64
-    lib.oracle_expert_rows.argtypes = [P, I32, P, P, P, I32, I64, I64, I64, P, P, I32, P]
-    lib.oracle_moe_tokens.argtypes = [P, I32, P, P, P, I32, I64, I64, I32, I64, P, P, P, P, I32, P, P, P, I32, P]
+    lib.oracle_expert_rows.argtypes = [P, I32, P, P, P, I32, I64, I64, I64, P, P, P]
+    lib.oracle_moe_tokens.argtypes = [P, I32, P, P, P, I32, I64, I64, I32, I64, P, P, P, P, I32, P, P, P, P]
     return lib
 
 
@@ -241,7 +241,7 @@ def dispatch(idx: np.ndarray, E: int, cap: int = -1):
     return offsets, perm[:int(offsets[E])].copy(), inv, int(dropped)
 
 
-def expert_rows(x, w_gate, w_up, w_down, tok, expert, h_round: bool = False) -> np.ndarray:
+def expert_rows(x, w_gate, w_up, w_down, tok, expert) -> np.ndarray:
     """``SwiGLU_e(x[t])`` in fp64 for each requested (token, expert) row."""
     lib = _load()
     xs, xdt = _as_stored(x)
@@ -254,16 +254,15 @@ def expert_rows(x, w_gate, w_up, w_down, tok, expert, h_round: bool = False) -> 
     expert = np.ascontiguousarray(expert, dtype=np.int32)
     n = tok.shape[0]
     y = np.empty((n, d), dtype=np.float64)
-    lib.oracle_expert_rows(_ptr(xs), xdt, _ptr(g), _ptr(u), _ptr(dn), dt, d, I, n, _ptr(tok), _ptr(expert),
-                           int(h_round), _ptr(y))
+    lib.oracle_expert_rows(_ptr(xs), xdt, _ptr(g), _ptr(u), _ptr(dn), dt, d, I, n, _ptr(tok), _ptr(expert), _ptr(y))
     return y
 
 
-def moe_tokens(x, w_gate, w_up, w_down, tok, idx, gate, h_round: bool = False, keep=None,
-               shared=None) -> np.ndarray:
+def moe_tokens(x, w_gate, w_up, w_down, tok, idx, gate, keep=None, shared=None) -> np.ndarray:
     """``out[i] = sum_j keep[i,j] gate[i,j] SwiGLU_{idx[i,j]}(x[tok[i]])
     + sum_s SharedSwiGLU_s(x[tok[i]])`` in fp64. ``shared`` is None or the
-    (gate [S,I,d], up [S,I,d], down [S,d,I]) weights of the shared experts."""
+    (gate [S,I,d], up [S,I,d], down [S,d,I]) weights of the shared experts;
+    ``idx``/``gate`` may have zero columns (shared experts alone)."""
     lib = _load()
     xs, xdt = _as_stored(x)
     g, dt = _as_stored(w_gate)
@@ -287,7 +286,7 @@ def moe_tokens(x, w_gate, w_up, w_down, tok, idx, gate, h_round: bool = False, k
         ns = 0
     out = np.empty((ntok, d), dtype=np.float64)
     lib.oracle_moe_tokens(_ptr(xs), xdt, _ptr(g), _ptr(u), _ptr(dn), dt, d, I, k, ntok, _ptr(tok), _ptr(idx),
-                          _ptr(gate), _ptr(kp), ns, _ptr(sg), _ptr(su), _ptr(sd), int(h_round), _ptr(out))
+                          _ptr(gate), _ptr(kp), ns, _ptr(sg), _ptr(su), _ptr(sd), _ptr(out))
     return out
 
 
@@ -312,8 +311,7 @@ class OracleResult:
     xhat: np.ndarray = None  # [T, d] fp64 normalised input, when a norm was applied
 
 
-def forward(x, w_router, b_router, w_gate, w_up, w_down, k: int, renorm: bool, tokens=None,
-            h_round: bool = False, *, norm_form: int = 0, norm_weight=None, norm_eps: float = 1e-5,
+def forward(x, w_router, b_router, w_gate, w_up, w_down, k: int, renorm: bool, tokens=None, *, norm_form: int = 0, norm_weight=None, norm_eps: float = 1e-5,
             capacity_factor: float = 0.0, shared=None) -> OracleResult:
     """The whole layer. Routing, statistics and dispatch cover every token;
     the expert output is evaluated for ``tokens`` (all tokens if None).
@@ -338,7 +336,6 @@ def forward(x, w_router, b_router, w_gate, w_up, w_down, k: int, renorm: bool, t
         tokens = np.arange(T, dtype=np.int32)
     tokens = np.asarray(tokens, dtype=np.int32)
     keep = (inv[tokens] >= 0) if cap >= 0 else None
-    out = moe_tokens(xin, w_gate, w_up, w_down, tokens, idx[tokens], gate[tokens], h_round=h_round, keep=keep,
-                     shared=shared)
+    out = moe_tokens(xin, w_gate, w_up, w_down, tokens, idx[tokens], gate[tokens], keep=keep, shared=shared)
     return OracleResult(probs, idx, gate, gap, counts, mean_prob, aux, offsets, perm, inv, tokens, out,
                         logits=logits, z_loss=z_loss(logits), capacity=cap, dropped=dropped, xhat=xhat)

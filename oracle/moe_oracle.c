@@ -328,12 +328,10 @@ int64_t oracle_dispatch(const int32_t* topk_idx, int64_t T, int k, int E, int64_
 /* ---- expert SwiGLU MLP ---------------------------------------------------- */
 
 /* y[r, :] = down_e(SiLU(gate_e(x_t)) * up_e(x_t)) for each requested row
- * (t = tok[r], e = expert[r]); x is read as x_dtype, the weights as dtype.
- * h_round = 1 rounds the hidden activation to
- * bf16 (a diagnostic mode; the parity bars use h_round = 0). */
+ * (t = tok[r], e = expert[r]); x is read as x_dtype, the weights as dtype. */
 void oracle_expert_rows(const void* x, int x_dtype, const void* w_gate, const void* w_up, const void* w_down,
                         int dtype, int64_t d, int64_t I, int64_t n, const int32_t* tok,
-                        const int32_t* expert, int h_round, double* y) {
+                        const int32_t* expert, double* y) {
 #pragma omp parallel
   {
     double* xv = (double*)malloc(sizeof(double) * (size_t)d);
@@ -352,7 +350,6 @@ void oracle_expert_rows(const void* x, int x_dtype, const void* w_gate, const vo
         }
         double silu = g / (1.0 + exp(-g));
         h[i] = silu * u;
-        if (h_round) h[i] = round_to_bf16(h[i]);
       }
       for (int64_t o = 0; o < d; ++o) {
         const int64_t wrow = (e * d + o) * I;
@@ -376,7 +373,7 @@ void oracle_expert_rows(const void* x, int x_dtype, const void* w_gate, const vo
 void oracle_moe_tokens(const void* x, int x_dtype, const void* w_gate, const void* w_up, const void* w_down,
                        int dtype, int64_t d, int64_t I, int k, int64_t ntok, const int32_t* tok,
                        const int32_t* idx, const double* gate, const int8_t* keep, int n_shared,
-                       const void* s_gate, const void* s_up, const void* s_down, int h_round, double* out) {
+                       const void* s_gate, const void* s_up, const void* s_down, double* out) {
   const int64_t n = ntok * k;
   const int64_t ns = ntok * n_shared;
   int32_t* rtok = (int32_t*)malloc(sizeof(int32_t) * (size_t)(n > 0 ? n : 1));
@@ -386,13 +383,13 @@ void oracle_moe_tokens(const void* x, int x_dtype, const void* w_gate, const voi
   double* ys = (double*)malloc(sizeof(double) * (size_t)(ns > 0 ? ns * d : 1));
   for (int64_t i = 0; i < ntok; ++i)
     for (int j = 0; j < k; ++j) rtok[i * k + j] = tok[i];
-  oracle_expert_rows(x, x_dtype, w_gate, w_up, w_down, dtype, d, I, n, rtok, idx, h_round, y);
+  oracle_expert_rows(x, x_dtype, w_gate, w_up, w_down, dtype, d, I, n, rtok, idx, y);
   for (int64_t i = 0; i < ntok; ++i)
     for (int s = 0; s < n_shared; ++s) {
       stok[i * n_shared + s] = tok[i];
       sexp[i * n_shared + s] = s;
     }
-  if (ns > 0) oracle_expert_rows(x, x_dtype, s_gate, s_up, s_down, dtype, d, I, ns, stok, sexp, h_round, ys);
+  if (ns > 0) oracle_expert_rows(x, x_dtype, s_gate, s_up, s_down, dtype, d, I, ns, stok, sexp, ys);
   for (int64_t i = 0; i < ntok; ++i)
     for (int64_t c = 0; c < d; ++c) {
       double acc = 0.0;

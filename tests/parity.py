@@ -12,27 +12,28 @@ Rules:
     checked against the oracle evaluated at the GPU's choice.
   * Counts and the dispatch order are checked exactly against the oracle's
     own dispatch of the GPU's indices (integer work is bit-exact).
-  * Gates within 2e-6 absolute for fp32 and 2e-5 for bf16, the statistic
-    within 1e-4 absolute. A gate is a softmax ratio of two or more logits,
-    |dg| <= max|dl| / 2, and the bf16 router accumulates its d products on the
-    tensor cores in fp32 (not round-to-nearest at every add), which leaves a
-    logit error of a few 1e-5 at d = 4096 (a relative 1e-6 of sum |x_c w_c|).
+  * Gates within GATE_TOL absolute, the statistic within 1e-4 absolute. A
+    gate is a softmax ratio of logits: with every logit off by at most dl,
+    |dp_j| = p_j |dl_j - sum_i p_i dl_i| <= 2 dl p_j (1 - p_j) <= dl / 2 (and
+    the same for a renormalised gate, a softmax over the k chosen logits).
+    So the gate bar is half the router's logit error bar plus the fp32
+    rounding of the softmax. The logit error bar of the bf16 router (fp32
+    tensor-core accumulation of d bf16 products) is pinned by
+    test_router_logit_error_pin, which reads the logits back from the gates
+    of a k = E call at d = 4096; the fp32 router adds its d FFMA products in
+    index order.
   * Outputs: max-abs <= 2e-2 and relative Frobenius <= 1e-2 for bf16;
-    both <= 1e-4 for fp32.
+    both <= 1e-4 for fp32; every token's output row is compared unless a
+    test names a subset.
   * Options. RMSNorm: the oracle normalises in fp64 and routes and evaluates
     the experts on x_hat. Capacity: the kept rows, inv (-1 for a dropped
     slot) and the dropped count are compared exactly with the oracle's
     capacity dispatch of the GPU's indices. Shared experts: part of the
-    output comparison. On the bf16 path with the norm or shared experts the
-    output bars are split: relative Frobenius <= 1e-2 against the pure fp64
-    oracle, and max-abs <= 2e-2 against the fp64 oracle that rounds the two
-    stored bf16 operands (x_hat and H) as the kernels store them. The
-    max-abs bar is an absolute bound set for the plain layer at the
-    benchmark workloads' shapes; x_hat is one more bf16 rounding and each shared
-    expert one more full expert output of weight 1, which at the Mixtral
-    prefill shape takes the pure-oracle max-abs to about 4e-2 while the
-    relative error stays below 3e-3. z-loss: relative error <= 1e-4 (each token's
-    logsumexp carries the router's logit error of a few 1e-5 and an fp32
+    output comparison. Every output bar is held against the pure fp64
+    oracle: relative Frobenius <= 1e-2 unchanged; the bf16 max-abs bar is
+    widened for the norm and the shared experts only by amounts the oracle
+    computes by itself (option_max_abs_bar). z-loss: relative error <= 1e-4
+    (each token's logsumexp carries the router's logit error and an fp32
     rounding; the per-block fp32 sums of at most 128 terms add at most
     128 * 2^-24 relative).
 """
@@ -45,7 +46,11 @@ import oracle
 
 GAP_THRESHOLD = 1e-4
 TOL = {"bf16": dict(max_abs=2e-2, rel_fro=1e-2), "f32": dict(max_abs=1e-4, rel_fro=1e-4)}
-GATE_TOL = {"bf16": 2e-5, "f32": 2e-6}
+# Router logit error bars (test_router_logit_error_pin measures them against
+# fp64); the gate bars follow from them (module docstring) plus a few fp32
+# roundings of values <= 1.
+LOGIT_TOL = {"bf16": 4e-5, "f32": 4e-6}
+GATE_TOL = {dt: LOGIT_TOL[dt] / 2 + 5e-7 for dt in LOGIT_TOL}
 Z_REL_TOL = 1e-4
 
 
@@ -53,10 +58,11 @@ def _np(t):
     return t.detach().cpu().numpy()
 
 
-def check(inp, res, perm, k, renorm, dtype, tokens=None, h_round=False, report=None, options=None):
+def check(inp, res, perm, k, renorm, dtype, tokens=None, report=None, options=None):
     """inp: workloads.Inputs (CUDA tensors); res: MoEOutputs; perm: (offsets,
-    perm_tok, inv) from get_permutation; tokens: sample of tokens whose output
-    rows are compared (None = all); options: the MoEOptions of the call."""
+    perm_tok, inv) from get_permutation; tokens: the tokens whose output rows
+    are compared (None, the default, compares every token); options: the
+    MoEOptions of the call."""
     x = inp.x.cpu()
     wr = inp.w_router.cpu()
     b = None if inp.b_router is None else inp.b_router.cpu()
@@ -147,7 +153,7 @@ def check(inp, res, perm, k, renorm, dtype, tokens=None, h_round=False, report=N
         rep["z_loss"] = z_g
         assert abs(z_g - z_o) <= Z_REL_TOL * abs(z_o) + 1e-7, f"z-loss {z_g} vs {z_o}"
 
-    # --- outputs -------------------------------------------------------------
+    # --- outputs ---------------------------------------------------------------
     if tokens is None:
         tokens = np.arange(T, dtype=np.int32)
     tokens = np.asarray(tokens, dtype=np.int32)
@@ -155,51 +161,63 @@ def check(inp, res, perm, k, renorm, dtype, tokens=None, h_round=False, report=N
     if tokens.size:
         keep = (inv_r[tokens] >= 0) if cap >= 0 else None
         wts = (inp.w_gate.cpu(), inp.w_up.cpu(), inp.w_down.cpu())
-        ref = oracle.moe_tokens(xin, *wts, tokens, idx_g[tokens], gate_ref[tokens], h_round=h_round, keep=keep,
-                                shared=shared)
+        # the pure fp64 layer: routed part and shared part evaluated apart
+        # (their sum is the layer's output up to the order of two fp64 adds)
+        routed = oracle.moe_tokens(xin, *wts, tokens, idx_g[tokens], gate_ref[tokens], keep=keep)
+        ref = routed
+        shared_part = None
+        if shared is not None:
+            shared_part = oracle.moe_tokens(xin, *wts, tokens, idx_g[tokens][:, :0], gate_ref[tokens][:, :0],
+                                            shared=shared)
+            ref = routed + shared_part
         got = _np(res.out)[tokens].astype(np.float64)
+        assert np.isfinite(got).all()
         diff = got - ref
         max_abs = float(np.abs(diff).max())
         rel_fro = float(np.linalg.norm(diff) / max(np.linalg.norm(ref), 1e-300))
         rep["max_abs"] = max_abs
         rep["rel_fro"] = rel_fro
         tol = TOL[dtype]
-        assert np.isfinite(got).all()
-        split_bars = dtype == "bf16" and options is not None and (options.norm_form or options.n_shared)
-        if dtype == "bf16" and not h_round:
-            norm_on = options is not None and options.norm_form
-            xr = oracle.round_bf16(xin) if norm_on else xin
-            ref_r = oracle.moe_tokens(xr, *wts, tokens, idx_g[tokens], gate_ref[tokens], h_round=True, keep=keep,
-                                      shared=shared)
-            max_abs_r = float(np.abs(got - ref_r).max())
-            rep["max_abs_vs_rounded_operands"] = max_abs_r
-        if split_bars:
-            assert max_abs_r <= tol["max_abs"], f"max-abs {max_abs_r} > {tol['max_abs']} ({rep})"
-        else:
-            assert max_abs <= tol["max_abs"], f"max-abs {max_abs} > {tol['max_abs']} ({rep})"
+        bar = tol["max_abs"]
+        if dtype == "bf16" and options is not None and (options.norm_form or options.n_shared):
+            bar = option_max_abs_bar(rep, xin, wts, tokens, idx_g[tokens], gate_ref[tokens], keep, shared,
+                                     routed, shared_part, options)
+        assert max_abs <= bar, f"max-abs {max_abs} > {bar} ({rep})"
         assert rel_fro <= tol["rel_fro"], f"relative Frobenius {rel_fro} > {tol['rel_fro']} ({rep})"
     return rep
 
 
-def sample_tokens(perm, T, k, n_random=64, edge=4, seed=0, cap=None):
-    """Tokens whose rows sit at the start and the ragged end of every expert's
-    segment (and of every 128-row tile boundary nearby), plus random ones."""
-    offs, perm_tok, _ = (_np(a) for a in perm)
-    pick = set()
-    rng = np.random.default_rng(seed)
-    for e in range(len(offs) - 1):
-        a, bnd = int(offs[e]), int(offs[e + 1])
-        if bnd <= a:
-            continue
-        for r in list(range(a, min(bnd, a + edge))) + list(range(max(a, bnd - edge), bnd)):
-            pick.add(int(perm_tok[r]))
-        for r in range(a + 127, bnd, 128):
-            pick.add(int(perm_tok[r]))
-            if r + 1 < bnd:
-                pick.add(int(perm_tok[r + 1]))
-    pick.update(rng.choice(T, size=min(T, n_random), replace=False).tolist())
-    pick.update([0, T - 1])
-    out = np.array(sorted(pick), dtype=np.int32)
-    if cap is not None and out.size > cap:
-        out = np.sort(rng.choice(out, size=cap, replace=False)).astype(np.int32)
-    return out
+def option_max_abs_bar(rep, xin, wts, tokens, idx, gate, keep, shared, routed, shared_part, options):
+    """Max-abs bar of the bf16 layer with the RMSNorm or shared experts,
+    derived from the oracle alone (nothing here mirrors the kernels).
+
+    The 2e-2 bar is stated for the plain layer, whose bf16 error comes from
+    rounding the stored bf16 operands of the expert GEMMs. Two options change
+    that error:
+      * shared experts add full expert outputs of weight 1. The rounding
+        error of an expert's output is relative to that output, and the
+        routed and shared parts' errors are independent, so the plain bar is
+        scaled by sqrt(1 + (rms shared / rms routed)^2), both RMS values taken
+        from the pure oracle over the compared rows;
+      * the normalised input x_hat of a bf16 layer is itself a bf16 tensor:
+        its one rounding moves the output by at most
+        A = max |oracle(bf16(x_hat)) - oracle(x_hat)| (same routing and gates,
+        everything else exact), which is added to the bar (triangle
+        inequality).
+    """
+    bar = TOL["bf16"]["max_abs"]
+    if shared_part is not None:
+        rr = float(np.sqrt(np.mean(routed ** 2)))
+        rs = float(np.sqrt(np.mean(shared_part ** 2)))
+        scale = float(np.sqrt(1.0 + (rs / max(rr, 1e-300)) ** 2))
+        rep["shared_scale"] = scale
+        bar *= scale
+    if options.norm_form:
+        xr = oracle.round_bf16(xin)
+        ref_r = oracle.moe_tokens(xr, *wts, tokens, idx, gate, keep=keep, shared=shared)
+        ref = routed if shared_part is None else routed + shared_part
+        allow = float(np.abs(ref_r - ref).max())
+        rep["xhat_allowance"] = allow
+        bar += allow
+    rep["max_abs_bar"] = bar
+    return bar
