@@ -119,12 +119,12 @@ def test_t0_with_options():
 
 @pytest.mark.parametrize("name", ["mixtral_prefill", "fine_grained"])
 def test_full_size_with_all_options(name):
-    """Full-size workload with the norm, two shared experts, a capacity of
-    1.25 and the z-loss, outputs compared on sampled tokens."""
+    """Full-size workload with the norm, shared experts (one at the Mixtral
+    shape, two at the fine-grained one), a capacity of 1.25 and the z-loss;
+    every token's output row is compared."""
     wl = WORKLOADS[name]
     opts = make_options(wl, 1, True, 2 if name == "fine_grained" else 1, 1.25, True)
     inp, res, perm = run(wl, opts, seed=0)
-    tokens = parity.sample_tokens(perm, wl.T, wl.k, n_random=24, edge=2, cap=48)
-    rep = parity.check(inp, res, perm, wl.k, wl.renorm, wl.dtype, tokens=tokens, options=opts)
+    rep = parity.check(inp, res, perm, wl.k, wl.renorm, wl.dtype, options=opts)
     print(f"\n[{wl.name}+options] {rep}")
     assert np.isfinite(rep["max_abs"])
