@@ -86,12 +86,27 @@ def load_traffic(workload, kernel):
 
 # ------------------------------------------------------------ algorithmic work
 
-def algorithmic(wl, counts, opts=None):
-    """Algorithmic FLOPs and DRAM bytes per launch of each kernel (the minimum
-    traffic: every input read once, every output written once). Rows are the
-    kept assignments (all of them without a capacity) plus T per shared
-    expert."""
+def plan_of(wl, opts=None):
+    """The library's launch plan for this workload and options (MOE_PLAN_*
+    bits of include/moe.h: which kernels are merged)."""
+    from sparse_mixture_experts_renorm_b200 import launch_plan
+
     o = opts or {}
+    return launch_plan(wl.T, wl.d, wl.E, wl.k, wl.I, wl.torch_dtype, n_shared=o.get("shared", 0),
+                       norm_form=o.get("norm", 0), norm_weight=bool(o.get("norm", 0)))
+
+
+def algorithmic(wl, counts, opts=None):
+    """Algorithmic FLOPs and DRAM bytes per launch of each kernel slot (the
+    minimum traffic: every input read once, every output written once). Rows
+    are the kept assignments (all of them without a capacity) plus T per
+    shared expert. Where the library merges kernels (plan_of), the merged
+    kernel's slot carries the work of both and the other slot none; an
+    intermediate that stays between the merged steps (H) is not counted."""
+    from sparse_mixture_experts_renorm_b200 import _binding as B
+
+    o = opts or {}
+    plan = plan_of(wl, o)
     T, d, E, k, I = wl.T, wl.d, wl.E, wl.k, wl.I
     S = o.get("shared", 0)
     counts = np.asarray(counts)
@@ -108,30 +123,78 @@ def algorithmic(wl, counts, opts=None):
     scan = dict(flops=0.0, bytes=nb * E * 12 + (E + 1) * 8 + E * 4)
     xrows = kept + (T if S else 0)
     gate_up = dict(flops=4.0 * R * d * I, bytes=2 * used * I * d * el + R * d * el + R * I * el)
-    if not fused_combine(wl, S):
-        return {
+    if not plan & B.MOE_PLAN_FUSED_COMBINE:
+        work = {
             "router_topk": router, "route_scan": scan,
             "permute": dict(flops=0.0, bytes=T * d * el + xrows * d * el + T * k * 12),
             "grouped_gemm_gateup_swiglu": gate_up,
             "grouped_gemm_down": dict(flops=2.0 * R * d * I, bytes=used * d * I * el + R * I * el + R * d * 4),
             "combine": dict(flops=2.0 * R * d, bytes=R * d * 4 + T * d * 4 + T * k * 8),
         }
-    return {
-        "router_topk": router, "route_scan": scan,
-        "permute": dict(flops=0.0, bytes=T * d * el + xrows * d * el + T * k * 16 + T * d * 4),
-        "grouped_gemm_gateup_swiglu": gate_up,
-        # down projection with the combine folded in: weights, H, and the fp32
-        # output accumulated in place (read + write)
-        "grouped_gemm_down": dict(flops=2.0 * R * d * I + 2.0 * R * d,
-                                  bytes=used * d * I * el + R * I * el + 2 * T * d * 4 + R * 8),
-        "combine": dict(flops=0.0, bytes=0),
-    }
+    else:
+        work = {
+            "router_topk": router, "route_scan": scan,
+            "permute": dict(flops=0.0, bytes=T * d * el + xrows * d * el + T * k * 16 + T * d * 4),
+            "grouped_gemm_gateup_swiglu": gate_up,
+            # down projection with the combine folded in: weights, H, and the fp32
+            # output accumulated in place (read + write)
+            "grouped_gemm_down": dict(flops=2.0 * R * d * I + 2.0 * R * d,
+                                      bytes=used * d * I * el + R * I * el + 2 * T * d * 4 + R * 8),
+            "combine": dict(flops=0.0, bytes=0),
+        }
+    if plan & B.MOE_PLAN_FUSED_SCAN:
+        rt, sc = work["router_topk"], work["route_scan"]
+        work["router_topk"] = dict(flops=rt["flops"], bytes=rt["bytes"] + sc["bytes"])
+        work["route_scan"] = dict(flops=0.0, bytes=0)
+    if plan & B.MOE_PLAN_FUSED_GEMMS:
+        gu, dn = work["grouped_gemm_gateup_swiglu"], work["grouped_gemm_down"]
+        work["grouped_gemm_gateup_swiglu"] = dict(flops=gu["flops"] + dn["flops"],
+                                                  bytes=gu["bytes"] + dn["bytes"] - 2 * R * I * el)
+        work["grouped_gemm_down"] = dict(flops=0.0, bytes=0)
+    return work
 
 
 def fused_combine(wl, n_shared=0):
-    """k = 2 on the bf16 path without shared experts: the combine runs inside
-    the down GEMM's epilogue."""
-    return wl.dtype == "bf16" and wl.k == 2 and n_shared == 0
+    """The combine runs inside the down GEMM's epilogue (the library's plan:
+    k = 2 on the bf16 path without shared experts)."""
+    from sparse_mixture_experts_renorm_b200 import _binding as B
+
+    return bool(plan_of(wl, {"shared": n_shared}) & B.MOE_PLAN_FUSED_COMBINE)
+
+
+def fused_gemms(wl, n_shared=0):
+    """Both projections run in one kernel (the library's plan: bf16 batches of
+    at most 32 tokens)."""
+    from sparse_mixture_experts_renorm_b200 import _binding as B
+
+    return bool(plan_of(wl, {"shared": n_shared}) & B.MOE_PLAN_FUSED_GEMMS)
+
+
+def slot_names(wl, opts=None):
+    """Names of the kernel slots of one call, merged kernels marked."""
+    from sparse_mixture_experts_renorm_b200 import _binding as B
+
+    plan = plan_of(wl, opts)
+    names = list(KERNELS)
+    if plan & B.MOE_PLAN_FUSED_SCAN:
+        names[0] = "router_topk (with the routing scan)"
+        names[1] = "route_scan (in router_topk)"
+    if plan & B.MOE_PLAN_FUSED_GEMMS:
+        names[3] = "grouped_gemm_gateup_down (both projections)"
+        names[4] = "grouped_gemm_down (in the fused kernel)"
+    if plan & B.MOE_PLAN_FUSED_COMBINE:
+        names[5] = "combine (in grouped_gemm_down)"
+    return names
+
+
+def launches_per_step(wl, opts=None):
+    """Kernels one call launches."""
+    from sparse_mixture_experts_renorm_b200 import _binding as B
+
+    plan = plan_of(wl, opts)
+    return (B.MOE_NUM_KERNELS - (1 if plan & B.MOE_PLAN_FUSED_COMBINE else 0)
+            - (1 if plan & B.MOE_PLAN_FUSED_GEMMS else 0) - (1 if plan & B.MOE_PLAN_FUSED_SCAN else 0)
+            + (1 if plan & B.MOE_PLAN_ROUTER_WEIGHT_SPLIT else 0))
 
 
 # --------------------------------------------------------------------- clocks
@@ -309,13 +372,272 @@ def config_of(wl, n_gpus, opts=None, n_shared=0):
 
 # ------------------------------------------------------------------------ ours
 
+NOMINAL_HBM_GBS = 8000.0  # nominal HBM3e bandwidth of a B200 (context for the decode target)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # FFMA peak: SMs x fp32 lanes x 2 FLOP x max SM clock
+
+
+class NvmlClockSampler:
+    """Samples the SM clock, the power draw and the clock-event reasons of one
+    GPU through NVML from a background thread every `period_s` (reads only),
+    so that regions of a few tens of milliseconds still get many samples.
+    Falls back to `nvidia-smi` sampling if NVML is unavailable."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, device, period_s=0.002):
+        import threading
+
+        self.samples = []
+        self.fallback = None
+        self.stop_flag = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device)
+            bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.nv = pynvml
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self.nv = None
+            self.fallback = ClockSampler(device)
+            return
+        self.period = period_s
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_flag:
+            t = time.time()
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1e3
+                self.samples.append((t, float(sm), int(rs), float(pw)))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def stop(self, t0, t1):
+        if self.nv is None:
+            return self.fallback.stop(t0, t1)
+        time.sleep(0.01)
+        self.stop_flag = True
+        self.thread.join(timeout=2)
+        sel = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not sel:
+            near = sorted(self.samples, key=lambda s: abs(s[0] - 0.5 * (t0 + t1)))
+            sel = near[:2]
+        reasons = sorted({nm for nm, bit in self.REASONS.items() for s in sel if s[2] & bit})
+        sm = [s[1] for s in sel]
+        pw = [s[3] for s in sel]
+        out = {"sm_mhz": float(np.median(sm)) if sm else None, "sm_min_mhz": min(sm) if sm else None,
+               "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(sel),
+               "power_w_max": max(pw) if pw else None, "sampler": "nvml, 2 ms"}
+        if "sw_power_cap" in reasons:
+            out["note"] = ("NVML reports the SM clock setting; under sw_power_cap the SMs run slower than it "
+                           "(in-kernel %clock64 against %globaltimer, measured apart from this run)")
+        return out
+
+
+def roofline_entry(wl, work, name, t_s, peaks, sustained):
+    """The roofline of one kernel (or of the whole step) at its algorithmic work."""
+    tc_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    hbm_peak = peaks["hbm_gbs"]
+    w = work
+    if wl.dtype != "bf16":
+        achieved = w["flops"] / t_s / 1e12
+        return {"bound": "alu", "achieved": achieved, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                "frac": achieved / FP32_ALU_TFLOPS, "kernel": name,
+                "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz (FFMA path)",
+                "algorithmic_per_launch": w["flops"]}
+    tensor_bound = (w["flops"] / (tc_peak * 1e12)) >= (w["bytes"] / (hbm_peak * 1e9))
+    if tensor_bound:
+        achieved = w["flops"] / t_s / 1e12
+        r = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s", "frac": achieved / tc_peak,
+             "peak_source": f"measured ({'sustained' if sustained else 'burst'} bf16)"}
+    else:
+        achieved = w["bytes"] / t_s / 1e9
+        r = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+             "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS, "peak_source": "measured (HBM copy)"}
+    r["kernel"] = name
+    r["algorithmic_per_launch"] = w["flops"] if tensor_bound else w["bytes"]
+    return r
+
+
+def step_work(wl, work):
+    """Algorithmic FLOPs and DRAM bytes of one whole step (every kernel)."""
+    return {"flops": sum(w["flops"] for w in work.values()), "bytes": sum(w["bytes"] for w in work.values())}
+
+
+def measure(wl, args, dev, world, rank, options=None, opts=None, with_e2e=True):
+    """Times K steps of the layer on workload `wl` (after W warm-up steps),
+    then the same K steps with per-kernel events, then (optionally) the
+    end-to-end host pipeline. Returns a dict of raw timings (max over ranks)."""
+    from sparse_mixture_experts_renorm_b200 import HostPipeline, MoELayer
+    from sparse_mixture_experts_renorm_b200 import _binding as B
+    from sparse_mixture_experts_renorm_b200 import parallel as par
+
+    n_shared = (opts or {}).get("shared", 0)
+    inp = make_inputs(wl, dev, seed=0)  # same weights on every rank
+    x = make_tokens(wl, wl.T, dev, seed=par.batch_seed(rank)) if world > 1 else inp.x
+    layer = MoELayer(inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k, wl.renorm, wl.T,
+                     options=options)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        layer(x)
+    torch.cuda.synchronize()
+    status = int(layer.status.item())
+    if status:
+        raise RuntimeError(f"{wl.name}: device status word {status:#x} after warm-up")
+
+    nk = B.MOE_NUM_KERNELS
+    flush = needs_flush(wl, n_shared)
+    scratch = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev) if flush else None
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps if flush else 0)]
+    sampler = NvmlClockSampler(dev)
+    time.sleep(0.5)  # both timed passes start from an idle GPU's power state
+    par.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        if flush:  # evict the weights, then time the step alone
+            scratch.fill_(float(i))
+            step_ev[i][0].record(stream)
+            layer(x)
+            step_ev[i][1].record(stream)
+        else:
+            layer(x)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    par.barrier()
+    clocks = sampler.stop(t_wall0, t_wall1)
+    local_ms = sum(a.elapsed_time(b) for a, b in step_ev) if flush else start.elapsed_time(stop)
+    ms = par.max_over_ranks(local_ms, dev)
+
+    # per-kernel device times: the same steps again, with an event recorded
+    # before each kernel and after the last
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
+    for row in evs:  # create the events outside the timed loop
+        for ev in row:
+            ev.record(stream)
+    torch.cuda.synchronize()
+    time.sleep(0.5)
+    for i in range(args.steps):
+        if flush:
+            scratch.fill_(float(i))
+        layer(x, events=evs[i])
+    torch.cuda.synchronize()
+    per_kernel = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(nk)] for i in range(args.steps)])
+    status = int(layer.status.item())
+    if status:
+        raise RuntimeError(f"{wl.name}: device status word {status:#x} after the timed region")
+
+    ms_e2e = None
+    e2e_steps = max(1, min(args.steps, 50))
+    if with_e2e:
+        # end to end through the library's host-memory pipeline (moe_pipeline_*
+        # of the C ABI): pinned x in, out + aux back, the copies of
+        # neighbouring steps overlapped with the compute
+        x_host = x.detach().to("cpu").pin_memory()
+        outs = [torch.empty((wl.T, wl.d), dtype=torch.float32).pin_memory() for _ in range(2)]
+        auxs = [torch.empty((1,), dtype=torch.float32).pin_memory() for _ in range(2)]
+        pipe = HostPipeline(layer)
+        for i in range(3):
+            pipe.submit(x_host, outs[i & 1], auxs[i & 1])
+        pipe.synchronize()
+        torch.cuda.synchronize()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        par.barrier()
+        torch.cuda.synchronize()
+        s2.record(pipe.stream(B.MOE_PIPELINE_COPY_IN))  # before the first batch's copy in
+        for i in range(e2e_steps):
+            pipe.submit(x_host, outs[i & 1], auxs[i & 1])
+        e2.record(pipe.stream(B.MOE_PIPELINE_COPY_OUT))  # after the last batch's copy out
+        pipe.synchronize()
+        torch.cuda.synchronize()
+        par.barrier()
+        ms_e2e = par.max_over_ranks(s2.elapsed_time(e2), dev)
+        pipe.close()
+
+    res = {"ms": ms, "clocks": clocks, "per_kernel": per_kernel, "counts": layer.counts.cpu().numpy(),
+           "ms_e2e": ms_e2e, "e2e_steps": e2e_steps, "x_bytes": int(x.numel() * x.element_size()),
+           "inp": inp if rank == 0 else None, "layer": layer}
+    return res
+
+
+def summarise(wl, args, world, r, opts=None):
+    """The JSON fields of one workload from the raw timings of measure()."""
+    from sparse_mixture_experts_renorm_b200 import parallel as par
+
+    opts = opts or {}
+    n_shared = opts.get("shared", 0)
+    ms = r["ms"]
+    counts = r["counts"]
+    work = algorithmic(wl, counts, opts)
+    tokens = par.job_tokens(wl.T, world, args.steps)
+    tok_s = tokens / (ms / 1e3)
+    # active FLOPs: the three projections of every computed row plus the router
+    rows = work["grouped_gemm_gateup_swiglu"]["flops"] / (4.0 * wl.d * wl.I)
+    step_flops = 6.0 * wl.d * wl.I * rows + 2.0 * wl.d * wl.E * wl.T
+    tflops = step_flops * world * args.steps / (ms / 1e3) / 1e12
+    peaks, peak_src = load_peaks()
+    # the sustained bf16 figure was measured over seconds under the 1 kW power
+    # cap: it applies to a timed region of a second or more; a shorter region
+    # is held to the burst figure (the stricter one), even when the power cap
+    # engaged inside it
+    sustained = ms / 1e3 >= 1.0
+    avg = r["per_kernel"].mean(axis=0)
+    kern = []
+    names = slot_names(wl, opts)
+    for j, name in enumerate(KERNELS):
+        w = work[name]
+        t_s = avg[j] / 1e3
+        kern.append({"name": names[j],
+                     "avg_us": float(avg[j] * 1e3), "share": float(avg[j] / avg.sum()),
+                     "tflops": w["flops"] / t_s / 1e12 if t_s > 0 else None,
+                     "gbs": w["bytes"] / t_s / 1e9 if t_s > 0 else None})
+    dom = int(np.argmax(avg))
+    dname = KERNELS[dom]
+    roof = roofline_entry(wl, work[dname], names[dom], avg[dom] / 1e3, peaks, sustained)
+    roof["traffic"] = load_traffic(wl.name, dname) if not opts else None
+    roof["peak_source"] = f"{peak_src}: {roof['peak_source']}"
+    if roof["bound"] == "tensor":
+        roof["frac_of_sustained"] = roof["achieved"] / peaks["bf16_tflops_sustained"]
+    step_roof = roofline_entry(wl, step_work(wl, work), "whole step", ms / 1e3 / args.steps, peaks, sustained)
+    step_roof.pop("kernel")
+    if step_roof["bound"] == "tensor":
+        step_roof["frac_of_sustained"] = step_roof["achieved"] / peaks["bf16_tflops_sustained"]
+    out = {
+        "workload": wl.name, "ms_per_step": ms / args.steps, "tokens_per_s": tok_s, "tflops_active": tflops,
+        "dtype": wl.dtype, "config": config_of(wl, world, opts or None, n_shared),
+        "roofline": roof, "step_roofline": step_roof, "kernels": kern, "clocks": r["clocks"],
+        "counts": counts.tolist() if wl.E <= 16 else {"max": int(counts.max()), "min": int(counts.min()),
+                                                      "mean": float(counts.mean())},
+        "gpu_launches": launches_per_step(wl, opts) * args.steps,
+    }
+    if r["ms_e2e"] is not None:
+        out["e2e"] = {"value": par.job_tokens(wl.T, world, r["e2e_steps"]) / (r["ms_e2e"] / 1e3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": r["x_bytes"], "d2h_bytes_per_step": int(wl.T * wl.d * 4 + 4)}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mixtral_prefill", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=None, choices=sorted(WORKLOADS),
+                    help="time this workload alone (default: mixtral_prefill as the headline, then every other "
+                         "workload under the line's 'workloads' key)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--norm", type=int, default=0, choices=[0, 1, 2],
@@ -325,15 +647,14 @@ def main():
     ap.add_argument("--zloss", action="store_true", help="also compute the router z-loss statistic")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
-    wl = WORKLOADS[args.workload]
+    headline = args.workload or "mixtral_prefill"
+    wl = WORKLOADS[headline]
 
     if args.impl == "reference":
         return run_reference(args, wl)
 
     import torch.distributed as dist
 
-    from sparse_mixture_experts_renorm_b200 import MoELayer
-    from sparse_mixture_experts_renorm_b200 import _binding as B
     from sparse_mixture_experts_renorm_b200 import parallel as par
 
     world, rank, local = par.env_ranks()
@@ -342,8 +663,6 @@ def main():
     if world > 1:
         par.init("nccl", 120.0, device=dev)
 
-    inp = make_inputs(wl, dev, seed=0)  # same weights on every rank
-    x = make_tokens(wl, wl.T, dev, seed=par.batch_seed(rank)) if world > 1 else inp.x
     opts = {}
     options = None
     if args.norm or args.shared or args.capacity > 0 or args.zloss:
@@ -359,159 +678,53 @@ def main():
             import math
 
             opts["cap"] = min(wl.T, int(math.ceil(args.capacity * wl.T * wl.k / wl.E)))
-    layer = MoELayer(inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k, wl.renorm, wl.T,
-                     options=options)
-    stream = torch.cuda.current_stream(dev)
-    barrier = par.barrier
 
-    for _ in range(args.warmup):
-        layer(x)
-    torch.cuda.synchronize()
-    status = int(layer.status.item())
-    if status:
-        raise RuntimeError(f"device status word {status:#x} after warm-up")
+    r = measure(wl, args, dev, world, rank, options, opts)
+    layer = r.pop("layer")
+    metric_extra = None
+    if opts:
+        metric_extra = {"z_loss": float(layer.z_loss.item()) if args.zloss else None,
+                        "dropped": int(layer.dropped.item()) if args.capacity > 0 else None}
+    del layer
+    head = summarise(wl, args, world, r, opts)
+    inp = r.pop("inp")
 
-    nk = B.MOE_NUM_KERNELS
-    sampler = ClockSampler(dev)
-    time.sleep(0.3)
-    flush = needs_flush(wl, args.shared)
-    scratch = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev) if flush else None
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps if flush else 0)]
-    barrier()
-    torch.cuda.synchronize()
-    t_wall0 = time.time()
-    start.record(stream)
-    for i in range(args.steps):
-        if flush:  # evict the weights, then time the step alone
-            scratch.fill_(float(i))
-            step_ev[i][0].record(stream)
-            layer(x)
-            step_ev[i][1].record(stream)
-        else:
-            layer(x)
-    stop.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    t_wall1 = time.time()
-    clocks = sampler.stop(t_wall0, t_wall1)
-    local_ms = sum(a.elapsed_time(b) for a, b in step_ev) if flush else start.elapsed_time(stop)
-    ms = par.max_over_ranks(local_ms, dev)
+    # the other workloads, each with its own warm-up, timed region, per-kernel
+    # events and clocks (same K and W), when no single workload was asked for
+    others = []
+    if args.workload is None and not opts:
+        for name in ("mixtral_decode", "fine_grained", "small_bf16", "tiny_f32"):
+            torch.cuda.empty_cache()
+            ro = measure(WORKLOADS[name], args, dev, world, rank)
+            ro.pop("layer")
+            ro.pop("inp")
+            others.append(summarise(WORKLOADS[name], args, world, ro))
+            del ro
+            torch.cuda.empty_cache()
 
-    # ---- per-kernel device times: the same steps again, with an event recorded
-    # before each kernel and after the last (events between the kernels also
-    # stop the next kernel's set-up from overlapping the previous one's tail)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(args.steps)]
-    for row in evs:  # create the events outside the timed loop
-        for ev in row:
-            ev.record(stream)
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        if flush:
-            scratch.fill_(float(i))
-        layer(x, events=evs[i])
-    torch.cuda.synchronize()
-    per_kernel = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(nk)] for i in range(args.steps)])
-    status = int(layer.status.item())
-    if status:
-        raise RuntimeError(f"device status word {status:#x} after the timed region")
-
-    # ---- end to end through the host API: pinned x in, out + aux back, with
-    # the copies of neighbouring steps overlapped with the compute
-    from sparse_mixture_experts_renorm_b200 import HostPipeline
-
-    e2e_steps = max(1, min(args.steps, 50))
-    x_host = x.detach().to("cpu").pin_memory()
-    outs = [torch.empty((wl.T, wl.d), dtype=torch.float32).pin_memory() for _ in range(2)]
-    auxs = [torch.empty((1,), dtype=torch.float32).pin_memory() for _ in range(2)]
-    pipe = HostPipeline(layer)
-    for i in range(3):
-        pipe.submit(x_host, outs[i & 1], auxs[i & 1])
-    pipe.synchronize()
-    torch.cuda.synchronize()
-    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    s2.record(pipe.h2d)
-    for i in range(e2e_steps):
-        pipe.submit(x_host, outs[i & 1], auxs[i & 1])
-    e2.record(pipe.d2h)
-    pipe.synchronize()
-    torch.cuda.synchronize()
-    barrier()
-    ms_e2e = par.max_over_ranks(s2.elapsed_time(e2), dev)
-
-    counts = layer.counts.cpu().numpy()
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
         return 0
 
-    work = algorithmic(wl, counts, opts)
-    tokens = par.job_tokens(wl.T, world, args.steps)
-    tok_s = tokens / (ms / 1e3)
-    # active FLOPs: the three projections of every computed row plus the router
-    rows = work["grouped_gemm_gateup_swiglu"]["flops"] / (4.0 * wl.d * wl.I)
-    step_flops = 6.0 * wl.d * wl.I * rows + 2.0 * wl.d * wl.E * wl.T
-    tflops = step_flops * world * args.steps / (ms / 1e3) / 1e12
-    peaks, peak_src = load_peaks()
-    region_s = ms / 1e3
-    # the sustained bf16 figure was measured under the 1 kW power cap: use it
-    # when the timed region is long or the clocks show the cap engaged
-    sustained = region_s >= 1.0 or "sw_power_cap" in clocks.get("reasons", [])
-    tc_peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
-    hbm_peak = peaks["hbm_gbs"]
-    avg = per_kernel.mean(axis=0)
-    kern = []
-    for j, name in enumerate(KERNELS):
-        w = work[name]
-        t_s = avg[j] / 1e3
-        ent = {"name": name if not (name == "combine" and fused_combine(wl, args.shared))
-               else "combine (in grouped_gemm_down)",
-               "avg_us": float(avg[j] * 1e3), "share": float(avg[j] / avg.sum()),
-               "tflops": w["flops"] / t_s / 1e12 if t_s > 0 else None,
-               "gbs": w["bytes"] / t_s / 1e9 if t_s > 0 else None}
-        kern.append(ent)
-    dom = int(np.argmax(avg))
-    dname = KERNELS[dom]
-    w = work[dname]
-    t_dom = avg[dom] / 1e3
-    # which roof binds this kernel at its algorithmic work
-    tensor_bound = (w["flops"] / (tc_peak * 1e12)) >= (w["bytes"] / (hbm_peak * 1e9)) and wl.dtype == "bf16"
-    if tensor_bound:
-        achieved = w["flops"] / t_dom / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
-                "frac": achieved / tc_peak}
-    else:
-        achieved = w["bytes"] / t_dom / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak}
-    roof["kernel"] = dname
-    roof["traffic"] = load_traffic(wl.name, dname) if not opts else None
-    roof["peak_source"] = (f"{peak_src} ({'sustained' if sustained and tensor_bound else 'burst'}"
-                           f"{' bf16' if tensor_bound else ' HBM copy'})")
-    roof["algorithmic_per_launch"] = w["flops"] if tensor_bound else w["bytes"]
-
     line = {
-        "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "metric": METRIC, "value": head["tokens_per_s"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": wl.dtype, "data": "synthetic (seeded, random-init weights)",
-        "tflops_active": tflops,
-        "config": config_of(wl, world, opts, args.shared),
-        "roofline": roof,
-        "kernels": kern,
-        "e2e": {"value": par.job_tokens(wl.T, world, e2e_steps) / (ms_e2e / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": int(x.numel() * x.element_size()),
-                "d2h_bytes_per_step": int(wl.T * wl.d * 4 + 4)},
-        "gpu_launches": (nk - (1 if fused_combine(wl, args.shared) else 0)
-                         + (1 if args.norm and wl.dtype == "bf16" else 0)) * args.steps,
-        "clocks": clocks,
-        "counts": counts.tolist() if wl.E <= 16 else {"max": int(counts.max()), "min": int(counts.min()),
-                                                      "mean": float(counts.mean())},
+        "tflops_active": head["tflops_active"],
+        "config": head["config"],
+        "roofline": head["roofline"],
+        "step_roofline": head["step_roofline"],
+        "kernels": head["kernels"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
+        "counts": head["counts"],
     }
-    if opts:
-        line["metric_extra"] = {"z_loss": float(layer.z_loss.item()) if args.zloss else None,
-                                "dropped": int(layer.dropped.item()) if args.capacity > 0 else None}
+    if metric_extra:
+        line["metric_extra"] = metric_extra
+    if others:
+        line["workloads"] = [head] + others
     if world == 1 and not args.no_cpu_baseline and not opts:
         inp_cpu = inputs_to_cpu(inp)
         rate, n, dt, threads = cpu_oracle_rate(inp_cpu, wl, args.cpu_budget_s)

@@ -119,6 +119,8 @@ moe_status moe_forward(const void* x, const void* w_router, const float* b_route
  *   0 router_topk, 1 route_scan, 2 permute, 3 grouped_gemm_gateup_swiglu,
  *   4 grouped_gemm_down, 5 combine.
  * moe_kernel_name(i) returns the name (a static string; NULL out of range).
+ * Some shapes merge kernels (moe_launch_plan says which); a merged kernel's
+ * slot is then empty.
  */
 #define MOE_NUM_KERNELS 6
 const char* moe_kernel_name(int i);
@@ -229,6 +231,27 @@ moe_status moe_forward_ex(const void* x, const void* w_router, const float* b_ro
                           int32_t* status_dev, void* stream, void* const* events, int n_events);
 
 /*
+ * moe_launch_plan — which kernels a call with this shape and these options
+ * (NULL: none) launches, as a bit set; -1 if the arguments are invalid (see
+ * moe_last_error_detail). Host only; launches nothing.
+ *   MOE_PLAN_FUSED_COMBINE: the combine runs in the down GEMM's epilogue
+ *     (bf16, k = 2, no shared experts): kernel 5 is not launched.
+ *   MOE_PLAN_FUSED_GEMMS: both projections run in one persistent kernel
+ *     (bf16, 1 <= T <= 32, where the GEMMs stream the weights from HBM):
+ *     slot 3 times both, slot 4 is empty.
+ *   MOE_PLAN_ROUTER_WEIGHT_SPLIT: a small kernel splits w * W_r into two
+ *     bf16 terms before the router (bf16 RMSNorm with a weight); its time
+ *     falls in slot 0.
+ *   MOE_PLAN_FUSED_SCAN: the router does the routing scan itself (bf16,
+ *     1 <= T <= 128 tokens, one router block, E <= 16): slot 1 is empty.
+ */
+#define MOE_PLAN_FUSED_COMBINE 1
+#define MOE_PLAN_FUSED_GEMMS 2
+#define MOE_PLAN_ROUTER_WEIGHT_SPLIT 4
+#define MOE_PLAN_FUSED_SCAN 8
+int moe_launch_plan(int T, int d, int E, int k, int I, moe_dtype dtype, const moe_options* opt);
+
+/*
  * moe_forward_noalloc — moe_forward for callers that cannot allocate device
  * memory: the same layer, arguments and results, but the scratch lives in a
  * static array of MOE_NOALLOC_SCRATCH_BYTES inside the library's device image
@@ -261,6 +284,63 @@ moe_status moe_forward_noalloc(const void* x, const void* w_router, const float*
                                int T, int d, int E, int k, int I, int renorm, moe_dtype dtype,
                                float* out, int32_t* topk_idx, float* topk_gate, int32_t* counts,
                                float* aux, int32_t* status_dev, void* stream);
+
+/*
+ * moe_pipeline — the layer called repeatedly on batches that live in host
+ * memory, the end-to-end path of a serving loop: the pipeline copies batch
+ * i+1 in and batch i-1 out while batch i computes, on three streams (its own
+ * copy-in and copy-out streams, and the caller's compute stream). The pages
+ * have no counterpart (their layers take tensors already in place).
+ *
+ * moe_layer_desc describes the layer once: device weights as for
+ * moe_forward_ex, the shape and dtype, options (copied at create; NULL for
+ * none), the caller's workspace (moe_workspace_size[_ex] bytes), device
+ * buffers shared by every batch (topk_idx [T,k], topk_gate [T,k], counts [E]
+ * or NULL, status_dev [1] or NULL) and two device staging slots per batch
+ * tensor: x_dev[b] [T,d] in the dtype, out_dev[b] [T,d] fp32, aux_dev[b] [1]
+ * fp32. The library allocates no device memory; create makes two streams
+ * and six events, which destroy releases.
+ *
+ * moe_pipeline_submit(p, x_host, out_host, aux_host) enqueues one batch and
+ * returns without waiting: x_host [T,d] in the dtype, out_host [T,d] fp32,
+ * aux_host [1] fp32 or NULL, in host memory (pinned memory lets the copies
+ * overlap the compute; pageable memory works but serialises). The host
+ * buffers must stay untouched until moe_pipeline_synchronize returns; the
+ * topk_idx/topk_gate/counts buffers hold the last computed batch's values.
+ * moe_pipeline_stream(p, MOE_PIPELINE_COPY_IN | _COMPUTE | _COPY_OUT) gives
+ * the streams, for callers that order their own work or timing events
+ * against them. moe_pipeline_destroy synchronises, then frees.
+ */
+typedef struct moe_layer_desc {
+  size_t struct_bytes;          /* sizeof(moe_layer_desc) */
+  const void* w_router;         /* device [E, d] */
+  const float* b_router;        /* device [E] or NULL */
+  const void* w_gate;           /* device [E, I, d] */
+  const void* w_up;             /* device [E, I, d] */
+  const void* w_down;           /* device [E, d, I] */
+  int T, d, E, k, I, renorm;
+  moe_dtype dtype;
+  const moe_options* opt;       /* NULL: the plain layer */
+  void* workspace;
+  size_t workspace_bytes;
+  int32_t* topk_idx;            /* device [T, k] */
+  float* topk_gate;             /* device [T, k] */
+  int32_t* counts;              /* device [E] or NULL */
+  int32_t* status_dev;          /* device [1] or NULL */
+  void* x_dev[2];               /* device [T, d] dtype, one per slot */
+  float* out_dev[2];            /* device [T, d] fp32 */
+  float* aux_dev[2];            /* device [1] fp32 */
+} moe_layer_desc;
+
+typedef struct moe_pipeline moe_pipeline;
+#define MOE_PIPELINE_COPY_IN 0
+#define MOE_PIPELINE_COMPUTE 1
+#define MOE_PIPELINE_COPY_OUT 2
+moe_status moe_pipeline_create(const moe_layer_desc* desc, void* compute_stream, moe_pipeline** out);
+moe_status moe_pipeline_submit(moe_pipeline* p, const void* x_host, float* out_host, float* aux_host);
+moe_status moe_pipeline_synchronize(moe_pipeline* p);
+void* moe_pipeline_stream(const moe_pipeline* p, int which);
+moe_status moe_pipeline_destroy(moe_pipeline* p);
 
 /*
  * moe_selftest_wait_timeout — a diagnostic of the failure handling every

@@ -18,7 +18,7 @@ from . import _binding as B
 from ._binding import MoEError, load_library
 
 __all__ = ["MoEError", "MoEOptions", "MoEOutputs", "MoELayer", "HostPipeline", "moe_forward", "workspace_size",
-           "get_permutation", "load_library"]
+           "get_permutation", "launch_plan", "load_library"]
 
 
 def _dtype_code(t: torch.dtype) -> int:
@@ -83,6 +83,26 @@ def workspace_size(T: int, d: int, E: int, k: int, I: int, dtype: torch.dtype,
     if n == 0:
         raise MoEError(B.MOE_ERR_INVALID_ARG, B.last_error_detail(lib))
     return int(n)
+
+
+def launch_plan(T: int, d: int, E: int, k: int, I: int, dtype: torch.dtype, n_shared: int = 0,
+                norm_form: int = 0, norm_weight: bool = False) -> int:
+    """The library's launch plan for a call of this shape (``moe_launch_plan``:
+    MOE_PLAN_* bits saying which kernels are merged). A host-side query: the
+    weight pointers it passes are placeholders that nothing dereferences."""
+    lib = load_library()
+    o = B.moe_options()
+    o.struct_bytes = ctypes.sizeof(B.moe_options)
+    o.norm_form = int(norm_form)
+    o.norm_eps = 1e-5
+    o.norm_weight = 256 if norm_weight else None
+    o.n_shared = int(n_shared)
+    if n_shared:
+        o.shared_gate = o.shared_up = o.shared_down = 256
+    plan = lib.moe_launch_plan(T, d, E, k, I, _dtype_code(dtype), ctypes.byref(o))
+    if plan < 0:
+        raise MoEError(B.MOE_ERR_INVALID_ARG, B.last_error_detail(lib))
+    return int(plan)
 
 
 def _check_options(options: MoEOptions, x, E: int, I: int):
@@ -246,50 +266,81 @@ class MoELayer:
 
 
 class HostPipeline:
-    """Runs batches that live in pinned host memory through a ``MoELayer``
-    with the copies overlapped: batch i+1 is copied in and batch i-1 copied
-    out while batch i computes (two device buffers each for x and out, one
-    stream per direction). ``submit`` returns without synchronising; the
-    host output buffer may be read after ``synchronize``."""
+    """Runs batches that live in host memory through a ``MoELayer`` with the
+    library's native pipeline (``moe_pipeline_*`` in include/moe.h): batch
+    i+1 is copied in and batch i-1 copied out while batch i computes (two
+    device slots each for x, out and aux, allocated here with torch; one
+    stream per copy direction inside the library; compute on torch's
+    current stream). ``submit`` returns without synchronising; the host
+    output buffers may be read after ``synchronize``. Pinned host buffers
+    let the copies overlap."""
 
     def __init__(self, layer: "MoELayer"):
         self.layer = layer
+        lib = load_library()
         dev = layer.w_gate.device
         T, d = layer.T, layer.d
         self.x_dev = [torch.empty((T, d), dtype=layer.dtype, device=dev) for _ in range(2)]
         self.out_dev = [torch.empty((T, d), dtype=torch.float32, device=dev) for _ in range(2)]
         self.aux_dev = [torch.empty((1,), dtype=torch.float32, device=dev) for _ in range(2)]
         self.compute = torch.cuda.current_stream(dev)
-        self.h2d = torch.cuda.Stream(dev)
-        self.d2h = torch.cuda.Stream(dev)
-        self.in_ready = [torch.cuda.Event() for _ in range(2)]
-        self.computed = [torch.cuda.Event() for _ in range(2)]
-        self.out_free = [torch.cuda.Event() for _ in range(2)]
-        self.i = 0
+        desc = B.moe_layer_desc()
+        desc.struct_bytes = ctypes.sizeof(B.moe_layer_desc)
+        desc.w_router = layer.w_router.data_ptr()
+        desc.b_router = None if layer.b_router is None else layer.b_router.data_ptr()
+        desc.w_gate, desc.w_up, desc.w_down = layer.w_gate.data_ptr(), layer.w_up.data_ptr(), layer.w_down.data_ptr()
+        desc.T, desc.d, desc.E, desc.k, desc.I = T, d, layer.E, layer.k, layer.I
+        desc.renorm = int(bool(layer.renorm))
+        desc.dtype = _dtype_code(layer.dtype)
+        self._opt = None
+        if layer.options is not None:
+            o = layer.options
+            self._opt = o.to_c(dropped=layer.dropped if o.capacity_factor > 0 else None,
+                               z_loss=layer.z_loss if o.z_loss else None)
+            desc.opt = ctypes.pointer(self._opt)
+        desc.workspace = layer.workspace.data_ptr()
+        desc.workspace_bytes = layer.workspace.numel()
+        desc.topk_idx, desc.topk_gate = layer.topk_idx.data_ptr(), layer.topk_gate.data_ptr()
+        desc.counts, desc.status_dev = layer.counts.data_ptr(), layer.status.data_ptr()
+        for b in range(2):
+            desc.x_dev[b] = self.x_dev[b].data_ptr()
+            desc.out_dev[b] = self.out_dev[b].data_ptr()
+            desc.aux_dev[b] = self.aux_dev[b].data_ptr()
+        handle = ctypes.c_void_p()
+        B.check(lib.moe_pipeline_create(ctypes.byref(desc), ctypes.c_void_p(self.compute.cuda_stream),
+                                        ctypes.byref(handle)), lib)
+        self._lib = lib
+        self._p = handle
 
-    def submit(self, x_host, out_host, aux_host) -> None:
-        b = self.i & 1
+    def stream(self, which: int) -> torch.cuda.ExternalStream:
+        """One of the pipeline's streams (B.MOE_PIPELINE_COPY_IN / _COMPUTE /
+        _COPY_OUT), e.g. to record timing events on it."""
+        ptr = self._lib.moe_pipeline_stream(self._p, which)
+        return torch.cuda.ExternalStream(ptr, device=self.layer.w_gate.device)
+
+    def submit(self, x_host, out_host, aux_host=None) -> None:
         L = self.layer
-        if self.i >= 2:
-            self.h2d.wait_event(self.computed[b])  # x buffer b no longer read
-        with torch.cuda.stream(self.h2d):
-            self.x_dev[b].copy_(x_host, non_blocking=True)
-            self.in_ready[b].record(self.h2d)
-        self.compute.wait_event(self.in_ready[b])
-        if self.i >= 2:
-            self.compute.wait_event(self.out_free[b])  # out buffer b copied out
-        moe_forward(self.x_dev[b], L.w_router, L.b_router, L.w_gate, L.w_up, L.w_down, L.k, L.renorm,
-                    out=self.out_dev[b], topk_idx=L.topk_idx, topk_gate=L.topk_gate, counts=L.counts,
-                    aux=self.aux_dev[b], workspace=L.workspace, status=L.status,
-                    stream=self.compute.cuda_stream, options=L.options, z_loss=L.z_loss, dropped=L.dropped)
-        self.computed[b].record(self.compute)
-        self.d2h.wait_event(self.computed[b])
-        with torch.cuda.stream(self.d2h):
-            out_host.copy_(self.out_dev[b], non_blocking=True)
-            aux_host.copy_(self.aux_dev[b], non_blocking=True)
-            self.out_free[b].record(self.d2h)
-        self.i += 1
+        if tuple(x_host.shape) != (L.T, L.d) or x_host.dtype != L.dtype or x_host.device.type != "cpu" \
+                or not x_host.is_contiguous():
+            raise ValueError(f"x_host must be a contiguous host tensor [{L.T}, {L.d}] of {L.dtype}")
+        if tuple(out_host.shape) != (L.T, L.d) or out_host.dtype != torch.float32 \
+                or out_host.device.type != "cpu" or not out_host.is_contiguous():
+            raise ValueError(f"out_host must be a contiguous host float32 tensor [{L.T}, {L.d}]")
+        if aux_host is not None and (aux_host.numel() != 1 or aux_host.dtype != torch.float32
+                                     or aux_host.device.type != "cpu"):
+            raise ValueError("aux_host must be a host float32 tensor of one element")
+        B.check(self._lib.moe_pipeline_submit(self._p, _ptr(x_host), _ptr(out_host), _ptr(aux_host)), self._lib)
 
     def synchronize(self) -> None:
-        self.d2h.synchronize()
-        self.compute.synchronize()
+        B.check(self._lib.moe_pipeline_synchronize(self._p), self._lib)
+
+    def close(self) -> None:
+        if self._p is not None and self._p.value:
+            B.check(self._lib.moe_pipeline_destroy(self._p), self._lib)
+        self._p = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

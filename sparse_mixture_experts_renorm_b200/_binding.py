@@ -27,11 +27,13 @@ STATUS_NAMES = {
 
 EXPORTED = ("moe_workspace_size", "moe_forward", "moe_forward_events", "moe_kernel_name", "moe_get_permutation",
             "moe_last_error_detail", "moe_forward_noalloc", "moe_selftest_wait_timeout", "moe_workspace_size_ex",
-            "moe_forward_ex")
+            "moe_forward_ex", "moe_launch_plan", "moe_pipeline_create", "moe_pipeline_submit",
+            "moe_pipeline_synchronize", "moe_pipeline_stream", "moe_pipeline_destroy")
 MOE_NORM_NONE, MOE_NORM_RMS, MOE_NORM_RMS_EPS_OUTSIDE = 0, 1, 2
 MOE_MAX_SHARED = 8
 MOE_NOALLOC_SCRATCH_BYTES = 16 << 20
 MOE_NUM_KERNELS = 6
+MOE_PLAN_FUSED_COMBINE, MOE_PLAN_FUSED_GEMMS, MOE_PLAN_ROUTER_WEIGHT_SPLIT, MOE_PLAN_FUSED_SCAN = 1, 2, 4, 8
 
 
 class moe_options(ctypes.Structure):
@@ -49,6 +51,35 @@ class moe_options(ctypes.Structure):
         ("capacity_factor", ctypes.c_double),
         ("dropped", ctypes.c_void_p),
         ("z_loss", ctypes.c_void_p),
+    ]
+
+
+MOE_PIPELINE_COPY_IN, MOE_PIPELINE_COMPUTE, MOE_PIPELINE_COPY_OUT = 0, 1, 2
+
+
+class moe_layer_desc(ctypes.Structure):
+    """The C struct ``moe_layer_desc`` of include/moe.h (same field order and types)."""
+
+    _fields_ = [
+        ("struct_bytes", ctypes.c_size_t),
+        ("w_router", ctypes.c_void_p),
+        ("b_router", ctypes.c_void_p),
+        ("w_gate", ctypes.c_void_p),
+        ("w_up", ctypes.c_void_p),
+        ("w_down", ctypes.c_void_p),
+        ("T", ctypes.c_int), ("d", ctypes.c_int), ("E", ctypes.c_int), ("k", ctypes.c_int), ("I", ctypes.c_int),
+        ("renorm", ctypes.c_int),
+        ("dtype", ctypes.c_int),
+        ("opt", ctypes.POINTER(moe_options)),
+        ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t),
+        ("topk_idx", ctypes.c_void_p),
+        ("topk_gate", ctypes.c_void_p),
+        ("counts", ctypes.c_void_p),
+        ("status_dev", ctypes.c_void_p),
+        ("x_dev", ctypes.c_void_p * 2),
+        ("out_dev", ctypes.c_void_p * 2),
+        ("aux_dev", ctypes.c_void_p * 2),
     ]
 
 
@@ -87,6 +118,18 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     lib.moe_forward_ex.argtypes = ([P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, OPT, P, P, P, P, P, P, SZ, P,
                                     P, ctypes.POINTER(ctypes.c_void_p), I32])
     lib.moe_forward_ex.restype = I32
+    lib.moe_launch_plan.argtypes = [I32, I32, I32, I32, I32, I32, OPT]
+    lib.moe_launch_plan.restype = I32
+    lib.moe_pipeline_create.argtypes = [ctypes.POINTER(moe_layer_desc), P, ctypes.POINTER(ctypes.c_void_p)]
+    lib.moe_pipeline_create.restype = I32
+    lib.moe_pipeline_submit.argtypes = [P, P, P, P]
+    lib.moe_pipeline_submit.restype = I32
+    lib.moe_pipeline_synchronize.argtypes = [P]
+    lib.moe_pipeline_synchronize.restype = I32
+    lib.moe_pipeline_stream.argtypes = [P, I32]
+    lib.moe_pipeline_stream.restype = P
+    lib.moe_pipeline_destroy.argtypes = [P]
+    lib.moe_pipeline_destroy.restype = I32
     lib.moe_kernel_name.argtypes = [I32]
     lib.moe_kernel_name.restype = ctypes.c_char_p
     lib.moe_forward_noalloc.argtypes = [P, P, P, P, P, P, I32, I32, I32, I32, I32, I32, I32, P, P, P, P, P, P, P]

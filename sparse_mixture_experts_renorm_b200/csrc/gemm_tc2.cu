@@ -214,16 +214,60 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, int n_tiles, const in
 
 __device__ __forceinline__ float silu_f32(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
+// One GEMM of the kernel: its shared-expert groups, output width N (hidden
+// units for gate/up, features for down), reduction length K and output.
+struct GemmPhase {
+  SharedGroups sh;
+  int N, K;
+  void* out;
+};
+
+// Orders this thread's generic-proxy global accesses with its async-proxy
+// (TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Waits until *counter >= target (acquire at GPU scope), polling with a short
+// sleep, for at most limit_ns; on time-out MOE_DEV_TIMEOUT is OR-ed into the
+// status word and the CTA-wide abort flag raised. Returns false when giving up.
+__device__ __forceinline__ bool wait_counter_geq(const int32_t* counter, int target, volatile int* abort_flag,
+                                                 int32_t* status, uint64_t limit_ns) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+  if (v >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    __nanosleep(128);
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+    if (v >= target) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      atomicOr(status, MOE_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// kMode 0: gate/up only; 1: down only; 2: both in one persistent launch
+// (every gate/up tile, then every down tile; a down tile's producers wait
+// until all gate/up tiles of its token tile have stored their H rows, counted
+// in mt_done, so one projection's last round overlaps the other's first).
+// Maps: tmA0/tmA1 (W_gate/W_up, or W_down twice in mode 1), tmS0/tmS1 (the
+// shared experts' counterparts), tmB/tmBs (the B operand in 128- and 16-row
+// boxes); in mode 2 tmD/tmSD/tmH/tmHs are the down projection's.
 template <int kMode, int kSt, int kEw, int kBRows>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
     grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                             const __grid_constant__ CUtensorMap tmS0, const __grid_constant__ CUtensorMap tmS1,
                             const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBs,
+                            const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmSD,
+                            const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmHs,
                             const int32_t* __restrict__ offsets, const int32_t* __restrict__ mtile256, int E,
-                            const SharedGroups sh, int N, int K, void* __restrict__ out,
-                            const int32_t* __restrict__ perm_tok,
-                            const float* __restrict__ rgate, float* __restrict__ comb_out, int32_t* status,
-                            uint64_t limit_ns) {
+                            const GemmPhase p0, const GemmPhase p1, const int32_t* __restrict__ perm_tok,
+                            const float* __restrict__ rgate, float* __restrict__ comb_out,
+                            int32_t* __restrict__ mt_done, int32_t* status, uint64_t limit_ns) {
   using Cfg = Gemm2Cfg<kSt, kEw, kBRows>;
   constexpr int kBSlot = Cfg::kBSlotBytes;
   constexpr int kGroups = kEw / 4;  // groups of four epilogue warps (one per TMEM lane quarter each)
@@ -243,16 +287,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_off = reinterpret_cast<int*>(s_tmem + 4);  // [E+1]
   int* s_mt = s_off + (E + 1);                       // [G+1]
-  const int G = E + sh.n;                            // GEMM groups: routed, then shared experts
+  const int G = E + p0.sh.n;                         // GEMM groups: routed, then shared experts
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int cid = (int)cluster_id_x();
   const int ncl = (int)num_clusters_x();
-  // weight blocks per expert: 128 hidden units (gate + up rows) or 256 output features
-  const int n_wb = kMode == 0 ? (N + 127) / 128 : (N + 255) / 256;
-  const int KB = K / kBK;
+  // weight blocks per expert: 128 hidden units (gate + up rows) or 256 output
+  // features; phase 1 exists in mode 2 only
+  const int n_wb0 = kMode == 1 ? (p0.N + 255) / 256 : (p0.N + 127) / 128;
+  const int n_wb1 = kMode == 2 ? (p1.N + 255) / 256 : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSt; ++s) {
@@ -269,12 +314,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA0);
-    if (kMode == 0) tma_prefetch_desc(&tmA1);
+    if (kMode != 1) tma_prefetch_desc(&tmA1);
     tma_prefetch_desc(&tmB);
     tma_prefetch_desc(&tmBs);
-    if (sh.n > 0) {
+    if (p0.sh.n > 0) {
       tma_prefetch_desc(&tmS0);
-      if (kMode == 0) tma_prefetch_desc(&tmS1);
+      if (kMode != 1) tma_prefetch_desc(&tmS1);
+    }
+    if (kMode == 2) {
+      tma_prefetch_desc(&tmD);
+      tma_prefetch_desc(&tmH);
+      tma_prefetch_desc(&tmHs);
+      if (p0.sh.n > 0) tma_prefetch_desc(&tmSD);
     }
   }
   if (warp == 1) {
@@ -291,7 +342,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
   cluster_sync();  // the peer's barriers are initialised before any remote signal
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
-  const int total = s_mt[G] * n_wb;
+  const int total0 = s_mt[G] * n_wb0;          // tiles of the first (or only) GEMM
+  const int total = total0 + s_mt[G] * n_wb1;  // plus the down tiles in mode 2
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer --
@@ -301,8 +353,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
       int issued = 0;
       bool ok = true;
       for (int tile = cid; ok && tile < total; tile += ncl) {
-        const TileCoord tc = decode_tile(tile, n_wb, s_mt, G);
-        const GroupRows gr = group_rows(tc.e, s_off, E, sh);
+        const bool ph1 = kMode == 2 && tile >= total0;
+        const int mode = kMode == 2 ? (ph1 ? 1 : 0) : kMode;
+        const GemmPhase& P = ph1 ? p1 : p0;
+        const int KB = P.K / kBK;
+        const TileCoord tc = decode_tile(ph1 ? tile - total0 : tile, ph1 ? n_wb1 : n_wb0, s_mt, G);
+        const GroupRows gr = group_rows(tc.e, s_off, E, P.sh);
         const int ntok = min(256, gr.cnt - tc.m * 256);
         const int half = ((ntok + 15) & ~15) >> 1;  // token rows of B held by each CTA
         const bool small = half <= kSmallRows;
@@ -313,11 +369,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
           break;
         }
         const int brow = gr.in0 + tc.m * 256 + (int)rank * half;
-        const int arow =
-            kMode == 0 ? gr.widx * N + tc.n * 128 + (int)rank * 64 : gr.widx * N + tc.n * 256 + (int)rank * 128;
-        const CUtensorMap* mA0 = gr.shared ? &tmS0 : &tmA0;
-        const CUtensorMap* mA1 = gr.shared ? &tmS1 : &tmA1;
+        const int arow = mode == 0 ? gr.widx * P.N + tc.n * 128 + (int)rank * 64
+                                   : gr.widx * P.N + tc.n * 256 + (int)rank * 128;
+        const CUtensorMap* mA0 = ph1 ? (gr.shared ? &tmSD : &tmD) : (gr.shared ? &tmS0 : &tmA0);
+        const CUtensorMap* mA1 = ph1 ? mA0 : (gr.shared ? &tmS1 : &tmA1);
+        const CUtensorMap* mB = ph1 ? (small ? &tmHs : &tmH) : (small ? &tmBs : &tmB);
         const uint32_t bytes = 2u * (uint32_t)(kHalfBytes + (small ? kSmallRows * 128 : kHalfBytes));
+        if (ph1) {
+          // the H rows of this token tile are complete once every epilogue
+          // warp of both CTAs of every gate/up tile over them has stored its
+          // part (one count per warp and tile)
+          if (!wait_counter_geq(mt_done + s_mt[tc.e] + tc.m, 2 * kEw * n_wb0, s_abort, status, limit_ns)) {
+            ok = false;
+            break;
+          }
+          fence_proxy_async_global();  // the TMA reads below see those generic-proxy stores
+        }
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, s_abort, status, limit_ns)) {
             ok = false;
@@ -325,14 +392,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
           }
           const uint32_t fbar = map_to_cta(&full[stage], 0);
           if (leader) mbar_arrive_expect_tx(&full[stage], bytes);
-          if (kMode == 0) {
+          if (mode == 0) {
             // rows 0-63: gate rows of this CTA's 64 hidden units, 64-127: up rows
             tma_load_2d_pair(sA + stage * kHalfBytes, mA0, fbar, kb * kBK, arow);
             tma_load_2d_pair(sA + stage * kHalfBytes + kHalfBytes / 2, mA1, fbar, kb * kBK, arow);
           } else {
             tma_load_2d_pair(sA + stage * kHalfBytes, mA0, fbar, kb * kBK, arow);
           }
-          tma_load_2d_pair(sB + stage * kBSlot, small ? &tmBs : &tmB, fbar, kb * kBK, brow);
+          tma_load_2d_pair(sB + stage * kBSlot, mB, fbar, kb * kBK, brow);
           ++issued;
           if (++stage == kSt) {
             stage = 0;
@@ -364,8 +431,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int tile = cid; ok && tile < total; tile += ncl) {
-        const TileCoord tc = decode_tile(tile, n_wb, s_mt, G);
-        const int ntok = min(256, group_rows(tc.e, s_off, E, sh).cnt - tc.m * 256);
+        const bool ph1 = kMode == 2 && tile >= total0;
+        const GemmPhase& P = ph1 ? p1 : p0;
+        const int KB = P.K / kBK;
+        const TileCoord tc = decode_tile(ph1 ? tile - total0 : tile, ph1 ? n_wb1 : n_wb0, s_mt, G);
+        const int ntok = min(256, group_rows(tc.e, s_off, E, P.sh).cnt - tc.m * 256);
         const int nt16 = (ntok + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(256, nt16);
         // narrow tiles spread their K loop over independent accumulators
@@ -414,8 +484,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = cid; tile < total; tile += ncl) {
-      const TileCoord tc = decode_tile(tile, n_wb, s_mt, G);
-      const GroupRows gr = group_rows(tc.e, s_off, E, sh);
+      const bool ph1 = kMode == 2 && tile >= total0;
+      const int mode = kMode == 2 ? (ph1 ? 1 : 0) : kMode;
+      const GemmPhase& P = ph1 ? p1 : p0;
+      const int N = P.N;
+      const TileCoord tc = decode_tile(ph1 ? tile - total0 : tile, ph1 ? n_wb1 : n_wb0, s_mt, G);
+      const GroupRows gr = group_rows(tc.e, s_off, E, P.sh);
       const int ntok = min(256, gr.cnt - tc.m * 256);
       const size_t row0 = static_cast<size_t>(gr.out0) + static_cast<size_t>(tc.m * 256);
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, s_abort, status, limit_ns))) break;
@@ -425,7 +499,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
       const int nt16 = (ntok + 15) & ~15;
       const int nacc = nt16 <= 64 ? 4 : (nt16 <= 128 ? 2 : 1);
       const int acc_stride = kBN / nacc;
-      if (kMode == 0) {
+      if (mode == 0) {
         // TMEM lanes 0-63 hold the gate rows, 64-127 the up rows of this
         // CTA's 64 hidden units. Per 32-token chunk both halves go to shared
         // memory; then every thread finishes 16 (token, unit) pairs and
@@ -457,7 +531,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
           epi_bar(half);
           const int tok = c * 32 + tt;
           if (tok < ntok && hid0 < N) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + (row0 + tok) * N + hid0 + ug);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(P.out) + (row0 + tok) * N + hid0 + ug);
             dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
           }
@@ -491,7 +565,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
                   red_add_v4(comb_out + (size_t)perm_tok[r] * N + o0 + vc, g * val.x, g * val.y, g * val.z,
                              g * val.w);
                 } else {
-                  *reinterpret_cast<float4*>(static_cast<float*>(out) + (row0 + tok) * N + o0 + vc) = val;
+                  *reinterpret_cast<float4*>(static_cast<float*>(P.out) + (row0 + tok) * N + o0 + vc) = val;
                 }
               }
             }
@@ -501,6 +575,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
       __syncwarp();
       tc_fence_before();
       mbar_arrive_cluster(acc == 0 ? tempty_leader0 : tempty_leader1);
+      if (kMode == 2 && !ph1) {
+        // this warp's H stores of the tile are done: count them for the down
+        // tiles that read these rows (release at GPU scope after the warp's
+        // stores; the readers acquire, then fence the async proxy)
+        fence_proxy_async_global();
+        __syncwarp();
+        if (lane == 0) {
+          asm volatile("fence.acq_rel.gpu;" ::: "memory");
+          atomicAdd(mt_done + s_mt[tc.e] + tc.m, 1);
+        }
+      }
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
@@ -548,23 +633,30 @@ int max_active_pairs(const void* kern) {
   }
 }
 
+// The tensor maps of one launch (see the kernel; unused ones repeat others).
+struct Tc2Maps {
+  CUtensorMap a0, a1, s0, s1, b, bs, d, sd, h, hs;
+};
+
 template <int kMode, class Cfg>
-cudaError_t launch_tc2_cfg(const CUtensorMap& tmA0, const CUtensorMap& tmA1, const CUtensorMap& tmS0,
-                           const CUtensorMap& tmS1, const CUtensorMap& tmB, const CUtensorMap& tmBs,
-                           const int32_t* offsets, const int32_t* mtile256, int R_rows, int E, const SharedGroups& sh,
-                           int N, int K, void* out, const int32_t* perm_tok, const float* rgate, float* comb_out,
-                           int32_t* status, cudaStream_t stream) {
+cudaError_t launch_tc2_cfg(const Tc2Maps& m, const int32_t* offsets, const int32_t* mtile256, int R_rows, int E,
+                           const GemmPhase& p0, const GemmPhase& p1, const int32_t* perm_tok, const float* rgate,
+                           float* comb_out, int32_t* mt_done, int32_t* status, cudaStream_t stream) {
   auto kern = grouped_gemm_tc2_kernel<kMode, Cfg::kStages, Cfg::kEpiWarps, Cfg::kBSlotRows>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (err != cudaSuccess) return err;
   const int pairs = max_active_pairs<Cfg>(reinterpret_cast<const void*>(kern));
   if (pairs <= 0) return cudaErrorInvalidConfiguration;
-  const int n_wb = kMode == 0 ? (N + 127) / 128 : (N + 255) / 256;
-  const long long max_tiles = (long long)(R_rows / 256 + E + sh.n) * n_wb;
+  const int n_wb0 = kMode == 1 ? (p0.N + 255) / 256 : (p0.N + 127) / 128;
+  const int n_wb1 = kMode == 2 ? (p1.N + 255) / 256 : 0;
+  const long long max_tiles = (long long)(R_rows / 256 + E + p0.sh.n) * (n_wb0 + n_wb1);
+  // mode 2 needs every cluster resident at once (a down tile waits for gate/up
+  // tiles of other clusters): never more clusters than fit on the GPU
   const int clusters = (int)(max_tiles < pairs ? max_tiles : pairs);
   if (clusters <= 0) return cudaSuccess;
-  return launch_pdl(kern, dim3(2 * clusters), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, tmA0, tmA1, tmS0, tmS1,
-                    tmB, tmBs, offsets, mtile256, E, sh, N, K, out, perm_tok, rgate, comb_out, status, kWaitLimitNs);
+  return launch_pdl(kern, dim3(2 * clusters), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, m.a0, m.a1, m.s0, m.s1,
+                    m.b, m.bs, m.d, m.sd, m.h, m.hs, offsets, mtile256, E, p0, p1, perm_tok, rgate, comb_out, mt_done,
+                    status, kWaitLimitNs);
 }
 
 // Batches whose every group has at most 32 rows (max_rows_per_group: T, the
@@ -574,20 +666,18 @@ cudaError_t launch_tc2_cfg(const CUtensorMap& tmA0, const CUtensorMap& tmA1, con
 // only with the combine folded in (its fp32 Y stores run better with fewer
 // epilogue warps and the deeper ring).
 template <int kMode>
-cudaError_t launch_tc2(const CUtensorMap& tmA0, const CUtensorMap& tmA1, const CUtensorMap& tmS0,
-                       const CUtensorMap& tmS1, const CUtensorMap& tmB, const CUtensorMap& tmBs, const int32_t* offsets,
-                       const int32_t* mtile256, int R_rows, int max_rows_per_group, int E, const SharedGroups& sh,
-                       int N, int K, void* out, const int32_t* perm_tok, const float* rgate, float* comb_out,
-                       int32_t* status, cudaStream_t stream) {
-  const bool wide = (long long)R_rows >= 64ll * (E + sh.n) && (kMode == 0 || comb_out != nullptr);
+cudaError_t launch_tc2(const Tc2Maps& m, const int32_t* offsets, const int32_t* mtile256, int R_rows,
+                       int max_rows_per_group, int E, const GemmPhase& p0, const int32_t* perm_tok,
+                       const float* rgate, float* comb_out, int32_t* status, cudaStream_t stream) {
+  const bool wide = (long long)R_rows >= 64ll * (E + p0.sh.n) && (kMode == 0 || comb_out != nullptr);
   if (max_rows_per_group <= 2 * kSmallRows)
-    return launch_tc2_cfg<kMode, Gemm2Stream>(tmA0, tmA1, tmS0, tmS1, tmB, tmBs, offsets, mtile256, R_rows, E, sh, N,
-                                              K, out, perm_tok, rgate, comb_out, status, stream);
+    return launch_tc2_cfg<kMode, Gemm2Stream>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate, comb_out,
+                                              nullptr, status, stream);
   if (wide)
-    return launch_tc2_cfg<kMode, Gemm2Wide>(tmA0, tmA1, tmS0, tmS1, tmB, tmBs, offsets, mtile256, R_rows, E, sh, N, K,
-                                            out, perm_tok, rgate, comb_out, status, stream);
-  return launch_tc2_cfg<kMode, Gemm2Narrow>(tmA0, tmA1, tmS0, tmS1, tmB, tmBs, offsets, mtile256, R_rows, E, sh, N, K,
-                                            out, perm_tok, rgate, comb_out, status, stream);
+    return launch_tc2_cfg<kMode, Gemm2Wide>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate, comb_out,
+                                            nullptr, status, stream);
+  return launch_tc2_cfg<kMode, Gemm2Narrow>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate, comb_out,
+                                            nullptr, status, stream);
 }
 
 }  // namespace
@@ -597,8 +687,9 @@ cudaError_t launch_gemm_gateup_tc2(const CUtensorMap& tm_wg, const CUtensorMap& 
                                    const int32_t* offsets, const int32_t* mtile, int R_rows, int E,
                                    const SharedGroups& sh, int I, int d, void* h, int32_t* status,
                                    cudaStream_t stream) {
-  return launch_tc2<0>(tm_wg, tm_wu, tm_sg, tm_su, tm_xp, tm_xp_small, offsets, mtile, R_rows, sh.rows, E, sh, I, d, h,
-                       nullptr, nullptr, nullptr, status, stream);
+  const Tc2Maps m{tm_wg, tm_wu, tm_sg, tm_su, tm_xp, tm_xp_small, tm_wg, tm_sg, tm_xp, tm_xp_small};
+  const GemmPhase p0{sh, I, d, h};
+  return launch_tc2<0>(m, offsets, mtile, R_rows, sh.rows, E, p0, nullptr, nullptr, nullptr, status, stream);
 }
 
 cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_wd, const CUtensorMap& tm_sd, const CUtensorMap& tm_h,
@@ -606,8 +697,26 @@ cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_wd, const CUtensorMap& tm
                                  int R_rows, int E, const SharedGroups& sh, int I, int d, float* y,
                                  const int32_t* perm_tok, const float* rgate, float* comb_out, int32_t* status,
                                  cudaStream_t stream) {
-  return launch_tc2<1>(tm_wd, tm_wd, tm_sd, tm_sd, tm_h, tm_h_small, offsets, mtile, R_rows, sh.rows, E, sh, d, I, y,
-                       perm_tok, rgate, comb_out, status, stream);
+  const Tc2Maps m{tm_wd, tm_wd, tm_sd, tm_sd, tm_h, tm_h_small, tm_wd, tm_sd, tm_h, tm_h_small};
+  const GemmPhase p0{sh, d, I, y};
+  return launch_tc2<1>(m, offsets, mtile, R_rows, sh.rows, E, p0, perm_tok, rgate, comb_out, status, stream);
+}
+
+bool gemms_fused(int T, moe_dtype dtype) { return dtype == MOE_BF16 && T > 0 && T <= 2 * kSmallRows; }
+
+cudaError_t launch_gemm_fused_tc2(const CUtensorMap& tm_wg, const CUtensorMap& tm_wu, const CUtensorMap& tm_sg,
+                                  const CUtensorMap& tm_su, const CUtensorMap& tm_xp_small, const CUtensorMap& tm_wd,
+                                  const CUtensorMap& tm_sd, const CUtensorMap& tm_h_small, const int32_t* offsets,
+                                  const int32_t* mtile, int R_rows, int E, const SharedGroups& sh_up,
+                                  const SharedGroups& sh_down, int I, int d, void* h, float* y,
+                                  const int32_t* perm_tok, const float* rgate, float* comb_out, int32_t* mt_done,
+                                  int32_t* status, cudaStream_t stream) {
+  // every group holds at most 32 rows, so the 16-row boxes serve every tile
+  const Tc2Maps m{tm_wg, tm_wu, tm_sg, tm_su, tm_xp_small, tm_xp_small, tm_wd, tm_sd, tm_h_small, tm_h_small};
+  const GemmPhase p0{sh_up, I, d, h};
+  const GemmPhase p1{sh_down, d, I, y};
+  return launch_tc2_cfg<2, Gemm2Stream>(m, offsets, mtile, R_rows, E, p0, p1, perm_tok, rgate, comb_out, mt_done,
+                                        status, stream);
 }
 
 }  // namespace moe

@@ -113,6 +113,9 @@ Workspace workspace_layout(int T, int d, int E, int k, int I, moe_dtype dtype, i
   w.rnorm = o;    o = align256(o + (norm ? 4 * (size_t)T : 0));
   w.wr_hi = o;    o = align256(o + (norm && dtype == MOE_BF16 ? 2 * (size_t)E * d : 0));
   w.wr_lo = o;    o = align256(o + (norm && dtype == MOE_BF16 ? 2 * (size_t)E * d : 0));
+  // token tiles of both GEMMs: at most (rows / 256) + one partial tile per group
+  w.n_mt = (R + (size_t)kMaxShared * T) / kTileM + (size_t)E + kMaxShared + 1;
+  w.mt_done = o;  o = align256(o + 4 * w.n_mt);
   w.total = o;
   return w;
 }
@@ -294,17 +297,32 @@ moe_status forward_impl(const void* x, const void* w_router, const float* b_rout
     if (err != cudaSuccess) return fail_cuda(err, "router weight split kernel");
   }
   float* blk_z = o.zloss ? reinterpret_cast<float*>(ws + w.blk_z) : nullptr;
+  const bool fused_gemms = gemms_fused(T, dtype);
+  int32_t* mt_done = fused_gemms ? reinterpret_cast<int32_t*>(ws + w.mt_done) : nullptr;
+  // a batch of one router block: the router also does the routing scan
+  const bool router_scan = router_does_scan(T, E, dtype);
+  RouterScan rs;
+  rs.counts = cnt;
+  rs.offsets = offsets;
+  rs.mtile = mtile;
+  rs.aux = aux_p;
+  rs.zloss = o.zloss;
+  rs.dropped = o.dropped;
+  rs.mt_done = mt_done;
+  rs.n_mt = mt_done ? (int)w.n_mt : 0;
+  rs.cap = cap;
+  rs.n_shared = o.n_shared;
   {
     NvtxRange r("router_topk");
     err = launch_router(dtype, x, w_router, b_router, T, d, E, k, renorm, rn, topk_idx, topk_gate, lrank, blk_cnt,
-                        blk_psum, blk_z, status, stream);
+                        blk_psum, blk_z, rs, status, stream);
   }
   if (err != cudaSuccess) return fail_cuda(err, "router kernel");
   marks.mark(stream);
-  {
+  if (!router_scan) {
     NvtxRange r("route_scan");
     err = launch_route_scan(router_blocks(T, dtype), T, E, k, cap, o.n_shared, blk_cnt, blk_psum, blk_z, cnt,
-                            offsets, mtile, aux_p, o.zloss, o.dropped, stream);
+                            offsets, mtile, aux_p, o.zloss, o.dropped, mt_done, (int)w.n_mt, stream);
   }
   if (err != cudaSuccess) return fail_cuda(err, "routing scan kernel");
   marks.mark(stream);
@@ -344,19 +362,32 @@ moe_status forward_impl(const void* x, const void* w_router, const float* b_rout
         !make_tmap_bf16_2d(&tm_h_s, h, (uint64_t)Rh, (uint64_t)I, 16))
       return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (driver entry point unavailable or bad pointer)");
     marks.mark(stream);
-    {
-      NvtxRange r("grouped_gemm_gateup_swiglu");
-      err = launch_gemm_gateup_tc2(tm_wg, tm_wu, tm_sg, tm_su, tm_xp, tm_xp_s, offsets, mtile, Rh, E, sh_up, I, d, h,
-                                   status, stream);
+    if (fused_gemms) {
+      // both projections in one launch (the down slot of the timing events
+      // is then empty)
+      {
+        NvtxRange r("grouped_gemm_gateup_down");
+        err = launch_gemm_fused_tc2(tm_wg, tm_wu, tm_sg, tm_su, tm_xp_s, tm_wd, tm_sd, tm_h_s, offsets, mtile, Rh, E,
+                                    sh_up, sh_down, I, d, h, y, perm_tok, rgate, fused_combine ? out : nullptr,
+                                    mt_done, status, stream);
+      }
+      if (err != cudaSuccess) return fail_cuda(err, "fused gate/up + down grouped GEMMs");
+      marks.mark(stream);
+    } else {
+      {
+        NvtxRange r("grouped_gemm_gateup_swiglu");
+        err = launch_gemm_gateup_tc2(tm_wg, tm_wu, tm_sg, tm_su, tm_xp, tm_xp_s, offsets, mtile, Rh, E, sh_up, I, d,
+                                     h, status, stream);
+      }
+      if (err != cudaSuccess) return fail_cuda(err, "gate/up grouped GEMM");
+      marks.mark(stream);
+      {
+        NvtxRange r("grouped_gemm_down");
+        err = launch_gemm_down_tc2(tm_wd, tm_sd, tm_h, tm_h_s, offsets, mtile, Rh, E, sh_down, I, d, y, perm_tok,
+                                   rgate, fused_combine ? out : nullptr, status, stream);
+      }
+      if (err != cudaSuccess) return fail_cuda(err, "down grouped GEMM");
     }
-    if (err != cudaSuccess) return fail_cuda(err, "gate/up grouped GEMM");
-    marks.mark(stream);
-    {
-      NvtxRange r("grouped_gemm_down");
-      err = launch_gemm_down_tc2(tm_wd, tm_sd, tm_h, tm_h_s, offsets, mtile, Rh, E, sh_down, I, d, y, perm_tok,
-                                 rgate, fused_combine ? out : nullptr, status, stream);
-    }
-    if (err != cudaSuccess) return fail_cuda(err, "down grouped GEMM");
   } else {
     marks.mark(stream);
     {
@@ -458,6 +489,18 @@ moe_status moe_forward_ex(const void* x, const void* w_router, const float* b_ro
   return forward_impl(x, w_router, b_router, w_gate, w_up, w_down, T, d, E, k, I, renorm, dtype, o, out, topk_idx,
                       topk_gate, counts, aux, workspace, workspace_bytes, status_dev, stream,
                       EventMarks{events, events ? MOE_NUM_KERNELS + 1 : 0});
+}
+
+int moe_launch_plan(int T, int d, int E, int k, int I, moe_dtype dtype, const moe_options* opt) {
+  if (check_shape(T, d, E, k, I, dtype) != MOE_OK) return -1;
+  Opts o;
+  if (parse_options(opt, T, d, k, I, &o) != MOE_OK) return -1;
+  int plan = 0;
+  if (dtype == MOE_BF16 && k == 2 && o.n_shared == 0) plan |= MOE_PLAN_FUSED_COMBINE;
+  if (gemms_fused(T, dtype)) plan |= MOE_PLAN_FUSED_GEMMS;
+  if (router_does_scan(T, E, dtype)) plan |= MOE_PLAN_FUSED_SCAN;
+  if (dtype == MOE_BF16 && o.norm_form != MOE_NORM_NONE && o.norm_w) plan |= MOE_PLAN_ROUTER_WEIGHT_SPLIT;
+  return plan;
 }
 
 const char* moe_kernel_name(int i) {

@@ -21,6 +21,7 @@ constexpr int kRouterTokensSimt = 32;
 constexpr int kRouterThreads = 256;
 constexpr int kMaxExperts = 256;
 constexpr int kMaxTopK = 8;
+constexpr int kRouterRegExperts = 16;  // up to this many experts the tensor-core router keeps logits in registers
 
 // tcgen05 grouped GEMM tiling.
 constexpr int kTileM = 256;       // dispatched tokens per tile of the CTA pair (UMMA N)
@@ -59,6 +60,8 @@ struct Workspace {
   size_t rnorm;       // fp32  [T]     RMSNorm scale of every token
   size_t wr_hi;       // bf16  [E, d]  high part of w * W_r (norm with a weight, bf16)
   size_t wr_lo;       // bf16  [E, d]  low part of w * W_r
+  size_t mt_done;     // int32 [n_mt]  per token tile: gate/up epilogue warps done (fused GEMMs)
+  size_t n_mt;        //               its length: an upper bound on the GEMMs' token tiles
   size_t total;
 };
 
@@ -119,15 +122,39 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 
 // ---- launchers (all asynchronous on `stream`) ----
 
+// The routing scan's outputs (see launch_route_scan), for a router that
+// computes them itself.
+struct RouterScan {
+  int32_t* counts = nullptr;
+  int32_t* offsets = nullptr;
+  int32_t* mtile = nullptr;
+  float* aux = nullptr;
+  float* zloss = nullptr;
+  int32_t* dropped = nullptr;
+  int32_t* mt_done = nullptr;
+  int n_mt = 0;
+  int cap = -1;
+  int n_shared = 0;
+};
+
+// A bf16 batch that fits one tensor-core router block (T <= 128) with at
+// most kRouterRegExperts experts: the router also does the routing scan, and
+// no scan kernel is launched.
+inline bool router_does_scan(int T, int E, moe_dtype dtype) {
+  return dtype == MOE_BF16 && T > 0 && T <= kRouterTokensTc && E <= kRouterRegExperts;
+}
+
 // blk_z (nullable): per-block sums of logsumexp(logits)^2 for the z-loss.
+// scan: where the scan's outputs go when router_does_scan (ignored otherwise).
 cudaError_t launch_router(moe_dtype dtype, const void* x, const void* w_router, const float* b_router, int T,
                           int d, int E, int k, int renorm, const RouterNorm& norm, int32_t* topk_idx,
                           float* topk_gate, int32_t* lrank, int32_t* blk_cnt, float* blk_psum, float* blk_z,
-                          int32_t* status, cudaStream_t stream);
+                          const RouterScan& scan, int32_t* status, cudaStream_t stream);
 
 cudaError_t launch_router_tc(const void* x, const void* w_router, const float* b_router, int T, int d, int E, int k,
                              int renorm, const RouterNorm& norm, int32_t* topk_idx, float* topk_gate, int32_t* lrank,
-                             int32_t* blk_cnt, float* blk_psum, float* blk_z, int32_t* status, cudaStream_t stream);
+                             int32_t* blk_cnt, float* blk_psum, float* blk_z, const RouterScan& scan,
+                             int32_t* status, cudaStream_t stream);
 
 // hi[e,c] + lo[e,c] = w[c] * W_r[e,c] (bf16 + bf16; the fp32 product is exact).
 cudaError_t launch_split_router_weight(const void* w_router, const void* norm_w, int E, int d, void* hi, void* lo,
@@ -136,9 +163,12 @@ cudaError_t launch_split_router_weight(const void* w_router, const void* norm_w,
 // cap < 0: no capacity. Writes counts (before dropping), offsets and the GEMM
 // tile prefix over the kept rows and the shared groups, aux, and optionally
 // the z-loss (from blk_z) and the dropped count.
+// mt_done (nullable): the fused GEMMs' per-token-tile counters, n_mt of them,
+// cleared here for the call.
 cudaError_t launch_route_scan(int nb, int T, int E, int k, int cap, int n_shared, int32_t* blk_cnt,
                               const float* blk_psum, const float* blk_z, int32_t* counts, int32_t* offsets,
-                              int32_t* mtile, float* aux, float* zloss, int32_t* dropped, cudaStream_t stream);
+                              int32_t* mtile, float* aux, float* zloss, int32_t* dropped, int32_t* mt_done, int n_mt,
+                              cudaStream_t stream);
 
 // Also records the gate of every dispatched row (rgate) and, when zero_out is
 // given, clears out[T, d] for a combine done by the down GEMM's epilogue.
@@ -176,6 +206,19 @@ cudaError_t launch_gemm_down_tc2(const CUtensorMap& tm_wd, const CUtensorMap& tm
                                  int R_rows, int E, const SharedGroups& sh, int I, int d, float* y,
                                  const int32_t* perm_tok, const float* rgate, float* comb_out, int32_t* status,
                                  cudaStream_t stream);
+
+// Both projections in one persistent launch (batches of at most 32 tokens,
+// where the GEMMs stream the weights): every gate/up tile, then every down
+// tile, a down tile starting once the gate/up tiles of its token tile are
+// stored (counted in mt_done, cleared by the routing scan).
+bool gemms_fused(int T, moe_dtype dtype);
+cudaError_t launch_gemm_fused_tc2(const CUtensorMap& tm_wg, const CUtensorMap& tm_wu, const CUtensorMap& tm_sg,
+                                  const CUtensorMap& tm_su, const CUtensorMap& tm_xp_small, const CUtensorMap& tm_wd,
+                                  const CUtensorMap& tm_sd, const CUtensorMap& tm_h_small, const int32_t* offsets,
+                                  const int32_t* mtile, int R_rows, int E, const SharedGroups& sh_up,
+                                  const SharedGroups& sh_down, int I, int d, void* h, float* y,
+                                  const int32_t* perm_tok, const float* rgate, float* comb_out, int32_t* mt_done,
+                                  int32_t* status, cudaStream_t stream);
 
 // fp32 SIMT grouped GEMMs (same groups as above; sw*: the shared weights).
 cudaError_t launch_gemm_gateup_simt(const float* xp, const float* wg, const float* wu, const float* swg,

@@ -282,7 +282,8 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int nb, int T, int E, 
                                                           const float* __restrict__ blk_z,
                                                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                                           int32_t* __restrict__ mtile, float* __restrict__ aux,
-                                                          float* __restrict__ zloss, int32_t* __restrict__ dropped) {
+                                                          float* __restrict__ zloss, int32_t* __restrict__ dropped,
+                                                          int32_t* __restrict__ mt_done, int n_mt) {
   __shared__ int s_cnt[1024];      // [slice][E] slice sums, then exclusive slice prefixes
   __shared__ double s_ps[1024];    // [slice][E] probability slice sums
   __shared__ int s_tot[kMaxExperts];
@@ -296,6 +297,8 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int nb, int T, int E, 
   const int chunk = (nb + S - 1) / S;
   const int b0 = min(nb, sl * chunk), b1 = min(nb, b0 + chunk);
   pdl_wait();
+  if (mt_done)  // the fused GEMMs' per-token-tile counters start from zero every call
+    for (int i = tid; i < n_mt; i += blockDim.x) mt_done[i] = 0;
   if (active) {
     int c = 0;
     double ps = 0.0;
@@ -402,11 +405,11 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(int nb, int T, int E, 
 
 cudaError_t launch_router(moe_dtype dtype, const void* x, const void* w_router, const float* b_router, int T, int d,
                           int E, int k, int renorm, const RouterNorm& norm, int32_t* topk_idx, float* topk_gate,
-                          int32_t* lrank, int32_t* blk_cnt, float* blk_psum, float* blk_z, int32_t* status,
-                          cudaStream_t stream) {
+                          int32_t* lrank, int32_t* blk_cnt, float* blk_psum, float* blk_z, const RouterScan& scan,
+                          int32_t* status, cudaStream_t stream) {
   if (dtype == MOE_BF16)
     return launch_router_tc(x, w_router, b_router, T, d, E, k, renorm, norm, topk_idx, topk_gate, lrank, blk_cnt,
-                            blk_psum, blk_z, status, stream);
+                            blk_psum, blk_z, scan, status, stream);
   const int nb = router_blocks(T, MOE_F32);
   const size_t smem = (size_t)kRouterTokensSimt * (E + 1) * sizeof(float);
   auto kern = E <= 32 ? router_kernel<1> : E <= 64 ? router_kernel<2> : E <= 128 ? router_kernel<4> : router_kernel<8>;
@@ -420,9 +423,10 @@ cudaError_t launch_router(moe_dtype dtype, const void* x, const void* w_router, 
 
 cudaError_t launch_route_scan(int nb, int T, int E, int k, int cap, int n_shared, int32_t* blk_cnt,
                               const float* blk_psum, const float* blk_z, int32_t* counts, int32_t* offsets,
-                              int32_t* mtile, float* aux, float* zloss, int32_t* dropped, cudaStream_t stream) {
+                              int32_t* mtile, float* aux, float* zloss, int32_t* dropped, int32_t* mt_done, int n_mt,
+                              cudaStream_t stream) {
   return launch_pdl(route_scan_kernel, dim3(1), dim3(1024), 0, stream, nb, T, E, k, cap, n_shared, blk_cnt, blk_psum,
-                    blk_z, counts, offsets, mtile, aux, zloss, dropped);
+                    blk_z, counts, offsets, mtile, aux, zloss, dropped, mt_done, n_mt);
 }
 
 }  // namespace moe

@@ -42,7 +42,7 @@ namespace moe {
 namespace {
 
 constexpr int kRB = kRouterTokensTc;  // 128 tokens per block
-constexpr int kRegE = 16;             // up to this many experts a token's logits stay in registers
+constexpr int kRegE = kRouterRegExperts;  // up to this many experts a token's logits stay in registers
 constexpr int kSplitE = 64;           // up to this many experts the K loop may be split over a cluster
 
 struct RouterCfg {
@@ -120,6 +120,60 @@ __device__ __forceinline__ void topk_insert(float (&bv)[kMaxTopK], int (&be)[kMa
   }
 }
 
+// The routing scan of a batch that is a single router block (E <= 32): warp
+// lanes are experts. Offsets and the GEMM tile prefix are inclusive shuffle
+// scans of the kept counts, the statistic and the dropped count xor-reduced
+// over the lanes in fp64, exactly as route_scan_kernel does for one block;
+// the block's base rows are the offsets themselves.
+__device__ __forceinline__ void single_block_scan(const RouterScan& sc, int T, int E, int k, int tot, float ps,
+                                                  float blk_zsum, int32_t* blk_cnt, int lane) {
+  const unsigned full = 0xffffffffu;
+  const bool has = lane < E;
+  if (!has) {
+    tot = 0;
+    ps = 0.f;
+  }
+  const int kept = sc.cap >= 0 ? min(tot, sc.cap) : tot;
+  const int tiles = (kept + kTileM - 1) / kTileM;
+  int ik = kept, it = tiles;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n1 = __shfl_up_sync(full, ik, o), n2 = __shfl_up_sync(full, it, o);
+    if (lane >= o) {
+      ik += n1;
+      it += n2;
+    }
+  }
+  double p = (double)ps;  // the probability sum of one block, widened as the scan does
+  double ae = has ? ((double)tot / ((double)T * (double)k)) * (p / (double)T) : 0.0;
+  int dr = tot - kept;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    ae += __shfl_xor_sync(full, ae, o);
+    dr += __shfl_xor_sync(full, dr, o);
+  }
+  if (has) {
+    const int off = ik - kept;
+    sc.offsets[lane] = off;
+    sc.mtile[lane] = it - tiles;
+    if (sc.counts) sc.counts[lane] = tot;
+    blk_cnt[lane] = off;  // base row of block 0
+  }
+  const int run = __shfl_sync(full, ik, 31), mt0 = __shfl_sync(full, it, 31);
+  if (lane == 0) {
+    sc.offsets[E] = run;
+    sc.mtile[E] = mt0;
+    int mt = mt0;
+    for (int s2 = 0; s2 < sc.n_shared; ++s2) {
+      mt += (T + kTileM - 1) / kTileM;
+      sc.mtile[E + 1 + s2] = mt;
+    }
+    if (sc.aux) *sc.aux = (float)((double)E * ae);
+    if (sc.dropped) *sc.dropped = dr;
+    if (sc.zloss) *sc.zloss = (float)((double)blk_zsum / (double)T);
+  }
+}
+
 // E <= kE: logits in registers (fully unrolled code); kE == 0: E > kRegE,
 // logits in shared memory and rolled loops (code executed once per block must
 // stay small: unrolled per-expert code for large E thrashes the instruction
@@ -132,7 +186,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                      int part_bytes, int tmem_cols, int norm_form, float norm_eps, float* __restrict__ rnorm,
                      int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate, int32_t* __restrict__ lrank,
                      int32_t* __restrict__ blk_cnt, float* __restrict__ blk_psum, float* __restrict__ blk_z,
-                     int32_t* status, uint64_t limit_ns) {
+                     const RouterScan scan, int32_t* status, uint64_t limit_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
@@ -483,6 +537,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     epi_bar();
     // block totals and the exclusive prefix over the 4 row quarters
+    int my_tot = 0;     // thread r < E: expert r's count in this block
+    float my_ps = 0.f;  //                and its probability sum
     for (int e = r; e < E; e += kRB) {
       int run = 0;
       for (int qq = 0; qq < 4; ++qq) {
@@ -500,8 +556,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         ps3 += s_p[(rr + 3) * ld + e];
       }
       blk_psum[(size_t)blk * E + e] = (ps0 + ps1) + (ps2 + ps3);
+      my_tot = run;
+      my_ps = (ps0 + ps1) + (ps2 + ps3);
     }
     if (blk_z && r == 0) blk_z[blk] = ((s_z[0] + s_z[1]) + s_z[2]) + s_z[3];
+    if (scan.offsets) {
+      // the whole batch is this one block: the routing scan's results follow
+      // from its counts directly (the same arithmetic and order as
+      // route_scan_kernel for one block), and no scan kernel runs
+      for (int i = r; i < scan.n_mt; i += kRB) scan.mt_done[i] = 0;
+      if (q == 0) single_block_scan(scan, T, E, k, my_tot, my_ps,
+                                    blk_z ? ((s_z[0] + s_z[1]) + s_z[2]) + s_z[3] : 0.f, blk_cnt, lane);
+    }
     epi_bar();
     if (valid) {
 #pragma unroll
@@ -709,7 +775,8 @@ int sm_count() {
 
 cudaError_t launch_router_tc(const void* x, const void* w_router, const float* b_router, int T, int d, int E, int k,
                              int renorm, const RouterNorm& norm, int32_t* topk_idx, float* topk_gate, int32_t* lrank,
-                             int32_t* blk_cnt, float* blk_psum, float* blk_z, int32_t* status, cudaStream_t stream) {
+                             int32_t* blk_cnt, float* blk_psum, float* blk_z, const RouterScan& scan,
+                             int32_t* status, cudaStream_t stream) {
   const bool split = norm.form != 0 && norm.w_hi != nullptr;
   const RouterCfg c = router_cfg(T, d, E, norm.form != 0, split, sm_count());
   CUtensorMap tmX, tmW, tmW2;
@@ -737,7 +804,8 @@ cudaError_t launch_router_tc(const void* x, const void* w_router, const float* b
   cfg.numAttrs = c.S > 1 ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, tmX, tmW, tmW2, b_router, T, d, E, k, renorm, c.npad, c.lo_col, split ? 1 : 0,
                             c.S, c.stages, c.stage_bytes, c.part_bytes, c.tmem_cols, norm.form, norm.eps, norm.rnorm,
-                            topk_idx, topk_gate, lrank, blk_cnt, blk_psum, blk_z, status, kWaitLimitNs);
+                            topk_idx, topk_gate, lrank, blk_cnt, blk_psum, blk_z,
+                            router_does_scan(T, E, MOE_BF16) ? scan : RouterScan{}, status, kWaitLimitNs);
 }
 
 namespace {

@@ -46,10 +46,15 @@ import oracle
 
 GAP_THRESHOLD = 1e-4
 TOL = {"bf16": dict(max_abs=2e-2, rel_fro=1e-2), "f32": dict(max_abs=1e-4, rel_fro=1e-4)}
-# Router logit error bars (test_router_logit_error_pin measures them against
-# fp64); the gate bars follow from them (module docstring) plus a few fp32
-# roundings of values <= 1.
-LOGIT_TOL = {"bf16": 4e-5, "f32": 4e-6}
+# Router logit error bars, set from test_router_logit_error_pin's
+# measurement against fp64 (largest of all tokens, read back through the
+# gates of a k = E call): 4.3e-6 for the bf16 tensor-core router at the
+# Mixtral prefill shape (d = 4096), 6.6e-7 at d = 1024, and 3.6e-6 for the
+# fp32 router on the tiny workload, whose router std of 0.5 gives logits of
+# std 5.7 (the read-back there includes the fp32 exponential of logit gaps
+# of up to ~20). The bars leave about 2.5x room. The gate bars follow from
+# them (module docstring) plus a few fp32 roundings of values <= 1.
+LOGIT_TOL = {"bf16": 1e-5, "f32": 1e-5}
 GATE_TOL = {dt: LOGIT_TOL[dt] / 2 + 5e-7 for dt in LOGIT_TOL}
 Z_REL_TOL = 1e-4
 

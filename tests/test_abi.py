@@ -24,7 +24,7 @@ def lib():
 def header_functions():
     text = open(os.path.join(ROOT, "include", "moe.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:size_t|moe_status|const char\s*\*)\s*(moe_\w+)\s*\(", text, flags=re.M)))
+    return sorted(set(re.findall(r"^\s*(?:size_t|moe_status|int|void\s*\*|const char\s*\*)\s*(moe_\w+)\s*\(", text, flags=re.M)))
 
 
 def test_header_declares_the_entry_points():
@@ -189,3 +189,53 @@ def test_forward_ex_event_count_is_checked(lib):
     st = lib.moe_forward_ex(fake, fake, None, fake, fake, fake, 64, 128, 4, 2, 128, 1, B.MOE_BF16, None,
                             fake, fake, fake, None, None, fake, 1 << 30, None, None, evs, 3)
     assert st == B.MOE_ERR_INVALID_ARG
+
+
+def test_launch_plan(lib):
+    """Which kernels a call merges: the combine into the down GEMM for bf16
+    k = 2 without shared experts; both projections into one kernel for bf16
+    batches of 1..32 tokens; the routing scan into the router for bf16
+    batches of one router block (1..128 tokens) with at most 16 experts; an
+    extra split of w * W_r for the bf16 norm with a weight; -1 for invalid
+    arguments."""
+    bf, f32 = B.MOE_BF16, B.MOE_F32
+    assert lib.moe_launch_plan(32, 4096, 8, 2, 14336, bf, None) == (B.MOE_PLAN_FUSED_COMBINE | B.MOE_PLAN_FUSED_GEMMS
+                                                                     | B.MOE_PLAN_FUSED_SCAN)
+    assert lib.moe_launch_plan(33, 4096, 8, 2, 14336, bf, None) == B.MOE_PLAN_FUSED_COMBINE | B.MOE_PLAN_FUSED_SCAN
+    assert lib.moe_launch_plan(129, 4096, 8, 2, 14336, bf, None) == B.MOE_PLAN_FUSED_COMBINE
+    assert lib.moe_launch_plan(100, 256, 17, 2, 256, bf, None) == B.MOE_PLAN_FUSED_COMBINE  # E > 16
+    assert lib.moe_launch_plan(4096, 4096, 8, 2, 14336, bf, None) == B.MOE_PLAN_FUSED_COMBINE
+    assert lib.moe_launch_plan(16384, 2048, 64, 6, 1408, bf, None) == 0
+    assert lib.moe_launch_plan(64, 128, 4, 2, 256, f32, None) == 0
+    assert lib.moe_launch_plan(0, 4096, 8, 2, 14336, bf, None) == B.MOE_PLAN_FUSED_COMBINE
+    o = B.moe_options()
+    o.struct_bytes = ctypes.sizeof(B.moe_options)
+    o.norm_form, o.norm_eps, o.norm_weight = B.MOE_NORM_RMS, 1e-5, 256
+    o.n_shared = 1
+    o.shared_gate = o.shared_up = o.shared_down = 256
+    assert lib.moe_launch_plan(32, 4096, 8, 2, 14336, bf, ctypes.byref(o)) == (B.MOE_PLAN_FUSED_GEMMS
+                                                                           | B.MOE_PLAN_ROUTER_WEIGHT_SPLIT
+                                                                           | B.MOE_PLAN_FUSED_SCAN)
+    assert lib.moe_launch_plan(32, 4096, 8, 9, 14336, bf, None) == -1  # k > E
+
+
+def test_pipeline_rejects_bad_arguments_before_any_cuda_call(lib):
+    """moe_pipeline_create validates its description on the host: a NULL
+    handle pointer or description, a short struct, an invalid shape and
+    missing device slots are refused before a stream or event is made."""
+    h = ctypes.c_void_p()
+    assert lib.moe_pipeline_create(None, None, ctypes.byref(h)) == B.MOE_ERR_INVALID_ARG
+    desc = B.moe_layer_desc()
+    desc.struct_bytes = ctypes.sizeof(B.moe_layer_desc)
+    assert lib.moe_pipeline_create(ctypes.byref(desc), None, None) == B.MOE_ERR_INVALID_ARG
+    desc.struct_bytes = 8
+    assert lib.moe_pipeline_create(ctypes.byref(desc), None, ctypes.byref(h)) == B.MOE_ERR_INVALID_ARG
+    desc.struct_bytes = ctypes.sizeof(B.moe_layer_desc)
+    desc.T, desc.d, desc.E, desc.k, desc.I, desc.renorm, desc.dtype = 32, 4096, 8, 9, 14336, 1, B.MOE_BF16
+    assert lib.moe_pipeline_create(ctypes.byref(desc), None, ctypes.byref(h)) == B.MOE_ERR_INVALID_ARG  # k > E
+    desc.k = 2
+    assert lib.moe_pipeline_create(ctypes.byref(desc), None, ctypes.byref(h)) == B.MOE_ERR_INVALID_ARG  # no slots
+    assert "x_dev" in B.last_error_detail(lib)
+    assert h.value is None
+    assert lib.moe_pipeline_destroy(None) == B.MOE_OK
+    assert lib.moe_pipeline_stream(None, 0) is None

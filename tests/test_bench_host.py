@@ -12,7 +12,14 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
 import bench  # noqa: E402
+from sparse_mixture_experts_renorm_b200 import build as build_mod  # noqa: E402
 from sparse_mixture_experts_renorm_b200.workloads import WORKLOADS  # noqa: E402
+
+
+@pytest.fixture(scope="module", autouse=True)
+def library():
+    """The launch plan comes from the library (a host-side query)."""
+    build_mod.build()
 
 
 def balanced(wl):
@@ -34,13 +41,18 @@ def test_prefill_gemm_work():
 
 
 def test_decode_streams_all_weights_once():
+    """At 32 tokens both projections run in one kernel: its slot streams the
+    three weight matrices of every used expert once, reads the dispatched x,
+    and accumulates the fp32 output in place; H stays between the two steps
+    and is not counted."""
     wl = WORKLOADS["mixtral_decode"]
     w = bench.algorithmic(wl, balanced(wl))
     weights = 3 * 8 * 4096 * 14336 * 2
     assert weights == pytest.approx(2.819e9, rel=1e-3)
-    streamed = (w["grouped_gemm_gateup_swiglu"]["bytes"] - 64 * 4096 * 2 - 64 * 14336 * 2
-                + w["grouped_gemm_down"]["bytes"] - 64 * 14336 * 2 - 2 * 32 * 4096 * 4 - 64 * 8)
+    assert w["grouped_gemm_down"]["bytes"] == 0 and w["grouped_gemm_down"]["flops"] == 0
+    streamed = w["grouped_gemm_gateup_swiglu"]["bytes"] - 64 * 4096 * 2 - 2 * 32 * 4096 * 4 - 64 * 8
     assert streamed == weights
+    assert w["grouped_gemm_gateup_swiglu"]["flops"] == pytest.approx(6.0 * 64 * 4096 * 14336 + 2.0 * 64 * 4096)
 
 
 def test_unused_experts_are_not_streamed():
@@ -48,9 +60,9 @@ def test_unused_experts_are_not_streamed():
     c = balanced(wl)
     c[3] += c[5]
     c[5] = 0
-    full = bench.algorithmic(wl, balanced(wl))["grouped_gemm_down"]["bytes"]
-    part = bench.algorithmic(wl, c)["grouped_gemm_down"]["bytes"]
-    assert full - part == 4096 * 14336 * 2
+    full = bench.algorithmic(wl, balanced(wl))["grouped_gemm_gateup_swiglu"]["bytes"]
+    part = bench.algorithmic(wl, c)["grouped_gemm_gateup_swiglu"]["bytes"]
+    assert full - part == 3 * 4096 * 14336 * 2
 
 
 def test_capacity_counts_only_kept_rows():
@@ -66,6 +78,17 @@ def test_fused_combine_rule():
     assert not bench.fused_combine(WORKLOADS["mixtral_prefill"], n_shared=1)
     assert not bench.fused_combine(WORKLOADS["fine_grained"])  # k = 6
     assert not bench.fused_combine(WORKLOADS["tiny_f32"])  # fp32 path
+
+
+def test_fused_gemms_rule():
+    """Both projections share one kernel for bf16 batches of at most 32 tokens."""
+    assert bench.fused_gemms(WORKLOADS["mixtral_decode"])
+    assert not bench.fused_gemms(WORKLOADS["mixtral_prefill"])
+    assert not bench.fused_gemms(WORKLOADS["tiny_f32"])  # fp32 path
+    assert bench.launches_per_step(WORKLOADS["mixtral_decode"]) == 3  # router (with the scan), permute, GEMMs
+    assert bench.launches_per_step(WORKLOADS["mixtral_prefill"]) == 5
+    assert bench.launches_per_step(WORKLOADS["fine_grained"]) == 6
+    assert bench.launches_per_step(WORKLOADS["mixtral_prefill"], {"norm": 1}) == 6  # + the router weight split
 
 
 @pytest.mark.parametrize("name,flush", [("tiny_f32", True), ("small_bf16", True), ("mixtral_prefill", False),
