@@ -165,6 +165,24 @@ def test_fine_grained_full_size_all_tokens():
     check(wl, inp, res, perm)
 
 
+def test_large_batch_all_tokens():
+    """A batch far past the benchmark workloads: 131072 tokens (1024 router
+    blocks, so the routing scan sums 8 blocks per slice over 128 slices, and
+    about 1030 token tiles across the GEMM groups), every token compared."""
+    wl = Workload("large_batch", T=131072, d=1024, E=8, k=2, I=128, renorm=True, dtype="bf16")
+    inp, res, perm = run(wl, seed=12)
+    check(wl, inp, res, perm)
+
+
+def test_most_experts_with_many_tokens():
+    """The largest expert count (256) and top-k (8) at 2048 tokens: 256 GEMM
+    groups of about 64 rows, the router's shared-memory path and a scan over
+    four slices of 256 experts."""
+    wl = Workload("max_experts", T=2048, d=256, E=256, k=8, I=128, renorm=True, dtype="bf16", router_std=0.3)
+    inp, res, perm = run(wl, seed=13)
+    check(wl, inp, res, perm)
+
+
 def test_mixtral_decode_all_tokens():
     wl = WORKLOADS["mixtral_decode"]
     inp, res, perm = run(wl)
