@@ -128,3 +128,33 @@ def test_full_size_with_all_options(name):
     rep = parity.check(inp, res, perm, wl.k, wl.renorm, wl.dtype, options=opts)
     print(f"\n[{wl.name}+options] {rep}")
     assert np.isfinite(rep["max_abs"])
+
+
+def test_host_pipeline_with_options_matches_device_calls():
+    """The library's host-memory pipeline carries the options (a copy taken
+    at creation): every batch's output and statistic equal those of a plain
+    device call with the same options, bit for bit."""
+    from sparse_mixture_experts_renorm_b200 import HostPipeline, MoELayer
+    from sparse_mixture_experts_renorm_b200.workloads import make_tokens
+
+    wl, form, nw, ns, cf, z = CASES[12]
+    opts = make_options(wl, form, nw, ns, cf, z)
+    inp = make_inputs(wl, "cuda", 3)
+    layer = MoELayer(inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k, wl.renorm, wl.T,
+                     options=opts)
+    pipe = HostPipeline(layer)
+    n = 4
+    xs = [make_tokens(wl, wl.T, "cpu", seed=200 + i).pin_memory() for i in range(n)]
+    outs = [torch.empty((wl.T, wl.d), dtype=torch.float32).pin_memory() for _ in range(n)]
+    auxs = [torch.empty((1,), dtype=torch.float32).pin_memory() for _ in range(n)]
+    for i in range(n):
+        pipe.submit(xs[i], outs[i], auxs[i])
+    pipe.synchronize()
+    pipe.close()
+    assert int(layer.status.item()) == 0
+    for i in range(n):
+        ref = moe_forward(xs[i].cuda(), inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k,
+                          wl.renorm, options=opts)
+        torch.cuda.synchronize()
+        assert torch.equal(outs[i], ref.out.cpu()), f"batch {i}"
+        assert torch.equal(auxs[i], ref.aux.cpu()), f"batch {i}"

@@ -286,7 +286,7 @@ def test_layer_replays_from_a_cuda_graph(name):
 
 # ------------------------------------------------------- host-memory path --
 
-@pytest.mark.parametrize("name", ["small_bf16", "tiny_f32"])
+@pytest.mark.parametrize("name", ["small_bf16", "tiny_f32", "mixtral_decode"])
 def test_host_pipeline_matches_device_calls(name):
     """The end-to-end path (pinned host batches in, copies on their own
     streams overlapped with the compute of neighbouring batches, fp32 output
