@@ -23,6 +23,15 @@
 // Per UMMA FLOP this moves a third fewer bytes from L2 to shared memory than
 // one CTA per 128 x 256 tile.
 //
+// In the wide configuration the gate/up GEMM turns the tile around: the 256
+// token rows are the UMMA M operand (128 per CTA) and the block's 128 hidden
+// units the N operand, CTA 0 staging their 128 gate rows and CTA 1 their 128
+// up rows. Every TMEM lane then holds one token's gate values in columns
+// 0-127 and its up values in columns 128-255, so SwiGLU needs no exchange
+// between warps: the epilogue goes from TMEM to registers to its token's H row
+// and leaves shared memory to the TMA ring and the UMMAs. The operand bytes
+// per tile are the same as in the weight-major form.
+//
 // Persistent: clusters walk a device-side tile list built from the routing
 // counts (experts in order; n-tile outer, m-tile inner inside an expert, so
 // clusters running together share weight tiles in L2). Shared experts
@@ -50,8 +59,9 @@ constexpr int kSmallRows = 16;                     // B box for tiles of <= 32 t
 // Epilogue staging: per group of four epilogue warps the gate and up rows of
 // a 32-token chunk (mode 0, 2 x 64 x 33 fp32), or one 32 x 32 fp32 transpose
 // tile per epilogue warp (mode 1, 32 x 36).
-template <int kSt, int kEw, int kBRows>
+template <int kSt, int kEw, int kBRows, bool kTokMajor = false>
 struct Gemm2Cfg {
+  static constexpr bool kTokM = kTokMajor;  // gate/up with the token rows as UMMA M (see the kernel)
   static constexpr int kStages = kSt;
   static constexpr int kEpiWarps = kEw;
   static constexpr int kBSlotRows = kBRows;            // token rows a stage holds per CTA
@@ -59,13 +69,15 @@ struct Gemm2Cfg {
   static constexpr int kThreads = 64 + 32 * kEw;
   static constexpr int kEpiBytesM0 = (kEw / 4) * (2 * 64 * 33 * 4);
   static constexpr int kEpiBytesM1 = kEw * 32 * 36 * 4;
-  static constexpr int kEpiBytes = kEpiBytesM1 > kEpiBytesM0 ? kEpiBytesM1 : kEpiBytesM0;
+  static constexpr int kEpiBytes = kTokMajor ? 0 : (kEpiBytesM1 > kEpiBytesM0 ? kEpiBytesM1 : kEpiBytesM0);
   static constexpr int kSmemBytes = kSt * (kHalfBytes + kBSlotBytes) + kEpiBytes + 1024 + 4096;
 };
 using Gemm2Wide = Gemm2Cfg<5, 8, 128>;
+using Gemm2WideTM = Gemm2Cfg<6, 8, 128, true>;  // token-major gate/up: no epilogue staging, a sixth stage
 using Gemm2Narrow = Gemm2Cfg<6, 4, 128>;
 using Gemm2Stream = Gemm2Cfg<11, 4, kSmallRows>;
-static_assert(Gemm2Wide::kSmemBytes <= 227 * 1024 && Gemm2Narrow::kSmemBytes <= 227 * 1024 &&
+static_assert(Gemm2Wide::kSmemBytes <= 227 * 1024 && Gemm2WideTM::kSmemBytes <= 227 * 1024 &&
+                  Gemm2Narrow::kSmemBytes <= 227 * 1024 &&
                   Gemm2Stream::kSmemBytes <= 227 * 1024,
               "shared memory");
 
@@ -257,7 +269,7 @@ __device__ __forceinline__ bool wait_counter_geq(const int32_t* counter, int tar
 // Maps: tmA0/tmA1 (W_gate/W_up, or W_down twice in mode 1), tmS0/tmS1 (the
 // shared experts' counterparts), tmB/tmBs (the B operand in 128- and 16-row
 // boxes); in mode 2 tmD/tmSD/tmH/tmHs are the down projection's.
-template <int kMode, int kSt, int kEw, int kBRows>
+template <int kMode, int kSt, int kEw, int kBRows, bool kTokM>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
     grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                             const __grid_constant__ CUtensorMap tmS0, const __grid_constant__ CUtensorMap tmS1,
@@ -268,7 +280,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
                             const GemmPhase p0, const GemmPhase p1, const int32_t* __restrict__ perm_tok,
                             const float* __restrict__ rgate, float* __restrict__ comb_out,
                             int32_t* __restrict__ mt_done, int32_t* status, uint64_t limit_ns) {
-  using Cfg = Gemm2Cfg<kSt, kEw, kBRows>;
+  using Cfg = Gemm2Cfg<kSt, kEw, kBRows, kTokM>;
+  // token-major gate/up: the tile's 256 token rows are the UMMA M operand
+  // (128 per CTA) and its 128 hidden units the N operand, gate rows from CTA
+  // 0 and up rows from CTA 1, so each TMEM lane holds one token's gate
+  // (columns 0-127) and up (128-255) values side by side
+  constexpr bool kTM = kTokM && kMode == 0;
   constexpr int kBSlot = Cfg::kBSlotBytes;
   constexpr int kGroups = kEw / 4;  // groups of four epilogue warps (one per TMEM lane quarter each)
   extern __shared__ uint8_t smem_raw[];
@@ -360,8 +377,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
         const TileCoord tc = decode_tile(ph1 ? tile - total0 : tile, ph1 ? n_wb1 : n_wb0, s_mt, G);
         const GroupRows gr = group_rows(tc.e, s_off, E, P.sh);
         const int ntok = min(256, gr.cnt - tc.m * 256);
-        const int half = ((ntok + 15) & ~15) >> 1;  // token rows of B held by each CTA
-        const bool small = half <= kSmallRows;
+        const int half = kTM ? 128 : ((ntok + 15) & ~15) >> 1;  // token rows of the tile held by each CTA
+        const bool small = !kTM && half <= kSmallRows;
         if (!small && kBRows < 128) {  // the launcher guarantees this cannot happen
           atomicOr(status, MOE_DEV_INTERNAL);
           *s_abort = 1;
@@ -369,10 +386,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
           break;
         }
         const int brow = gr.in0 + tc.m * 256 + (int)rank * half;
-        const int arow = mode == 0 ? gr.widx * P.N + tc.n * 128 + (int)rank * 64
-                                   : gr.widx * P.N + tc.n * 256 + (int)rank * 128;
-        const CUtensorMap* mA0 = ph1 ? (gr.shared ? &tmSD : &tmD) : (gr.shared ? &tmS0 : &tmA0);
-        const CUtensorMap* mA1 = ph1 ? mA0 : (gr.shared ? &tmS1 : &tmA1);
+        const int arow = kTM         ? gr.widx * P.N + tc.n * 128
+                         : mode == 0 ? gr.widx * P.N + tc.n * 128 + (int)rank * 64
+                                     : gr.widx * P.N + tc.n * 256 + (int)rank * 128;
+        const CUtensorMap* mA0 = kTM ? (rank == 0 ? (gr.shared ? &tmS0 : &tmA0) : (gr.shared ? &tmS1 : &tmA1))
+                                     : (ph1 ? (gr.shared ? &tmSD : &tmD) : (gr.shared ? &tmS0 : &tmA0));
+        const CUtensorMap* mA1 = kTM ? mA0 : (ph1 ? mA0 : (gr.shared ? &tmS1 : &tmA1));
         const CUtensorMap* mB = ph1 ? (small ? &tmHs : &tmH) : (small ? &tmBs : &tmB);
         const uint32_t bytes = 2u * (uint32_t)(kHalfBytes + (small ? kSmallRows * 128 : kHalfBytes));
         if (ph1) {
@@ -392,7 +411,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
           }
           const uint32_t fbar = map_to_cta(&full[stage], 0);
           if (leader) mbar_arrive_expect_tx(&full[stage], bytes);
-          if (mode == 0) {
+          if (kTM) {
+            // this CTA's 128 weight rows: gate rows of the block's 128 units
+            // in CTA 0, the same units' up rows in CTA 1
+            tma_load_2d_pair(sA + stage * kHalfBytes, mA0, fbar, kb * kBK, arow);
+            tma_load_2d_pair(sA + stage * kHalfBytes + kHalfBytes / 2, mA0, fbar, kb * kBK, arow + 64);
+          } else if (mode == 0) {
             // rows 0-63: gate rows of this CTA's 64 hidden units, 64-127: up rows
             tma_load_2d_pair(sA + stage * kHalfBytes, mA0, fbar, kb * kBK, arow);
             tma_load_2d_pair(sA + stage * kHalfBytes + kHalfBytes / 2, mA1, fbar, kb * kBK, arow);
@@ -436,10 +460,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
         const int KB = P.K / kBK;
         const TileCoord tc = decode_tile(ph1 ? tile - total0 : tile, ph1 ? n_wb1 : n_wb0, s_mt, G);
         const int ntok = min(256, group_rows(tc.e, s_off, E, P.sh).cnt - tc.m * 256);
-        const int nt16 = (ntok + 15) & ~15;
+        const int nt16 = kTM ? 256 : (ntok + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(256, nt16);
         // narrow tiles spread their K loop over independent accumulators
-        const int nacc = nt16 <= 64 ? 4 : (nt16 <= 128 ? 2 : 1);
+        const int nacc = kTM ? 1 : (nt16 <= 64 ? 4 : (nt16 <= 128 ? 2 : 1));
         const int acc_stride = kBN / nacc;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, s_abort, status, limit_ns)) break;
         tc_fence_after();
@@ -450,8 +474,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t adesc = sw128_kmajor_desc(smem_u32(sA + stage * kHalfBytes));
-          const uint64_t bdesc = sw128_kmajor_desc(smem_u32(sB + stage * kBSlot));
+          const uint32_t wslot = smem_u32(sA + stage * kHalfBytes), tslot = smem_u32(sB + stage * kBSlot);
+          const uint64_t adesc = sw128_kmajor_desc(kTM ? tslot : wslot);
+          const uint64_t bdesc = sw128_kmajor_desc(kTM ? wslot : tslot);
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const int a = kk % nacc;
@@ -499,7 +524,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
       const int nt16 = (ntok + 15) & ~15;
       const int nacc = nt16 <= 64 ? 4 : (nt16 <= 128 ? 2 : 1);
       const int acc_stride = kBN / nacc;
-      if (mode == 0) {
+      if (kTM) {
+        // TMEM lane = one token of this CTA's half of the tile; columns 0-127
+        // hold its gate and 128-255 its up values for the block's 128 hidden
+        // units. SwiGLU stays in the thread, which writes 32 units (64 bytes)
+        // of its token's H row per chunk; the two groups take alternate chunks.
+        const int tok = (int)rank * 128 + q * 32 + lane;
+        const bool live = tok < ntok;
+        __nv_bfloat16* hrow = static_cast<__nv_bfloat16*>(P.out) + (row0 + (live ? tok : 0)) * static_cast<size_t>(N);
+#pragma unroll 1
+        for (int c = (warp - 2) >> 2; c < 4; c += kGroups) {
+          uint32_t g[32], u[32];
+          __syncwarp();
+          tmem_ld_x32(tbase + c * 32, g);
+          tmem_ld_x32(tbase + 128 + c * 32, u);
+          tmem_ld_wait();
+          const int unit0 = tc.n * 128 + c * 32;
+          if (live && unit0 < N) {
+            uint4* dst = reinterpret_cast<uint4*>(hrow + unit0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int a = 8 * j + 2 * i;
+                pk[i] = pack_bf16x2(silu_f32(__uint_as_float(g[a])) * __uint_as_float(u[a]),
+                                    silu_f32(__uint_as_float(g[a + 1])) * __uint_as_float(u[a + 1]));
+              }
+              dst[j] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          }
+        }
+      } else if (mode == 0) {
         // TMEM lanes 0-63 hold the gate rows, 64-127 the up rows of this
         // CTA's 64 hidden units. Per 32-token chunk both halves go to shared
         // memory; then every thread finishes 16 (token, unit) pairs and
@@ -642,7 +698,7 @@ template <int kMode, class Cfg>
 cudaError_t launch_tc2_cfg(const Tc2Maps& m, const int32_t* offsets, const int32_t* mtile256, int R_rows, int E,
                            const GemmPhase& p0, const GemmPhase& p1, const int32_t* perm_tok, const float* rgate,
                            float* comb_out, int32_t* mt_done, int32_t* status, cudaStream_t stream) {
-  auto kern = grouped_gemm_tc2_kernel<kMode, Cfg::kStages, Cfg::kEpiWarps, Cfg::kBSlotRows>;
+  auto kern = grouped_gemm_tc2_kernel<kMode, Cfg::kStages, Cfg::kEpiWarps, Cfg::kBSlotRows, Cfg::kTokM>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (err != cudaSuccess) return err;
   const int pairs = max_active_pairs<Cfg>(reinterpret_cast<const void*>(kern));
@@ -672,6 +728,9 @@ cudaError_t launch_tc2(const Tc2Maps& m, const int32_t* offsets, const int32_t* 
   const bool wide = (long long)R_rows >= 64ll * (E + p0.sh.n) && (kMode == 0 || comb_out != nullptr);
   if (max_rows_per_group <= 2 * kSmallRows)
     return launch_tc2_cfg<kMode, Gemm2Stream>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate, comb_out,
+                                              nullptr, status, stream);
+  if (wide && kMode == 0)
+    return launch_tc2_cfg<kMode, Gemm2WideTM>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate, comb_out,
                                               nullptr, status, stream);
   if (wide)
     return launch_tc2_cfg<kMode, Gemm2Wide>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate, comb_out,
