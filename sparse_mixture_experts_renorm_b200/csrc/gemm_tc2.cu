@@ -61,7 +61,7 @@ constexpr int kSmallRows = 16;                     // B box for tiles of <= 32 t
 // tile per epilogue warp (mode 1, 32 x 36).
 template <int kSt, int kEw, int kBRows, bool kTokMajor = false>
 struct Gemm2Cfg {
-  static constexpr bool kTokM = kTokMajor;  // gate/up with the token rows as UMMA M (see the kernel)
+  static constexpr bool kTokM = kTokMajor;  // gate/up with the token rows as UMMA M (see the kernel; mode 0 only)
   static constexpr int kStages = kSt;
   static constexpr int kEpiWarps = kEw;
   static constexpr int kBSlotRows = kBRows;            // token rows a stage holds per CTA
@@ -729,12 +729,15 @@ cudaError_t launch_tc2(const Tc2Maps& m, const int32_t* offsets, const int32_t* 
   if (max_rows_per_group <= 2 * kSmallRows)
     return launch_tc2_cfg<kMode, Gemm2Stream>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate, comb_out,
                                               nullptr, status, stream);
-  if (wide && kMode == 0)
-    return launch_tc2_cfg<kMode, Gemm2WideTM>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate, comb_out,
+  if constexpr (kMode == 0) {  // the token-major configuration has no staging for down tiles
+    if (wide)
+      return launch_tc2_cfg<kMode, Gemm2WideTM>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate, comb_out,
+                                                nullptr, status, stream);
+  } else {
+    if (wide)
+      return launch_tc2_cfg<kMode, Gemm2Wide>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate, comb_out,
                                               nullptr, status, stream);
-  if (wide)
-    return launch_tc2_cfg<kMode, Gemm2Wide>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate, comb_out,
-                                            nullptr, status, stream);
+  }
   return launch_tc2_cfg<kMode, Gemm2Narrow>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate, comb_out,
                                             nullptr, status, stream);
 }
