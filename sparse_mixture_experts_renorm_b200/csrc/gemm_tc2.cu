@@ -61,7 +61,7 @@ constexpr int kSmallRows = 16;                     // B box for tiles of <= 32 t
 // tile per epilogue warp (mode 1, 32 x 36).
 template <int kSt, int kEw, int kBRows, bool kTokMajor = false>
 struct Gemm2Cfg {
-  static constexpr bool kTokM = kTokMajor;  // gate/up with the token rows as UMMA M (see the kernel; mode 0 only)
+  static constexpr bool kTokM = kTokMajor;  // token rows as the UMMA M operand (see the kernel)
   static constexpr int kStages = kSt;
   static constexpr int kEpiWarps = kEw;
   static constexpr int kBSlotRows = kBRows;            // token rows a stage holds per CTA
@@ -73,7 +73,7 @@ struct Gemm2Cfg {
   static constexpr int kSmemBytes = kSt * (kHalfBytes + kBSlotBytes) + kEpiBytes + 1024 + 4096;
 };
 using Gemm2Wide = Gemm2Cfg<5, 8, 128>;
-using Gemm2WideTM = Gemm2Cfg<6, 8, 128, true>;  // token-major gate/up: no epilogue staging, a sixth stage
+using Gemm2WideTM = Gemm2Cfg<6, 8, 128, true>;  // token-major: no epilogue staging, a sixth stage
 using Gemm2Narrow = Gemm2Cfg<6, 4, 128>;
 using Gemm2Stream = Gemm2Cfg<11, 4, kSmallRows>;
 static_assert(Gemm2Wide::kSmemBytes <= 227 * 1024 && Gemm2WideTM::kSmemBytes <= 227 * 1024 &&
@@ -281,11 +281,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
                             const float* __restrict__ rgate, float* __restrict__ comb_out,
                             int32_t* __restrict__ mt_done, int32_t* status, uint64_t limit_ns) {
   using Cfg = Gemm2Cfg<kSt, kEw, kBRows, kTokM>;
-  // token-major gate/up: the tile's 256 token rows are the UMMA M operand
-  // (128 per CTA) and its 128 hidden units the N operand, gate rows from CTA
-  // 0 and up rows from CTA 1, so each TMEM lane holds one token's gate
-  // (columns 0-127) and up (128-255) values side by side
-  constexpr bool kTM = kTokM && kMode == 0;
+  // token-major tiles: the tile's 256 token rows are the UMMA M operand (128
+  // per CTA) and its weight rows the N operand. Gate/up: the block's 128
+  // hidden units, gate rows from CTA 0 and up rows from CTA 1, so each TMEM
+  // lane holds one token's gate (columns 0-127) and up (128-255) values side
+  // by side. Down: the block's 256 output features, 128 W_down rows per CTA,
+  // so each lane holds one token's 256 outputs.
+  constexpr bool kTM = kTokM && kMode != 2;
   constexpr int kBSlot = Cfg::kBSlotBytes;
   constexpr int kGroups = kEw / 4;  // groups of four epilogue warps (one per TMEM lane quarter each)
   extern __shared__ uint8_t smem_raw[];
@@ -386,12 +388,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
           break;
         }
         const int brow = gr.in0 + tc.m * 256 + (int)rank * half;
-        const int arow = kTM         ? gr.widx * P.N + tc.n * 128
+        const bool tm_gu = kTM && mode == 0;  // token-major gate/up
+        const int arow = tm_gu       ? gr.widx * P.N + tc.n * 128
                          : mode == 0 ? gr.widx * P.N + tc.n * 128 + (int)rank * 64
                                      : gr.widx * P.N + tc.n * 256 + (int)rank * 128;
-        const CUtensorMap* mA0 = kTM ? (rank == 0 ? (gr.shared ? &tmS0 : &tmA0) : (gr.shared ? &tmS1 : &tmA1))
-                                     : (ph1 ? (gr.shared ? &tmSD : &tmD) : (gr.shared ? &tmS0 : &tmA0));
-        const CUtensorMap* mA1 = kTM ? mA0 : (ph1 ? mA0 : (gr.shared ? &tmS1 : &tmA1));
+        const CUtensorMap* mA0 = tm_gu ? (rank == 0 ? (gr.shared ? &tmS0 : &tmA0) : (gr.shared ? &tmS1 : &tmA1))
+                                       : (ph1 ? (gr.shared ? &tmSD : &tmD) : (gr.shared ? &tmS0 : &tmA0));
+        const CUtensorMap* mA1 = tm_gu ? mA0 : (ph1 ? mA0 : (gr.shared ? &tmS1 : &tmA1));
         const CUtensorMap* mB = ph1 ? (small ? &tmHs : &tmH) : (small ? &tmBs : &tmB);
         const uint32_t bytes = 2u * (uint32_t)(kHalfBytes + (small ? kSmallRows * 128 : kHalfBytes));
         if (ph1) {
@@ -411,7 +414,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
           }
           const uint32_t fbar = map_to_cta(&full[stage], 0);
           if (leader) mbar_arrive_expect_tx(&full[stage], bytes);
-          if (kTM) {
+          if (tm_gu) {
             // this CTA's 128 weight rows: gate rows of the block's 128 units
             // in CTA 0, the same units' up rows in CTA 1
             tma_load_2d_pair(sA + stage * kHalfBytes, mA0, fbar, kb * kBK, arow);
@@ -524,7 +527,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
       const int nt16 = (ntok + 15) & ~15;
       const int nacc = nt16 <= 64 ? 4 : (nt16 <= 128 ? 2 : 1);
       const int acc_stride = kBN / nacc;
-      if (kTM) {
+      if (kTM && mode == 0) {
         // TMEM lane = one token of this CTA's half of the tile; columns 0-127
         // hold its gate and 128-255 its up values for the block's 128 hidden
         // units. SwiGLU stays in the thread, which writes 32 units (64 bytes)
@@ -552,6 +555,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(64 + 32 * kEw, 1)
                                     silu_f32(__uint_as_float(g[a + 1])) * __uint_as_float(u[a + 1]));
               }
               dst[j] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          }
+        }
+      } else if (kTM) {
+        // TMEM lane = one token of this CTA's half of the tile, columns =
+        // the block's 256 output features. Each thread writes 32 features
+        // (128 bytes) of its token per chunk: fp32 Y rows, or with the
+        // combine folded in, gate * y added into the token's output row (two
+        // adds per element into a zeroed row, so the order cannot matter).
+        const int tok = (int)rank * 128 + q * 32 + lane;
+        const bool live = tok < ntok;
+        const size_t r = row0 + static_cast<size_t>(live ? tok : 0);
+        const bool fold = comb_out != nullptr && !gr.shared;
+        float* dst = fold ? comb_out + static_cast<size_t>(live ? perm_tok[r] : 0) * N
+                          : static_cast<float*>(P.out) + r * N;
+        const float gs = fold && live ? rgate[r] : 1.0f;
+#pragma unroll 1
+        for (int c = (warp - 2) >> 2; c < 8; c += kGroups) {
+          uint32_t v[32];
+          __syncwarp();
+          tmem_ld_x32(tbase + c * 32, v);
+          tmem_ld_wait();
+          const int o = tc.n * 256 + c * 32;
+          if (live && o < N) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float a0 = __uint_as_float(v[4 * j]), a1 = __uint_as_float(v[4 * j + 1]);
+              const float a2 = __uint_as_float(v[4 * j + 2]), a3 = __uint_as_float(v[4 * j + 3]);
+              if (fold)
+                red_add_v4(dst + o + 4 * j, gs * a0, gs * a1, gs * a2, gs * a3);
+              else
+                *reinterpret_cast<float4*>(dst + o + 4 * j) = make_float4(a0, a1, a2, a3);
             }
           }
         }
@@ -689,6 +724,18 @@ int max_active_pairs(const void* kern) {
   }
 }
 
+// Streaming multiprocessors of the current device, queried once per device.
+int device_sm_count() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  int n = cache[dev].load(std::memory_order_acquire);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 0;
+  cache[dev].store(n, std::memory_order_release);
+  return n;
+}
+
 // The tensor maps of one launch (see the kernel; unused ones repeat others).
 struct Tc2Maps {
   CUtensorMap a0, a1, s0, s1, b, bs, d, sd, h, hs;
@@ -729,14 +776,24 @@ cudaError_t launch_tc2(const Tc2Maps& m, const int32_t* offsets, const int32_t* 
   if (max_rows_per_group <= 2 * kSmallRows)
     return launch_tc2_cfg<kMode, Gemm2Stream>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate, comb_out,
                                               nullptr, status, stream);
-  if constexpr (kMode == 0) {  // the token-major configuration has no staging for down tiles
+  if constexpr (kMode == 0) {
     if (wide)
       return launch_tc2_cfg<kMode, Gemm2WideTM>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate, comb_out,
                                                 nullptr, status, stream);
   } else {
-    if (wide)
+    if (wide) {
+      // A grid of at most three down tiles per CTA pair exposes the last
+      // tile's epilogue: the token-major form, whose epilogue adds straight
+      // from TMEM into the output rows, finishes it sooner. On longer grids
+      // it needs fewer cycles but ran at a lower power-capped clock than the
+      // weight-major form, whose adds cover 128-byte output rows.
+      const long long tiles = (long long)(R_rows / 256 + E + p0.sh.n) * ((p0.N + 255) / 256);
+      if (tiles <= 3ll * (device_sm_count() / 2))
+        return launch_tc2_cfg<kMode, Gemm2WideTM>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate,
+                                                  comb_out, nullptr, status, stream);
       return launch_tc2_cfg<kMode, Gemm2Wide>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate, comb_out,
                                               nullptr, status, stream);
+    }
   }
   return launch_tc2_cfg<kMode, Gemm2Narrow>(m, offsets, mtile256, R_rows, E, p0, p0, perm_tok, rgate, comb_out,
                                             nullptr, status, stream);

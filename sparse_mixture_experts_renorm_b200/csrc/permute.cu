@@ -42,22 +42,28 @@ __device__ __forceinline__ uint4 scale_vec(uint4 v, uint4 w, float r, bool bf16,
   return make_uint4(u[0], u[1], u[2], u[3]);
 }
 
-// Block (token t, chunk c): threads j < k compute the row of slot j from the
-// per-block base row of its expert plus its rank inside the router block
-// (chunk 0 also records perm_tok / inv); then every thread copies one 16-byte
-// vector of x[t] (normalised when rnorm is given) to each of the token's kept
-// rows and, with shared experts, to row shared_row0 + t.
+// Block (tokens t0 .. t0+G-1, chunk c): threads g*k + j compute the row of
+// slot j of token t0+g from the per-block base row of its expert plus its
+// rank inside the router block (chunk 0 also records perm_tok / inv); then
+// the block copies its chunk of 16-byte vectors of the G rows of x
+// (normalised when rnorm is given) to each kept row of its token and, with
+// shared experts, to row shared_row0 + t. Several tokens per block put one
+// chain of dependent index loads in front of several rows of copying, and
+// four vectors in flight per thread.
+template <int G>
 __global__ void __launch_bounds__(kCopyThreads) permute_kernel(
-    const uint4* __restrict__ x, int nvec, int E, int k, int rb, int R, const int32_t* __restrict__ topk_idx,
+    const uint4* __restrict__ x, int T, int nvec, int E, int k, int rb, int R, const int32_t* __restrict__ topk_idx,
     const int32_t* __restrict__ lrank, const int32_t* __restrict__ blk_base, const int32_t* __restrict__ offsets,
     int has_cap, int32_t* __restrict__ perm_tok, int32_t* __restrict__ inv, uint4* __restrict__ xp,
     const float* __restrict__ gate, float* __restrict__ rgate, float4* __restrict__ zero_out, int nout4,
     const float* __restrict__ rnorm, const uint4* __restrict__ norm_w, int bf16, int shared_row0, int32_t* status) {
-  const int t = blockIdx.x;
-  __shared__ int s_rows[kMaxTopK];
+  const int t0 = blockIdx.x * G;
+  const int ng = min(G, T - t0);
+  __shared__ int s_rows[G][kMaxTopK];
   pdl_wait();
-  if (threadIdx.x < k) {
-    const int j = threadIdx.x;
+  if ((int)threadIdx.x < ng * k) {
+    const int g = threadIdx.x / k, j = threadIdx.x - g * k;
+    const int t = t0 + g;
     const int e = topk_idx[(size_t)t * k + j];
     int row = -1;
     bool bad = e < 0 || e >= E;
@@ -78,23 +84,45 @@ __global__ void __launch_bounds__(kCopyThreads) permute_kernel(
       inv[(size_t)t * k + j] = row;
       rgate[row] = gate[(size_t)t * k + j];
     }
-    s_rows[j] = row;
+    s_rows[g][j] = row;
   }
   __syncthreads();
-  if (zero_out) {  // the output row this block's x chunk maps to, for a combine done by atomics
+  if (zero_out) {  // the output rows this block's x chunk maps to, for a combine done by atomics
     const int per = (nout4 + gridDim.y - 1) / gridDim.y;
-    for (int o = blockIdx.y * per + threadIdx.x; o < min(nout4, (int)(blockIdx.y + 1) * per); o += kCopyThreads)
-      zero_out[(size_t)t * nout4 + o] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int o0 = blockIdx.y * per, w = min(nout4, o0 + per) - o0;
+    for (int idx = threadIdx.x; idx < ng * w; idx += kCopyThreads) {
+      const int g = idx / w;
+      zero_out[(size_t)(t0 + g) * nout4 + o0 + (idx - g * w)] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
-  const int i = blockIdx.y * kCopyThreads + threadIdx.x;
-  if (i >= nvec) return;
-  uint4 v = __ldg(x + (size_t)t * nvec + i);
-  if (rnorm) v = scale_vec(v, norm_w ? __ldg(norm_w + i) : make_uint4(0u, 0u, 0u, 0u), rnorm[t], bf16 != 0,
-                           norm_w != nullptr);
+  const int c0 = blockIdx.y * kCopyThreads;
+  const int cw = min(kCopyThreads, nvec - c0);  // vectors of this chunk in every row
+  const int n = ng * cw;
+  for (int base = threadIdx.x; base < n; base += 4 * kCopyThreads) {
+    uint4 v[4];
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j)
-    if (j < k && s_rows[j] >= 0) xp[(size_t)s_rows[j] * nvec + i] = v;
-  if (shared_row0 >= 0) xp[(size_t)(shared_row0 + t) * nvec + i] = v;
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * kCopyThreads;
+      if (idx < n) {
+        const int g = idx / cw, i = c0 + idx - g * cw;
+        v[u] = __ldg(x + (size_t)(t0 + g) * nvec + i);
+        if (rnorm)
+          v[u] = scale_vec(v[u], norm_w ? __ldg(norm_w + i) : make_uint4(0u, 0u, 0u, 0u), rnorm[t0 + g], bf16 != 0,
+                           norm_w != nullptr);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int idx = base + u * kCopyThreads;
+      if (idx < n) {
+        const int g = idx / cw, i = c0 + idx - g * cw;
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j)
+          if (j < k && s_rows[g][j] >= 0) xp[(size_t)s_rows[g][j] * nvec + i] = v[u];
+        if (shared_row0 >= 0) xp[(size_t)(shared_row0 + t0 + g) * nvec + i] = v[u];
+      }
+    }
+  }
 }
 
 // Block (token t, chunk c): every thread sums one float4 of its token's k
@@ -159,11 +187,19 @@ cudaError_t launch_permute(moe_dtype dtype, const void* x, int T, int d, int E, 
                            cudaStream_t stream) {
   const int elem = dtype == MOE_BF16 ? 2 : 4;
   const int nvec = d * elem / 16;
-  const dim3 grid(T, (nvec + kCopyThreads - 1) / kCopyThreads);
-  return launch_pdl(permute_kernel, grid, dim3(kCopyThreads), 0, stream, static_cast<const uint4*>(x), nvec, E, k, rb,
-                    T * k, topk_idx, lrank, blk_base, offsets, has_cap, perm_tok, inv, static_cast<uint4*>(xp),
-                    topk_gate, rgate, reinterpret_cast<float4*>(zero_out), d / 4, rnorm,
-                    static_cast<const uint4*>(norm_w), dtype == MOE_BF16 ? 1 : 0, shared_row0, status);
+  // tokens per block: up to 8 while the grid keeps about 512 blocks or more,
+  // and fewer as a token's copies grow (measured: with k = 6 rows of 4 KB a
+  // token, one token per block copies faster)
+  const int copy_bytes = k * nvec * 16;
+  const int gmax = copy_bytes <= 8192 ? 8 : copy_bytes <= 16384 ? 4 : 1;
+  const int gt = T >= 4096 ? 8 : T >= 2048 ? 4 : T >= 1024 ? 2 : 1;
+  const int G = gt < gmax ? gt : gmax;
+  const dim3 grid((T + G - 1) / G, (nvec + kCopyThreads - 1) / kCopyThreads);
+  auto kern = G == 8 ? permute_kernel<8> : G == 4 ? permute_kernel<4> : G == 2 ? permute_kernel<2> : permute_kernel<1>;
+  return launch_pdl(kern, grid, dim3(kCopyThreads), 0, stream, static_cast<const uint4*>(x), T, nvec, E, k, rb, T * k,
+                    topk_idx, lrank, blk_base, offsets, has_cap, perm_tok, inv, static_cast<uint4*>(xp), topk_gate,
+                    rgate, reinterpret_cast<float4*>(zero_out), d / 4, rnorm, static_cast<const uint4*>(norm_w),
+                    dtype == MOE_BF16 ? 1 : 0, shared_row0, status);
 }
 
 cudaError_t launch_combine(int T, int d, int k, const float* y, const int32_t* inv, const float* topk_gate,
