@@ -96,6 +96,18 @@ __global__ void __launch_bounds__(kCopyThreads) permute_kernel(
     }
   }
   const int c0 = blockIdx.y * kCopyThreads;
+  if constexpr (G == 1) {  // one vector per thread (fewer registers: eight blocks per SM)
+    const int i = c0 + threadIdx.x;
+    if (i >= nvec) return;
+    uint4 v = __ldg(x + (size_t)t0 * nvec + i);
+    if (rnorm) v = scale_vec(v, norm_w ? __ldg(norm_w + i) : make_uint4(0u, 0u, 0u, 0u), rnorm[t0], bf16 != 0,
+                             norm_w != nullptr);
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j)
+      if (j < k && s_rows[0][j] >= 0) xp[(size_t)s_rows[0][j] * nvec + i] = v;
+    if (shared_row0 >= 0) xp[(size_t)(shared_row0 + t0) * nvec + i] = v;
+    return;
+  }
   const int cw = min(kCopyThreads, nvec - c0);  // vectors of this chunk in every row
   const int n = ng * cw;
   for (int base = threadIdx.x; base < n; base += 4 * kCopyThreads) {
