@@ -146,6 +146,10 @@ def algorithmic(wl, counts, opts=None):
         rt, sc = work["router_topk"], work["route_scan"]
         work["router_topk"] = dict(flops=rt["flops"], bytes=rt["bytes"] + sc["bytes"])
         work["route_scan"] = dict(flops=0.0, bytes=0)
+    if plan & B.MOE_PLAN_PERMUTE_SCAN:
+        pm, sc = work["permute"], work["route_scan"]
+        work["permute"] = dict(flops=pm["flops"], bytes=pm["bytes"] + sc["bytes"])
+        work["route_scan"] = dict(flops=0.0, bytes=0)
     if plan & B.MOE_PLAN_FUSED_GEMMS:
         gu, dn = work["grouped_gemm_gateup_swiglu"], work["grouped_gemm_down"]
         work["grouped_gemm_gateup_swiglu"] = dict(flops=gu["flops"] + dn["flops"],
@@ -179,6 +183,9 @@ def slot_names(wl, opts=None):
     if plan & B.MOE_PLAN_FUSED_SCAN:
         names[0] = "router_topk (with the routing scan)"
         names[1] = "route_scan (in router_topk)"
+    if plan & B.MOE_PLAN_PERMUTE_SCAN:
+        names[1] = "route_scan (in permute)"
+        names[2] = "permute (with the routing scan)"
     if plan & B.MOE_PLAN_FUSED_GEMMS:
         names[3] = "grouped_gemm_gateup_down (both projections)"
         names[4] = "grouped_gemm_down (in the fused kernel)"
@@ -193,7 +200,8 @@ def launches_per_step(wl, opts=None):
 
     plan = plan_of(wl, opts)
     return (B.MOE_NUM_KERNELS - (1 if plan & B.MOE_PLAN_FUSED_COMBINE else 0)
-            - (1 if plan & B.MOE_PLAN_FUSED_GEMMS else 0) - (1 if plan & B.MOE_PLAN_FUSED_SCAN else 0)
+            - (1 if plan & B.MOE_PLAN_FUSED_GEMMS else 0)
+            - (1 if plan & (B.MOE_PLAN_FUSED_SCAN | B.MOE_PLAN_PERMUTE_SCAN) else 0)
             + (1 if plan & B.MOE_PLAN_ROUTER_WEIGHT_SPLIT else 0))
 
 

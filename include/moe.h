@@ -244,11 +244,16 @@ moe_status moe_forward_ex(const void* x, const void* w_router, const float* b_ro
  *     falls in slot 0.
  *   MOE_PLAN_FUSED_SCAN: the router does the routing scan itself (bf16,
  *     1 <= T <= 128 tokens, one router block, E <= 16): slot 1 is empty.
+ *   MOE_PLAN_PERMUTE_SCAN: otherwise, when the batch has few router blocks
+ *     (blocks of 128 tokens for bf16, 32 for fp32; blocks x E <= 4096), every
+ *     permute block redoes the scan's sums for its own rows and the permute
+ *     writes the scan's results: slot 1 is empty, slot 2 times both.
  */
 #define MOE_PLAN_FUSED_COMBINE 1
 #define MOE_PLAN_FUSED_GEMMS 2
 #define MOE_PLAN_ROUTER_WEIGHT_SPLIT 4
 #define MOE_PLAN_FUSED_SCAN 8
+#define MOE_PLAN_PERMUTE_SCAN 16
 int moe_launch_plan(int T, int d, int E, int k, int I, moe_dtype dtype, const moe_options* opt);
 
 /*

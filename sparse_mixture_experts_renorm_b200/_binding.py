@@ -34,6 +34,7 @@ MOE_MAX_SHARED = 8
 MOE_NOALLOC_SCRATCH_BYTES = 16 << 20
 MOE_NUM_KERNELS = 6
 MOE_PLAN_FUSED_COMBINE, MOE_PLAN_FUSED_GEMMS, MOE_PLAN_ROUTER_WEIGHT_SPLIT, MOE_PLAN_FUSED_SCAN = 1, 2, 4, 8
+MOE_PLAN_PERMUTE_SCAN = 16
 
 
 class moe_options(ctypes.Structure):

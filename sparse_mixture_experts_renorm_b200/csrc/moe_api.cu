@@ -319,7 +319,25 @@ moe_status forward_impl(const void* x, const void* w_router, const float* b_rout
   }
   if (err != cudaSuccess) return fail_cuda(err, "router kernel");
   marks.mark(stream);
-  if (!router_scan) {
+  const int nb = router_blocks(T, dtype);
+  const bool permute_scan = !router_scan && permute_does_scan(nb, E);
+  PermuteScanArgs ps;
+  if (permute_scan) {
+    ps.nb = nb;
+    ps.cap = cap;
+    ps.n_shared = o.n_shared;
+    ps.n_mt = mt_done ? (int)w.n_mt : 0;
+    ps.blk_psum = blk_psum;
+    ps.blk_z = blk_z;
+    ps.counts = cnt;
+    ps.offsets = offsets;
+    ps.mtile = mtile;
+    ps.aux = aux_p;
+    ps.zloss = o.zloss;
+    ps.dropped = o.dropped;
+    ps.mt_done = mt_done;
+  }
+  if (!router_scan && !permute_scan) {
     NvtxRange r("route_scan");
     err = launch_route_scan(router_blocks(T, dtype), T, E, k, cap, o.n_shared, blk_cnt, blk_psum, blk_z, cnt,
                             offsets, mtile, aux_p, o.zloss, o.dropped, mt_done, (int)w.n_mt, stream);
@@ -335,7 +353,7 @@ moe_status forward_impl(const void* x, const void* w_router, const float* b_rout
     NvtxRange r("permute");
     err = launch_permute(dtype, x, T, d, E, k, router_block_tokens(dtype), topk_idx, lrank, blk_cnt, offsets,
                          cap >= 0 ? 1 : 0, perm_tok, inv, xp, topk_gate, rgate, fused_combine ? out : nullptr, rnorm,
-                         o.norm_w, o.n_shared > 0 ? R : -1, status, stream);
+                         o.norm_w, o.n_shared > 0 ? R : -1, ps, status, stream);
   }
   if (err != cudaSuccess) return fail_cuda(err, "permute kernel");
 
@@ -498,7 +516,10 @@ int moe_launch_plan(int T, int d, int E, int k, int I, moe_dtype dtype, const mo
   int plan = 0;
   if (dtype == MOE_BF16 && k == 2 && o.n_shared == 0) plan |= MOE_PLAN_FUSED_COMBINE;
   if (gemms_fused(T, dtype)) plan |= MOE_PLAN_FUSED_GEMMS;
-  if (router_does_scan(T, E, dtype)) plan |= MOE_PLAN_FUSED_SCAN;
+  if (router_does_scan(T, E, dtype))
+    plan |= MOE_PLAN_FUSED_SCAN;
+  else if (T > 0 && permute_does_scan(router_blocks(T, dtype), E))
+    plan |= MOE_PLAN_PERMUTE_SCAN;
   if (dtype == MOE_BF16 && o.norm_form != MOE_NORM_NONE && o.norm_w) plan |= MOE_PLAN_ROUTER_WEIGHT_SPLIT;
   return plan;
 }

@@ -170,17 +170,39 @@ cudaError_t launch_route_scan(int nb, int T, int E, int k, int cap, int n_shared
                               int32_t* mtile, float* aux, float* zloss, int32_t* dropped, int32_t* mt_done, int n_mt,
                               cudaStream_t stream);
 
+// The routing scan's outputs for a permute that does the scan itself (see
+// permute_does_scan); offsets == NULL: the scan kernel ran, and blk_base
+// holds every router block's base rows.
+struct PermuteScanArgs {
+  int nb = 0, cap = -1, n_shared = 0, n_mt = 0;
+  const float* blk_psum = nullptr;
+  const float* blk_z = nullptr;
+  int32_t* counts = nullptr;
+  int32_t* offsets = nullptr;
+  int32_t* mtile = nullptr;
+  float* aux = nullptr;
+  float* zloss = nullptr;
+  int32_t* dropped = nullptr;
+  int32_t* mt_done = nullptr;
+};
+
+// When the router did not do the scan and the batch has few router blocks
+// (nb * E at most 4096 per-block counts, which every permute block sums
+// again), the permute does the routing scan and no scan kernel runs.
+inline bool permute_does_scan(int nb, int E) { return (long long)nb * E <= 4096; }
+
 // Also records the gate of every dispatched row (rgate) and, when zero_out is
 // given, clears out[T, d] for a combine done by the down GEMM's epilogue.
 // rnorm != NULL: rows are x * rnorm[t] * norm_w (norm_w NULL: ones), rounded
 // to the dtype. shared_row0 >= 0: the (normalised) row of token t is also
 // written at row shared_row0 + t. has_cap: a row past its expert's kept count
-// is a dropped slot (inv = -1), not an error.
+// is a dropped slot (inv = -1), not an error. scan.offsets != NULL: blk_base
+// holds the router's per-block counts and the permute does the routing scan.
 cudaError_t launch_permute(moe_dtype dtype, const void* x, int T, int d, int E, int k, int rb, const int32_t* topk_idx,
                            const int32_t* lrank, const int32_t* blk_base, const int32_t* offsets, int has_cap,
                            int32_t* perm_tok, int32_t* inv, void* xp, const float* topk_gate, float* rgate,
-                           float* zero_out, const float* rnorm, const void* norm_w, int shared_row0, int32_t* status,
-                           cudaStream_t stream);
+                           float* zero_out, const float* rnorm, const void* norm_w, int shared_row0,
+                           const PermuteScanArgs& scan, int32_t* status, cudaStream_t stream);
 
 // out[t] = sum_j gate[t,j] * Y[inv[t,j]] (dropped slots skipped when has_cap)
 //        + sum_s Y[shared_row0 + s*T + t].

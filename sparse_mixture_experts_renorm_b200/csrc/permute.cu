@@ -15,6 +15,38 @@ namespace moe {
 namespace {
 
 constexpr int kCopyThreads = 256;  // 16-byte vectors per block (4 KB of a row)
+static_assert(kMaxExperts <= kCopyThreads, "one thread per expert in the permute's scan");
+
+// Exclusive prefix sum of one int per thread over the block (kCopyThreads
+// threads, in thread order); *total gets the sum. s_w: kCopyThreads/32 + 1 ints.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* s_w, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  constexpr int kW = kCopyThreads / 32;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += n;
+  }
+  if (lane == 31) s_w[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int x = lane < kW ? s_w[lane] : 0;
+    int xi = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, xi, o);
+      if (lane >= o) xi += n;
+    }
+    if (lane < kW) s_w[lane] = xi - x;
+    if (lane == 31) s_w[kW] = xi;
+  }
+  __syncthreads();
+  const int r = s_w[w] + incl - v;
+  *total = s_w[kW];
+  __syncthreads();  // s_w is reused by the next call
+  return r;
+}
 
 // x_hat = x * r * w for one 16-byte vector (8 bf16 or 4 fp32), rounded to
 // the dtype (the pre-MoE RMSNorm applied on the copy).
@@ -50,17 +82,110 @@ __device__ __forceinline__ uint4 scale_vec(uint4 v, uint4 w, float r, bool bf16,
 // shared experts, to row shared_row0 + t. Several tokens per block put one
 // chain of dependent index loads in front of several rows of copying, and
 // four vectors in flight per thread.
-template <int G>
+// The routing scan done by every permute block itself (kScan), for batches
+// whose router blocks are few: each block sums the per-block expert counts
+// again for its own router block's base rows, and block 0 also writes the
+// scan's results (counts, offsets, the GEMMs' tile schedule, the load-balance
+// statistic, the z-loss, the dropped count, the fused GEMMs' counters
+// cleared). The integer results are route_scan_kernel's exactly (so are the
+// rows); the fp64 sums of the statistics run in another fixed order.
+struct PermuteScan {
+  int nb, cap, n_shared, n_mt;
+  const float* blk_psum;
+  const float* blk_z;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* mtile;
+  float* aux;
+  float* zloss;
+  int32_t* dropped;
+  int32_t* mt_done;
+};
+
+template <int G, bool kScan>
 __global__ void __launch_bounds__(kCopyThreads) permute_kernel(
     const uint4* __restrict__ x, int T, int nvec, int E, int k, int rb, int R, const int32_t* __restrict__ topk_idx,
     const int32_t* __restrict__ lrank, const int32_t* __restrict__ blk_base, const int32_t* __restrict__ offsets,
     int has_cap, int32_t* __restrict__ perm_tok, int32_t* __restrict__ inv, uint4* __restrict__ xp,
     const float* __restrict__ gate, float* __restrict__ rgate, float4* __restrict__ zero_out, int nout4,
-    const float* __restrict__ rnorm, const uint4* __restrict__ norm_w, int bf16, int shared_row0, int32_t* status) {
+    const float* __restrict__ rnorm, const uint4* __restrict__ norm_w, int bf16, int shared_row0, int32_t* status,
+    const PermuteScan sc) {
   const int t0 = blockIdx.x * G;
   const int ng = min(G, T - t0);
   __shared__ int s_rows[G][kMaxTopK];
+  __shared__ int s_base[kScan ? kMaxExperts : 1];  // first row of each expert for this router block
+  __shared__ int s_end[kScan ? kMaxExperts + 1 : 1];  // end of each expert's kept rows
   pdl_wait();
+  if constexpr (kScan) {
+    __shared__ int s_w[kCopyThreads / 32 + 1];
+    const int e = threadIdx.x;  // one expert per thread
+    const int bb = t0 / rb;     // this block's router block
+    int tot = 0, pre = 0;
+    if (e < E)
+      for (int b = 0; b < sc.nb; ++b) {
+        const int c = blk_base[(size_t)b * E + e];  // per-block counts (the router's histogram)
+        tot += c;
+        if (b < bb) pre += c;
+      }
+    const int kept = e < E ? (sc.cap >= 0 ? min(tot, sc.cap) : tot) : 0;
+    int run = 0;
+    const int off = block_exclusive_scan(kept, s_w, &run);
+    if (e < E) {
+      s_base[e] = off + pre;
+      s_end[e] = off + kept;
+    }
+    if (blockIdx.x == 0 && blockIdx.y == 0) {
+      for (int i = threadIdx.x; i < sc.n_mt; i += kCopyThreads) sc.mt_done[i] = 0;
+      const int tiles = (kept + kTileM - 1) / kTileM;
+      int mt = 0;
+      const int mt_off = block_exclusive_scan(tiles, s_w, &mt);
+      // the statistic: E * sum_e (count_e / (T k)) * (sum of p_e / T), in fp64
+      double ps = 0.0;
+      if (e < E)
+        for (int b = 0; b < sc.nb; ++b) ps += (double)sc.blk_psum[(size_t)b * E + e];
+      double ae = e < E ? ((double)tot / ((double)T * (double)k)) * (ps / (double)T) : 0.0;
+      int dr = e < E ? tot - kept : 0;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        ae += __shfl_xor_sync(0xffffffffu, ae, o);
+        dr += __shfl_xor_sync(0xffffffffu, dr, o);
+      }
+      __shared__ double s_ae[kCopyThreads / 32];
+      __shared__ int s_dr[kCopyThreads / 32];
+      if ((threadIdx.x & 31) == 0) {
+        s_ae[threadIdx.x >> 5] = ae;
+        s_dr[threadIdx.x >> 5] = dr;
+      }
+      if (e < E) {
+        sc.offsets[e] = off;
+        sc.mtile[e] = mt_off;
+        if (sc.counts) sc.counts[e] = tot;
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        double a = 0.0;
+        int drop = 0;
+        for (int w = 0; w < kCopyThreads / 32; ++w) {
+          a += s_ae[w];
+          drop += s_dr[w];
+        }
+        sc.offsets[E] = run;
+        sc.mtile[E] = mt;
+        for (int s2 = 0; s2 < sc.n_shared; ++s2) {
+          mt += (T + kTileM - 1) / kTileM;
+          sc.mtile[E + 1 + s2] = mt;
+        }
+        if (sc.aux) *sc.aux = (float)((double)E * a);
+        if (sc.dropped) *sc.dropped = drop;
+        if (sc.zloss) {
+          double z = 0.0;
+          for (int b = 0; b < sc.nb; ++b) z += (double)sc.blk_z[b];
+          *sc.zloss = (float)(z / (double)T);
+        }
+      }
+    }
+    __syncthreads();
+  }
   if ((int)threadIdx.x < ng * k) {
     const int g = threadIdx.x / k, j = threadIdx.x - g * k;
     const int t = t0 + g;
@@ -68,8 +193,8 @@ __global__ void __launch_bounds__(kCopyThreads) permute_kernel(
     int row = -1;
     bool bad = e < 0 || e >= E;
     if (!bad) {
-      row = blk_base[(size_t)(t / rb) * E + e] + lrank[(size_t)t * k + j];
-      if (has_cap && row >= offsets[e + 1]) {
+      row = (kScan ? s_base[e] : blk_base[(size_t)(t / rb) * E + e]) + lrank[(size_t)t * k + j];
+      if (has_cap && row >= (kScan ? s_end[e] : offsets[e + 1])) {
         row = -1;  // past the expert's capacity: this slot is dropped
         if (blockIdx.y == 0) inv[(size_t)t * k + j] = -1;
       } else if (row < 0 || row >= R) {
@@ -195,8 +320,8 @@ __global__ void __launch_bounds__(kCopyThreads) combine_kernel(const float4* __r
 cudaError_t launch_permute(moe_dtype dtype, const void* x, int T, int d, int E, int k, int rb, const int32_t* topk_idx,
                            const int32_t* lrank, const int32_t* blk_base, const int32_t* offsets, int has_cap,
                            int32_t* perm_tok, int32_t* inv, void* xp, const float* topk_gate, float* rgate,
-                           float* zero_out, const float* rnorm, const void* norm_w, int shared_row0, int32_t* status,
-                           cudaStream_t stream) {
+                           float* zero_out, const float* rnorm, const void* norm_w, int shared_row0,
+                           const PermuteScanArgs& scan, int32_t* status, cudaStream_t stream) {
   const int elem = dtype == MOE_BF16 ? 2 : 4;
   const int nvec = d * elem / 16;
   // tokens per block: up to 8 while the grid keeps about 512 blocks or more,
@@ -207,11 +332,29 @@ cudaError_t launch_permute(moe_dtype dtype, const void* x, int T, int d, int E, 
   const int gt = T >= 4096 ? 8 : T >= 2048 ? 4 : T >= 1024 ? 2 : 1;
   const int G = gt < gmax ? gt : gmax;
   const dim3 grid((T + G - 1) / G, (nvec + kCopyThreads - 1) / kCopyThreads);
-  auto kern = G == 8 ? permute_kernel<8> : G == 4 ? permute_kernel<4> : G == 2 ? permute_kernel<2> : permute_kernel<1>;
+  const bool in_scan = scan.offsets != nullptr;
+  auto kern = in_scan ? (G == 8 ? permute_kernel<8, true> : G == 4 ? permute_kernel<4, true>
+                         : G == 2 ? permute_kernel<2, true> : permute_kernel<1, true>)
+                      : (G == 8 ? permute_kernel<8, false> : G == 4 ? permute_kernel<4, false>
+                         : G == 2 ? permute_kernel<2, false> : permute_kernel<1, false>);
+  PermuteScan sc;
+  sc.nb = scan.nb;
+  sc.cap = scan.cap;
+  sc.n_shared = scan.n_shared;
+  sc.n_mt = scan.mt_done ? scan.n_mt : 0;
+  sc.blk_psum = scan.blk_psum;
+  sc.blk_z = scan.blk_z;
+  sc.counts = scan.counts;
+  sc.offsets = scan.offsets;
+  sc.mtile = scan.mtile;
+  sc.aux = scan.aux;
+  sc.zloss = scan.zloss;
+  sc.dropped = scan.dropped;
+  sc.mt_done = scan.mt_done;
   return launch_pdl(kern, grid, dim3(kCopyThreads), 0, stream, static_cast<const uint4*>(x), T, nvec, E, k, rb, T * k,
                     topk_idx, lrank, blk_base, offsets, has_cap, perm_tok, inv, static_cast<uint4*>(xp), topk_gate,
                     rgate, reinterpret_cast<float4*>(zero_out), d / 4, rnorm, static_cast<const uint4*>(norm_w),
-                    dtype == MOE_BF16 ? 1 : 0, shared_row0, status);
+                    dtype == MOE_BF16 ? 1 : 0, shared_row0, status, sc);
 }
 
 cudaError_t launch_combine(int T, int d, int k, const float* y, const int32_t* inv, const float* topk_gate,

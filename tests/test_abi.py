@@ -195,18 +195,22 @@ def test_launch_plan(lib):
     """Which kernels a call merges: the combine into the down GEMM for bf16
     k = 2 without shared experts; both projections into one kernel for bf16
     batches of 1..32 tokens; the routing scan into the router for bf16
-    batches of one router block (1..128 tokens) with at most 16 experts; an
-    extra split of w * W_r for the bf16 norm with a weight; -1 for invalid
-    arguments."""
+    batches of one router block (1..128 tokens) with at most 16 experts, else
+    into the permute while router blocks x E <= 4096; an extra split of
+    w * W_r for the bf16 norm with a weight; -1 for invalid arguments."""
     bf, f32 = B.MOE_BF16, B.MOE_F32
     assert lib.moe_launch_plan(32, 4096, 8, 2, 14336, bf, None) == (B.MOE_PLAN_FUSED_COMBINE | B.MOE_PLAN_FUSED_GEMMS
                                                                      | B.MOE_PLAN_FUSED_SCAN)
     assert lib.moe_launch_plan(33, 4096, 8, 2, 14336, bf, None) == B.MOE_PLAN_FUSED_COMBINE | B.MOE_PLAN_FUSED_SCAN
-    assert lib.moe_launch_plan(129, 4096, 8, 2, 14336, bf, None) == B.MOE_PLAN_FUSED_COMBINE
-    assert lib.moe_launch_plan(100, 256, 17, 2, 256, bf, None) == B.MOE_PLAN_FUSED_COMBINE  # E > 16
-    assert lib.moe_launch_plan(4096, 4096, 8, 2, 14336, bf, None) == B.MOE_PLAN_FUSED_COMBINE
-    assert lib.moe_launch_plan(16384, 2048, 64, 6, 1408, bf, None) == 0
-    assert lib.moe_launch_plan(64, 128, 4, 2, 256, f32, None) == 0
+    assert lib.moe_launch_plan(129, 4096, 8, 2, 14336, bf, None) == (B.MOE_PLAN_FUSED_COMBINE
+                                                                      | B.MOE_PLAN_PERMUTE_SCAN)
+    assert lib.moe_launch_plan(100, 256, 17, 2, 256, bf, None) == (B.MOE_PLAN_FUSED_COMBINE  # E > 16
+                                                                   | B.MOE_PLAN_PERMUTE_SCAN)
+    assert lib.moe_launch_plan(4096, 4096, 8, 2, 14336, bf, None) == (B.MOE_PLAN_FUSED_COMBINE
+                                                                       | B.MOE_PLAN_PERMUTE_SCAN)
+    assert lib.moe_launch_plan(16384, 2048, 64, 6, 1408, bf, None) == 0  # 128 blocks x 64 experts
+    assert lib.moe_launch_plan(65664, 4096, 8, 2, 14336, bf, None) == B.MOE_PLAN_FUSED_COMBINE  # 513 x 8
+    assert lib.moe_launch_plan(64, 128, 4, 2, 256, f32, None) == B.MOE_PLAN_PERMUTE_SCAN
     assert lib.moe_launch_plan(0, 4096, 8, 2, 14336, bf, None) == B.MOE_PLAN_FUSED_COMBINE
     o = B.moe_options()
     o.struct_bytes = ctypes.sizeof(B.moe_options)
