@@ -174,6 +174,24 @@ def test_large_batch_all_tokens():
     check(wl, inp, res, perm)
 
 
+@pytest.mark.parametrize("T,E,dtype,merged", [(65536, 8, "bf16", True), (65664, 8, "bf16", False),
+                                              (4096, 32, "f32", True), (4128, 32, "f32", False)])
+def test_routing_scan_in_permute_at_its_limit(T, E, dtype, merged):
+    """The permute does the routing scan while router blocks x experts stay
+    at most 4096 (bf16: 512 blocks of 128 tokens x 8 experts; fp32: 128
+    blocks of 32 tokens x 32 experts) and the scan kernel runs one block
+    later: both sides of the limit give every token's output, the counts
+    and the permutation of the oracle."""
+    from sparse_mixture_experts_renorm_b200 import launch_plan
+
+    wl = Workload(f"scan_limit_{T}_{E}_{dtype}", T=T, d=256 if dtype == "bf16" else 64, E=E, k=2,
+                  I=128 if dtype == "bf16" else 64, renorm=True, dtype=dtype)
+    plan = launch_plan(wl.T, wl.d, wl.E, wl.k, wl.I, wl.torch_dtype)
+    assert bool(plan & B.MOE_PLAN_PERMUTE_SCAN) == merged
+    inp, res, perm = run(wl, seed=14)
+    check(wl, inp, res, perm)
+
+
 def test_most_experts_with_many_tokens():
     """The largest expert count (256) and top-k (8) at 2048 tokens: 256 GEMM
     groups of about 64 rows, the router's shared-memory path and a scan over
