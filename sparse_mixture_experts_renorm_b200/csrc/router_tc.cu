@@ -99,6 +99,14 @@ __device__ __forceinline__ void st_cluster_f32(const void* local_in_leader_layou
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(addr) : "r"(smem_u32(local_in_leader_layout)), "r"(rank));
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
+// The same for four floats at a 16-byte aligned offset.
+__device__ __forceinline__ void st_cluster_v4(const void* local_in_leader_layout, uint32_t rank, float a, float b,
+                                              float c, float d) {
+  uint32_t addr;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(addr) : "r"(smem_u32(local_in_leader_layout)), "r"(rank));
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
 
 // Insert (v, e) into the list of the kMaxTopK best, kept sorted best first
 // (an element that ranks behind all of them leaves the list unchanged).
@@ -245,6 +253,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   pdl_wait();
 
   constexpr int kL = kE > 0 ? kE : 1;
+  float bias_pref = 0.f;  // b_r[r] for the leading CTA's epilogue thread r < E
   float lg[kL];    // this token's logits (register path)
   float ss = 0.f;  // this token's sum of x^2 (RMSNorm)
   if (warp == 0) {
@@ -315,6 +324,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     const int q = warp & 3;
     const int r = q * 32 + lane;
+    // the leading CTA's bias, read while the UMMAs run (E <= kRegE: one
+    // expert per thread of the first quarter)
+    if (kE > 0 && rank == 0 && br && r < E) bias_pref = br[r];
     // ------------- RMSNorm: this token's sum of x^2 over this CTA's K slice --
     // Row r of a 128B-swizzled x tile holds its 16-byte chunk c at position
     // c ^ (r & 7); each stage is summed on its own, then added to the total.
@@ -383,7 +395,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     if (S > 1 && rank > 0) {  // this CTA's share of the K loop goes to the leader
       float* dst = part + ((size_t)(rank - 1) * kRB + r) * E;
-      if (kE > 0) {
+      if (kE > 0 && (E & 3) == 0) {  // rows of E floats start on 16-byte boundaries
+#pragma unroll
+        for (int e = 0; e < kL; e += 4)
+          if (e < E) st_cluster_v4(dst + e, 0, lg[e], lg[e + 1], lg[e + 2], lg[e + 3]);
+      } else if (kE > 0) {
 #pragma unroll
         for (int e = 0; e < kL; ++e)
           if (e < E) st_cluster_f32(dst + e, 0, lg[e]);
@@ -412,8 +428,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       be[j] = 0x7fffffff;
     }
     bool finite = true;
-    if (br) {  // the bias once per block, then read from shared memory
-      for (int e = r; e < E; e += kRB) s_bias[e] = br[e];
+    if (br) {  // the bias once per block (read before the cluster barrier), then from shared memory
+      if (r < E) s_bias[r] = bias_pref;
       epi_bar();
     }
     // RMSNorm scale of this token (1 without the norm)
@@ -430,9 +446,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // bias, the maximum
       for (int s2 = 0; s2 < S - 1; ++s2) {
         const float* src = part + ((size_t)s2 * kRB + r) * E;
+        if ((E & 3) == 0) {
 #pragma unroll
-        for (int e = 0; e < kL; ++e)
-          if (e < E) lg[e] += src[e];
+          for (int e = 0; e < kL; e += 4)
+            if (e < E) {
+              const float4 p4 = *reinterpret_cast<const float4*>(src + e);
+              lg[e] += p4.x;
+              lg[e + 1] += p4.y;
+              lg[e + 2] += p4.z;
+              lg[e + 3] += p4.w;
+            }
+        } else {
+#pragma unroll
+          for (int e = 0; e < kL; ++e)
+            if (e < E) lg[e] += src[e];
+        }
       }
       // four independent chains (experts e mod 4) for the maximum and the sum
       float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -548,8 +576,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       blk_cnt[(size_t)blk * E + e] = run;
       float ps0 = 0.f, ps1 = 0.f, ps2 = 0.f, ps3 = 0.f;  // four chains over the block's tokens
+      // rows past the batch hold probability 0: stop at the last group of
+      // four that holds a token (the sums are the same)
+      const int nr4 = (min(kRB, T - tok0) + 3) & ~3;
 #pragma unroll 4
-      for (int rr = 0; rr < kRB; rr += 4) {
+      for (int rr = 0; rr < nr4; rr += 4) {
         ps0 += s_p[rr * ld + e];
         ps1 += s_p[(rr + 1) * ld + e];
         ps2 += s_p[(rr + 2) * ld + e];
