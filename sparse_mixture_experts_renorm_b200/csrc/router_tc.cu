@@ -815,7 +815,9 @@ cudaError_t launch_router_tc(const void* x, const void* w_router, const float* b
       !make_tmap_bf16_2d(&tmW, split ? norm.w_hi : w_router, (uint64_t)E, (uint64_t)d, (uint32_t)c.npad) ||
       !make_tmap_bf16_2d(&tmW2, split ? norm.w_lo : w_router, (uint64_t)E, (uint64_t)d, (uint32_t)c.npad))
     return cudaErrorInvalidValue;
-  auto kern = E <= kRegE ? router_tc_kernel<kRegE> : router_tc_kernel<0>;
+  // the register path unrolled for 8 or 16 experts: its code runs once per
+  // block, so the shorter body of the common E <= 8 spends less on fetching it
+  auto kern = E <= 8 ? router_tc_kernel<8> : E <= kRegE ? router_tc_kernel<kRegE> : router_tc_kernel<0>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, c.smem_bytes);
   if (err != cudaSuccess) return err;
   const int nb = (T + kRB - 1) / kRB;
