@@ -10,10 +10,11 @@
 // dimension of its own GEMM; 256-row tiles that run past the expert's last row
 // compute on neighbouring rows (or TMA zero fill) and are masked at the store.
 //
-// A cluster of two CTAs on two SMs owns one tile at a time. Each CTA stages
-// its own 128 rows of A and one half of the 256 B rows (mode 0: the 64 gate
-// rows and the 64 up rows of its 64 hidden units; mode 1: 128 W_down rows)
-// through a 5-stage TMA ring, both signalling the leading CTA's barrier. One
+// A cluster of two CTAs on two SMs owns one tile at a time. Weight-major
+// form: each CTA stages its own 128 weight rows as A (mode 0: the 64 gate rows
+// and the 64 up rows of its 64 hidden units; mode 1: 128 W_down rows) and one
+// half of the tile's token rows as B through a TMA ring (5 or 6 stages, 11
+// for the stream configuration), both signalling the leading CTA's barrier. One
 // thread of the leading CTA issues 256xNx16 UMMAs that read A and B from both
 // CTAs' shared memory and write each CTA's 128 rows of the fp32 accumulator
 // into that CTA's TMEM (double-buffered, 2 x 256 columns); commits are
@@ -23,14 +24,16 @@
 // Per UMMA FLOP this moves a third fewer bytes from L2 to shared memory than
 // one CTA per 128 x 256 tile.
 //
-// In the wide configuration the gate/up GEMM turns the tile around: the 256
-// token rows are the UMMA M operand (128 per CTA) and the block's 128 hidden
-// units the N operand, CTA 0 staging their 128 gate rows and CTA 1 their 128
-// up rows. Every TMEM lane then holds one token's gate values in columns
-// 0-127 and its up values in columns 128-255, so SwiGLU needs no exchange
-// between warps: the epilogue goes from TMEM to registers to its token's H row
-// and leaves shared memory to the TMA ring and the UMMAs. The operand bytes
-// per tile are the same as in the weight-major form.
+// Token-major form (the wide configuration's gate/up GEMM, and a down GEMM
+// whose grid has at most three tiles per CTA pair): the tile's 256 token rows
+// are the UMMA M operand (128 per CTA) and its weight rows the N operand. For
+// gate/up, CTA 0 stages the block's 128 gate rows and CTA 1 the same units'
+// 128 up rows, so every TMEM lane holds one token's gate values in columns
+// 0-127 and its up values in columns 128-255 and SwiGLU needs no exchange
+// between warps: the epilogue goes from TMEM to registers to its token's H
+// row and leaves shared memory to the TMA ring (6 stages) and the UMMAs. For
+// down, each lane holds one token's 256 outputs. The operand bytes per tile
+// are the same as in the weight-major form.
 //
 // Persistent: clusters walk a device-side tile list built from the routing
 // counts (experts in order; n-tile outer, m-tile inner inside an expert, so
@@ -48,9 +51,11 @@ namespace {
 constexpr int kHalfBytes = 128 * kBK * 2;          // 16 KB: 128 rows x 64 bf16
 constexpr int kSmallRows = 16;                     // B box for tiles of <= 32 tokens
 
-// Three configurations of the kernel. "Wide" tiles (many tokens per expert):
-// the epilogue is the long pole, so warps 2-9 drain the accumulator, two per
-// TMEM lane quarter taking alternate 32-token chunks, with a 5-stage ring.
+// Configurations of the kernel. "Wide" tiles (many tokens per expert): warps
+// 2-9 drain the accumulator, two per TMEM lane quarter taking alternate
+// 32-column chunks; token-major with a 6-stage ring and no epilogue staging
+// (WideTM), or weight-major with a 5-stage ring (Wide, the down GEMM with the
+// folded combine on longer grids).
 // "Narrow" tiles (decode-sized batches that stream the weights from HBM): a
 // deeper 6-stage ring keeps more bytes in flight and warps 2-5 drain it.
 // "Stream" (at most 32 tokens in the whole batch, so every tile's token rows
