@@ -265,7 +265,10 @@ __global__ void __launch_bounds__(kCopyThreads) permute_kernel(
 // Block (token t, chunk c): every thread sums one float4 of its token's k
 // expert rows, weighted by the gates, in slot order (fp32), skipping dropped
 // slots, then adds the token's rows of the shared experts in order.
-__global__ void __launch_bounds__(kCopyThreads) combine_kernel(const float4* __restrict__ y, int nvec4, int k, int R,
+// KM: the top-k rounded up to 2, 4, 6 or 8, so a thread holds only the rows
+// it can have (fewer registers, more resident blocks for the loads in flight).
+template <int KM>
+__global__ void __launch_bounds__(kCopyThreads, KM <= 6 ? 6 : 4) combine_kernel(const float4* __restrict__ y, int nvec4, int k, int R,
                                                               int T, const int32_t* __restrict__ inv,
                                                               const float* __restrict__ gate, int has_cap,
                                                               int n_shared, int shared_row0,
@@ -290,13 +293,13 @@ __global__ void __launch_bounds__(kCopyThreads) combine_kernel(const float4* __r
   __syncthreads();
   const int i = blockIdx.y * kCopyThreads + threadIdx.x;
   if (i >= nvec4) return;
-  float4 v[kMaxTopK];
+  float4 v[KM];
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j)
+  for (int j = 0; j < KM; ++j)
     if (j < k && s_rows[j] >= 0) v[j] = __ldg(y + (size_t)s_rows[j] * nvec4 + i);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) {
+  for (int j = 0; j < KM; ++j) {
     if (j < k && s_rows[j] >= 0) {
       const float g = s_g[j];
       acc.x = fmaf(g, v[j].x, acc.x);
@@ -362,7 +365,8 @@ cudaError_t launch_combine(int T, int d, int k, const float* y, const int32_t* i
                            cudaStream_t stream) {
   const int nvec4 = d / 4;
   const dim3 grid(T, (nvec4 + kCopyThreads - 1) / kCopyThreads);
-  return launch_pdl(combine_kernel, grid, dim3(kCopyThreads), 0, stream, reinterpret_cast<const float4*>(y), nvec4, k,
+  auto kern = k <= 2 ? combine_kernel<2> : k <= 4 ? combine_kernel<4> : k <= 6 ? combine_kernel<6> : combine_kernel<8>;
+  return launch_pdl(kern, grid, dim3(kCopyThreads), 0, stream, reinterpret_cast<const float4*>(y), nvec4, k,
                     T * k, T, inv, topk_gate, has_cap, n_shared, shared_row0, reinterpret_cast<float4*>(out), status);
 }
 
