@@ -192,6 +192,26 @@ def test_routing_scan_in_permute_at_its_limit(T, E, dtype, merged):
     check(wl, inp, res, perm)
 
 
+@pytest.mark.parametrize("T", [6016, 6144])
+def test_down_projection_forms_at_their_switch(T):
+    """The down GEMM (k = 2, combine folded in) runs token-major while its
+    grid has at most three tiles per CTA pair (6016 tokens: 220 tiles upper
+    bound on 148 SMs) and weight-major above (6144 tokens: 224): every token
+    of both compared with the oracle."""
+    wl = Workload(f"down_forms_{T}", T=T, d=1024, E=8, k=2, I=256, renorm=True, dtype="bf16")
+    inp, res, perm = run(wl, seed=15)
+    check(wl, inp, res, perm)
+
+
+@pytest.mark.parametrize("T", [255, 256])
+def test_gateup_forms_at_their_switch(T):
+    """The gate/up GEMM runs token-major once the batch averages 64 rows per
+    expert (R = 512 with E = 8) and weight-major (narrow) below."""
+    wl = Workload(f"gateup_forms_{T}", T=T, d=256, E=8, k=2, I=256, renorm=False, dtype="bf16")
+    inp, res, perm = run(wl, seed=16)
+    check(wl, inp, res, perm)
+
+
 def test_most_experts_with_many_tokens():
     """The largest expert count (256) and top-k (8) at 2048 tokens: 256 GEMM
     groups of about 64 rows, the router's shared-memory path and a scan over
