@@ -93,7 +93,8 @@ def plan_of(wl, opts=None):
 
     o = opts or {}
     return launch_plan(wl.T, wl.d, wl.E, wl.k, wl.I, wl.torch_dtype, n_shared=o.get("shared", 0),
-                       norm_form=o.get("norm", 0), norm_weight=bool(o.get("norm", 0)))
+                       norm_form=o.get("norm", 0), norm_weight=bool(o.get("norm", 0)),
+                       fold_combine=bool(o.get("fold_combine", False)))
 
 
 def algorithmic(wl, counts, opts=None):
@@ -653,6 +654,9 @@ def main():
     ap.add_argument("--shared", type=int, default=0, help="shared experts (each the routed experts' shape)")
     ap.add_argument("--capacity", type=float, default=0.0, help="capacity factor (0: no dropping)")
     ap.add_argument("--zloss", action="store_true", help="also compute the router z-loss statistic")
+    ap.add_argument("--fold-combine", action="store_true",
+                    help="fold the combine into the down GEMM for every top-k (atomic adds: not bit-reproducible "
+                         "for k > 2)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     headline = args.workload or "mixtral_prefill"
@@ -673,15 +677,17 @@ def main():
 
     opts = {}
     options = None
-    if args.norm or args.shared or args.capacity > 0 or args.zloss:
+    if args.norm or args.shared or args.capacity > 0 or args.zloss or args.fold_combine:
         from sparse_mixture_experts_renorm_b200 import MoEOptions
         from sparse_mixture_experts_renorm_b200.workloads import make_option_inputs
 
         oi = make_option_inputs(wl, dev, seed=0, n_shared=args.shared, norm_weight=bool(args.norm))
         options = MoEOptions(norm_form=args.norm, norm_eps=1e-5, norm_weight=oi.norm_weight,
                              shared_gate=oi.shared_gate, shared_up=oi.shared_up, shared_down=oi.shared_down,
-                             capacity_factor=args.capacity, z_loss=args.zloss)
+                             capacity_factor=args.capacity, z_loss=args.zloss, fold_combine=args.fold_combine)
         opts = {"norm": args.norm, "shared": args.shared, "capacity_factor": args.capacity, "z_loss": args.zloss}
+        if args.fold_combine:
+            opts["fold_combine"] = True
         if args.capacity > 0:
             import math
 

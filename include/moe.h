@@ -181,6 +181,16 @@ moe_status moe_get_permutation(const void* workspace, size_t workspace_bytes, in
  *
  * Router z-loss (the ST-MoE statistic of "moe_router_z_loss_weight"):
  *   z = (1/T) sum_t ( log sum_e exp(logit[t,e]) )^2, logits with their bias.
+ *
+ * Folded combine (no counterpart on the pages): on the bf16 path with k = 2
+ * and no shared experts the down GEMM's epilogue adds gate * y of every
+ * expert row into the zeroed fp32 output with atomic adds instead of storing
+ * Y for a combine kernel; two additions into zero commute, so that result is
+ * bit-identical from run to run. fold_combine != 0 does the same for every
+ * k (still bf16, no shared experts): no Y rows are written or read back, but
+ * with k > 2 the order of a token's additions varies between runs, so the
+ * output equals the combine kernel's up to fp32 rounding and is not
+ * bit-reproducible. Off by default.
  */
 typedef enum {
   MOE_NORM_NONE = 0,
@@ -202,6 +212,7 @@ typedef struct moe_options {
   double capacity_factor;    /* 0: no dropping; > 0 and finite: the cap above */
   int32_t* dropped;          /* device, [1] int32, or NULL: assignments dropped */
   float* z_loss;             /* device, [1] fp32, or NULL: the z-loss statistic */
+  int fold_combine;          /* nonzero: fold the combine into the down GEMM for every k (above) */
 } moe_options;
 
 /*
@@ -235,7 +246,8 @@ moe_status moe_forward_ex(const void* x, const void* w_router, const float* b_ro
  * (NULL: none) launches, as a bit set; -1 if the arguments are invalid (see
  * moe_last_error_detail). Host only; launches nothing.
  *   MOE_PLAN_FUSED_COMBINE: the combine runs in the down GEMM's epilogue
- *     (bf16, k = 2, no shared experts): kernel 5 is not launched.
+ *     (bf16, no shared experts, k = 2 or fold_combine set): kernel 5 is not
+ *     launched.
  *   MOE_PLAN_FUSED_GEMMS: both projections run in one persistent kernel
  *     (bf16, 1 <= T <= 32, where the GEMMs stream the weights from HBM):
  *     slot 3 times both, slot 4 is empty.

@@ -41,7 +41,9 @@ class MoEOptions:
     form w*x/(sqrt(mean x^2) + eps); norm_weight: [d] in the layer dtype or
     None for ones. shared_*: weights of the shared experts ([S, I, d],
     [S, I, d], [S, d, I]) or None. capacity_factor: 0 = no dropping.
-    z_loss: also compute the router z-loss statistic."""
+    z_loss: also compute the router z-loss statistic. fold_combine: fold the
+    combine into the down GEMM for every top-k (atomic fp32 adds: with k > 2
+    the result is not bit-reproducible between runs; k = 2 always folds)."""
     norm_form: int = 0
     norm_eps: float = 1e-5
     norm_weight: torch.Tensor | None = None
@@ -50,6 +52,7 @@ class MoEOptions:
     shared_down: torch.Tensor | None = None
     capacity_factor: float = 0.0
     z_loss: bool = False
+    fold_combine: bool = False
 
     @property
     def n_shared(self) -> int:
@@ -69,6 +72,7 @@ class MoEOptions:
         o.capacity_factor = float(self.capacity_factor)
         o.dropped = None if dropped is None else dropped.data_ptr()
         o.z_loss = None if z_loss is None else z_loss.data_ptr()
+        o.fold_combine = 1 if self.fold_combine else 0
         return o
 
 
@@ -86,7 +90,7 @@ def workspace_size(T: int, d: int, E: int, k: int, I: int, dtype: torch.dtype,
 
 
 def launch_plan(T: int, d: int, E: int, k: int, I: int, dtype: torch.dtype, n_shared: int = 0,
-                norm_form: int = 0, norm_weight: bool = False) -> int:
+                norm_form: int = 0, norm_weight: bool = False, fold_combine: bool = False) -> int:
     """The library's launch plan for a call of this shape (``moe_launch_plan``:
     MOE_PLAN_* bits saying which kernels are merged). A host-side query: the
     weight pointers it passes are placeholders that nothing dereferences."""
@@ -99,6 +103,7 @@ def launch_plan(T: int, d: int, E: int, k: int, I: int, dtype: torch.dtype, n_sh
     o.n_shared = int(n_shared)
     if n_shared:
         o.shared_gate = o.shared_up = o.shared_down = 256
+    o.fold_combine = 1 if fold_combine else 0
     plan = lib.moe_launch_plan(T, d, E, k, I, _dtype_code(dtype), ctypes.byref(o))
     if plan < 0:
         raise MoEError(B.MOE_ERR_INVALID_ARG, B.last_error_detail(lib))

@@ -52,6 +52,7 @@ class moe_options(ctypes.Structure):
         ("capacity_factor", ctypes.c_double),
         ("dropped", ctypes.c_void_p),
         ("z_loss", ctypes.c_void_p),
+        ("fold_combine", ctypes.c_int),
     ]
 
 

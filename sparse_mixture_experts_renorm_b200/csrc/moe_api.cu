@@ -151,6 +151,7 @@ struct Opts {
   double cf = 0.0;
   int32_t* dropped = nullptr;
   float* zloss = nullptr;
+  bool fold_combine = false;
 };
 
 moe_status parse_options(const moe_options* opt, int T, int d, int k, int I, Opts* o) {
@@ -187,7 +188,17 @@ moe_status parse_options(const moe_options* opt, int T, int d, int k, int I, Opt
   o->cf = opt->capacity_factor;
   o->dropped = opt->dropped;
   o->zloss = opt->z_loss;
+  o->fold_combine = opt->fold_combine != 0;
   return MOE_OK;
+}
+
+// The combine runs in the down GEMM's epilogue as fp32 atomic adds into the
+// zeroed output (bf16 path, no shared experts, whose rows the combine kernel
+// adds): always for k = 2, where the two additions into zero commute and the
+// result is deterministic, and for every k when the caller allows the
+// run-to-run order of the additions (fold_combine).
+bool combine_folded(moe_dtype dtype, int k, const Opts& o) {
+  return dtype == MOE_BF16 && o.n_shared == 0 && (k == 2 || o.fold_combine);
 }
 
 // Assignments an expert keeps: ceil(cf * T * k / E), clamped to T (an expert
@@ -346,9 +357,9 @@ moe_status forward_impl(const void* x, const void* w_router, const float* b_rout
   marks.mark(stream);
   // With k = 2 (and no shared experts) the bf16 path folds the combine into
   // the down GEMM's epilogue (two fp32 adds into a zeroed row commute, so the
-  // result stays deterministic); otherwise a separate combine kernel sums the
-  // rows in a fixed order.
-  const bool fused_combine = dtype == MOE_BF16 && k == 2 && o.n_shared == 0;
+  // result stays deterministic), and for any k with fold_combine; otherwise a
+  // separate combine kernel sums the rows in a fixed order.
+  const bool fused_combine = combine_folded(dtype, k, o);
   {
     NvtxRange r("permute");
     err = launch_permute(dtype, x, T, d, E, k, router_block_tokens(dtype), topk_idx, lrank, blk_cnt, offsets,
@@ -514,7 +525,7 @@ int moe_launch_plan(int T, int d, int E, int k, int I, moe_dtype dtype, const mo
   Opts o;
   if (parse_options(opt, T, d, k, I, &o) != MOE_OK) return -1;
   int plan = 0;
-  if (dtype == MOE_BF16 && k == 2 && o.n_shared == 0) plan |= MOE_PLAN_FUSED_COMBINE;
+  if (combine_folded(dtype, k, o)) plan |= MOE_PLAN_FUSED_COMBINE;
   if (gemms_fused(T, dtype)) plan |= MOE_PLAN_FUSED_GEMMS;
   if (router_does_scan(T, E, dtype))
     plan |= MOE_PLAN_FUSED_SCAN;

@@ -221,6 +221,18 @@ def test_launch_plan(lib):
                                                                            | B.MOE_PLAN_ROUTER_WEIGHT_SPLIT
                                                                            | B.MOE_PLAN_FUSED_SCAN)
     assert lib.moe_launch_plan(32, 4096, 8, 9, 14336, bf, None) == -1  # k > E
+    # fold_combine: the combine in the down GEMM for every k (bf16, no shared experts)
+    f = B.moe_options()
+    f.struct_bytes = ctypes.sizeof(B.moe_options)
+    f.fold_combine = 1
+    assert lib.moe_launch_plan(16384, 2048, 64, 6, 1408, bf, ctypes.byref(f)) == B.MOE_PLAN_FUSED_COMBINE
+    assert lib.moe_launch_plan(32, 4096, 8, 1, 14336, bf, ctypes.byref(f)) == (B.MOE_PLAN_FUSED_COMBINE
+                                                                           | B.MOE_PLAN_FUSED_GEMMS
+                                                                           | B.MOE_PLAN_FUSED_SCAN)
+    assert lib.moe_launch_plan(64, 128, 4, 3, 256, f32, ctypes.byref(f)) == B.MOE_PLAN_PERMUTE_SCAN
+    f.n_shared = 1
+    f.shared_gate = f.shared_up = f.shared_down = 256
+    assert lib.moe_launch_plan(16384, 2048, 64, 6, 1408, bf, ctypes.byref(f)) == 0
 
 
 def test_pipeline_rejects_bad_arguments_before_any_cuda_call(lib):

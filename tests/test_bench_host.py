@@ -13,6 +13,7 @@ sys.path.insert(0, ROOT)
 
 import bench  # noqa: E402
 from sparse_mixture_experts_renorm_b200 import build as build_mod  # noqa: E402
+from sparse_mixture_experts_renorm_b200 import _binding as B  # noqa: E402
 from sparse_mixture_experts_renorm_b200.workloads import WORKLOADS  # noqa: E402
 
 
@@ -78,6 +79,15 @@ def test_fused_combine_rule():
     assert not bench.fused_combine(WORKLOADS["mixtral_prefill"], n_shared=1)
     assert not bench.fused_combine(WORKLOADS["fine_grained"])  # k = 6
     assert not bench.fused_combine(WORKLOADS["tiny_f32"])  # fp32 path
+    # the fold_combine option: every k, the down GEMM's slot carrying the combine
+    fine, fold = WORKLOADS["fine_grained"], {"fold_combine": True}
+    assert bench.plan_of(fine, fold) & B.MOE_PLAN_FUSED_COMBINE
+    assert bench.launches_per_step(fine, fold) == 5
+    assert bench.slot_names(fine, fold)[5] == "combine (in grouped_gemm_down)"
+    w = bench.algorithmic(fine, balanced(fine), fold)
+    R = fine.T * fine.k
+    assert w["combine"]["bytes"] == 0
+    assert w["grouped_gemm_down"]["bytes"] == (64 * 2048 * 1408 * 2 + R * 1408 * 2 + 2 * fine.T * 2048 * 4 + R * 8)
 
 
 def test_fused_gemms_rule():

@@ -130,6 +130,49 @@ def test_full_size_with_all_options(name):
     assert np.isfinite(rep["max_abs"])
 
 
+# fold_combine: the combine done by the down GEMM's epilogue for every top-k
+# (fp32 atomic adds into the zeroed output): the same parity bars, and at full
+# size the output of the combine kernel up to the order of a token's adds.
+FOLD_CASES = [
+    (Workload("bf16_fold_k6_E64", T=700, d=256, E=64, k=6, I=128, renorm=False, dtype="bf16", router_std=0.1,
+              zipf_bias=True), 0.0),
+    (Workload("bf16_fold_k3_capacity", T=333, d=128, E=6, k=3, I=192, renorm=True, dtype="bf16", router_std=0.1,
+              zipf_bias=True), 0.5),
+    (Workload("bf16_fold_k1", T=200, d=128, E=4, k=1, I=256, renorm=True, dtype="bf16", router_std=0.3), 0.0),
+    (Workload("bf16_fold_k4_decode", T=24, d=256, E=8, k=4, I=256, renorm=True, dtype="bf16", router_std=0.3), 0.0),
+]
+
+
+@pytest.mark.parametrize("case", FOLD_CASES, ids=[c[0].name for c in FOLD_CASES])
+def test_fold_combine_parity(case):
+    wl, cf = case
+    opts = MoEOptions(capacity_factor=cf, fold_combine=True)
+    inp, res, perm = run(wl, opts)
+    rep = parity.check(inp, res, perm, wl.k, wl.renorm, wl.dtype, options=opts)
+    print(f"\n[{wl.name}] {rep}")
+    if cf > 0:
+        assert rep["dropped"] > 0, "the capacity case should drop assignments"
+
+
+def test_fold_combine_full_size_matches_the_combine_kernel():
+    """fine_grained (k = 6) with the folded combine against the default
+    path on the same inputs: identical routing and dispatch, and outputs
+    equal up to fp32 rounding of a different order of six additions."""
+    wl = WORKLOADS["fine_grained"]
+    inp = make_inputs(wl, "cuda", 0)
+    a = moe_forward(inp.x, inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k, wl.renorm)
+    b = moe_forward(inp.x, inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k, wl.renorm,
+                    options=MoEOptions(fold_combine=True))
+    torch.cuda.synchronize()
+    assert int(a.status.item()) == 0 and int(b.status.item()) == 0
+    assert torch.equal(a.topk_idx, b.topk_idx) and torch.equal(a.topk_gate, b.topk_gate)
+    assert torch.equal(a.counts, b.counts)
+    scale = a.out.abs().max().item()
+    diff = (a.out - b.out).abs().max().item()
+    print(f"\n[fine_grained fold] max |out| {scale:.4g}, max-abs difference {diff:.3g}")
+    assert diff <= 1e-5 * scale
+
+
 def test_host_pipeline_with_options_matches_device_calls():
     """The library's host-memory pipeline carries the options (a copy taken
     at creation): every batch's output and statistic equal those of a plain
