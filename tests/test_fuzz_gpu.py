@@ -3,7 +3,9 @@ router bias and the layer's options drawn together, so that combinations the
 hand-picked cases do not name (an odd expert count with the norm and a
 capacity, k = E with shared experts, a ragged tail in every GEMM tile) are
 compared with the fp64 oracle too. The draws are fixed by one numpy seed;
-every case is run through the C ABI exactly like the named cases."""
+every case is run through the C ABI exactly like the named cases. Every
+even-numbered case also sets fold_combine (the combine in the down GEMM's
+epilogue for every top-k), so both combine paths meet the random shapes."""
 import numpy as np
 import pytest
 import torch
@@ -47,10 +49,15 @@ def draw_cases(n=N_CASES, seed=2024):
 CASES = draw_cases()
 
 
+def folds(wl) -> bool:
+    """Even-numbered cases run with fold_combine (the draws stay the same)."""
+    return int(wl.name[2:]) % 2 == 0
+
+
 def case_id(c):
     wl, form, nw, ns, cf, z = c
     opts = "".join([f"n{form}" if form else "", "w" if nw else "", f"s{ns}" if ns else "",
-                    f"c{cf:.2f}" if cf else "", "z" if z else ""])
+                    f"c{cf:.2f}" if cf else "", "z" if z else "", "f" if folds(wl) else ""])
     return (f"{wl.name}-{wl.dtype}-T{wl.T}-d{wl.d}-E{wl.E}-k{wl.k}-I{wl.I}-{'r' if wl.renorm else 'nr'}"
             + (f"-{opts}" if opts else ""))
 
@@ -66,6 +73,8 @@ def test_draws_cover_the_options_and_shapes():
     assert any(w.T <= 32 and w.dtype == "bf16" for w in wls)
     assert any(c[1] == 1 for c in CASES) and any(c[1] == 2 for c in CASES)
     assert any(c[3] for c in CASES) and any(c[4] for c in CASES) and any(c[5] for c in CASES)
+    # the folded combine on the bf16 path with k != 2 and no shared experts, where it changes the plan
+    assert any(folds(c[0]) and c[0].dtype == "bf16" and c[0].k != 2 and not c[3] for c in CASES)
 
 
 @pytest.mark.gpu
@@ -74,10 +83,11 @@ def test_random_shape_parity(case):
     wl, form, nw, ns, cf, z = case
     inp = make_inputs(wl, "cuda", 17)
     opts = None
-    if form or ns or cf or z:
+    if form or ns or cf or z or folds(wl):
         oi = make_option_inputs(wl, "cuda", 17, n_shared=ns, norm_weight=nw)
         opts = MoEOptions(norm_form=form, norm_eps=1e-5, norm_weight=oi.norm_weight, shared_gate=oi.shared_gate,
-                          shared_up=oi.shared_up, shared_down=oi.shared_down, capacity_factor=cf, z_loss=z)
+                          shared_up=oi.shared_up, shared_down=oi.shared_down, capacity_factor=cf, z_loss=z,
+                          fold_combine=folds(wl))
     res = moe_forward(inp.x, inp.w_router, inp.b_router, inp.w_gate, inp.w_up, inp.w_down, wl.k, wl.renorm,
                       options=opts)
     torch.cuda.synchronize()
