@@ -255,3 +255,30 @@ def test_pipeline_rejects_bad_arguments_before_any_cuda_call(lib):
     assert h.value is None
     assert lib.moe_pipeline_destroy(None) == B.MOE_OK
     assert lib.moe_pipeline_stream(None, 0) is None
+
+
+def _c_layout(struct, fields, tmp_path):
+    """sizeof and offsetof of `fields` of `struct` as gcc lays out the
+    declarations of include/moe.h (a host program compiled for this test)."""
+    import subprocess
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    lines = [f'printf("%zu\\n", sizeof({struct}));'] + [f'printf("%zu\\n", offsetof({struct}, {f}));' for f in fields]
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"moe.h\"\nint main(void) {\n"
+                   + "\n".join(lines) + "\nreturn 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(root, "include"), str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    return int(out[0]), [int(v) for v in out[1:]]
+
+
+@pytest.mark.parametrize("cls,struct", [(B.moe_options, "moe_options"), (B.moe_layer_desc, "moe_layer_desc")])
+def test_ctypes_structs_match_the_header(cls, struct, tmp_path):
+    """The binding's ctypes mirrors of the option and pipeline structs have
+    the header's size and field offsets (a field added on one side only
+    would shift every later field)."""
+    names = [f[0] for f in cls._fields_]
+    size, offsets = _c_layout(struct, names, tmp_path)
+    assert ctypes.sizeof(cls) == size
+    assert [getattr(cls, n).offset for n in names] == offsets
